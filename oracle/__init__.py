@@ -1,0 +1,24 @@
+"""CPU oracle for the LatentIndex decode indexer.
+
+TEST INFRASTRUCTURE.  This package is the plain, slow, obviously correct
+statement of what the indexer computes: NumPy float64 (BLAS for the matrix
+products), a pure-Python brute force for tiny inputs, the cache element codecs
+written from their format definitions, and the closed-form counters printed in
+the LatentIndex summary.  Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import it.  The library never calls
+it and shares no code with it: the CUDA path must fail loudly when its
+extension is missing instead of falling back here.
+
+Pins (tests/test_oracle.py): a hand-computed worked example
+(tests/golden/hand_example.json), the storage and positions-scored numbers
+printed in the summary (tests/golden/printed_numbers.json), an independent
+pure-Python brute force that reconstructs every key explicitly, the method's
+invariants (absorption exactness, HS with B >= L equals full selection, a
+one-layer group with an identity decoder is DSA-style scoring), and the
+codecs against torch's bf16 / float8_e4m3fn conversions.  The pages print no
+score values of their own, so the score arithmetic is pinned by hand
+arithmetic and brute force rather than by a published example.
+"""
+from . import codecs, counters, indexer, bruteforce
+
+__all__ = ["codecs", "counters", "indexer", "bruteforce"]

@@ -1,0 +1,79 @@
+"""The pins must catch a plausible mistake in the oracle: each case plants one
+mistake (in the oracle, on the CPU) and checks that some pin then fails."""
+import numpy as np
+import pytest
+
+import oracle.indexer as ix
+from tests import test_oracle as pins
+
+
+def _dropped_relu(c_rows, qt, w, beta=None):
+    pre = np.asarray(c_rows, float) @ np.asarray(qt, float).T
+    if beta is not None:
+        pre = pre + beta
+    return pre @ np.asarray(w, float)
+
+
+def _relu_after_weight(c_rows, qt, w, beta=None):
+    pre = np.asarray(c_rows, float) @ np.asarray(qt, float).T
+    if beta is not None:
+        pre = pre + beta
+    return np.maximum(pre * np.asarray(w, float), 0).sum(axis=1)
+
+
+def _absorb_wrong_operand(q, W_K, b_K=None):
+    q = np.asarray(q, float)
+    W = np.asarray(W_K, float)
+    # a plausible slip: use the decoder's rows as the absorbed query directly
+    qt = np.einsum("...hk,kc->...hc", q, np.abs(W))
+    beta = None if b_K is None else np.einsum("...hk,k->...h", q, np.asarray(b_K, float))
+    return qt, beta
+
+
+def _topk_high_index_ties(scores, k, n=None):
+    s = np.asarray(scores)[: (len(scores) if n is None else n)]
+    n = len(s)
+    keff = min(k, n)
+    order = np.lexsort((-np.arange(n), -s.astype(float)))
+    sel = np.sort(order[:keff])
+    idx = np.full(k, -1, np.int32)
+    idx[:keff] = sel
+    vals = np.full(k, -np.inf)
+    vals[:keff] = s[sel]
+    return idx, vals
+
+
+def _topk_unsorted_output(scores, k, n=None):
+    s = np.asarray(scores)[: (len(scores) if n is None else n)]
+    n = len(s)
+    keff = min(k, n)
+    order = np.lexsort((np.arange(n), -s.astype(float)))[:keff]
+    idx = np.full(k, -1, np.int32)
+    idx[:keff] = order
+    vals = np.full(k, -np.inf)
+    vals[:keff] = s[order]
+    return idx, vals
+
+
+PIN_SETS = [pins.test_hand_example_scores_and_selection, pins.test_hand_example_hs,
+            pins.test_hand_example_bias,
+            lambda: pins.test_absorbed_scoring_equals_explicit_keys(0),
+            lambda: pins.test_topk_matches_sorted(5)]
+
+
+@pytest.mark.parametrize("name,attr,bad", [
+    ("dropped ReLU", "score", _dropped_relu),
+    ("ReLU after weighting", "score", _relu_after_weight),
+    ("wrong absorbed operand", "absorb", _absorb_wrong_operand),
+    ("ties to the higher index", "topk", _topk_high_index_ties),
+    ("selection not in position order", "topk", _topk_unsorted_output),
+])
+def test_planted_mistake_is_caught(monkeypatch, name, attr, bad):
+    monkeypatch.setattr(ix, attr, bad)
+    failures = 0
+    for pin in PIN_SETS:
+        try:
+            pin()
+        except AssertionError:
+            failures += 1
+    assert failures > 0, f"no pin caught: {name}"

@@ -1,0 +1,139 @@
+"""Seeded synthetic inputs for the indexer workloads.
+
+Both the CUDA path (through the tests and the bench) and the CPU oracle read
+their inputs from here, so this module does data synthesis only: Gaussian
+draws, a rank-one "affinity" spike that makes a few tokens score high, and the
+outlier channel of the fp8 workload.  It performs no scoring, absorption,
+quantisation or selection.
+
+Recipe (all draws from ``numpy.random.default_rng(seed)``, float32):
+
+* sigma_c = 1/sqrt(d_model): the spread a latent c = W_down h has when h and
+  W_down are N(0, 1/sqrt(d_model)) (std).  Workloads with
+  ``latent_from_hidden`` draw h [b, cap, d_model] and W_down [d_c, d_model]
+  instead and let the append step build c.
+* Decoders W_K[l] = (G_l + sqrt(d_c) * v_l u^T) / sqrt(d_k), G_l ~ N(0, 1):
+  Gaussian plus a rank-one spike that maps the latent direction u onto the
+  key direction v_l.
+* Head weights w[l] ~ N(0, 1/sqrt(H)) (std); queries
+  q[l] = (g + 2 sign(w[l]) v_l) / sqrt(d_k), g ~ N(0, 1), so heads with
+  positive weight lean toward +v_l and heads with negative weight toward -v_l.
+* Planted tokens: ceil(p * len) positions per sequence, sampled without
+  replacement, get c += 3 sigma_c sqrt(d_c) u (or h += 3 sigma_h sqrt(d_model)
+  * unit(W_down^T u) when the latent is built from h).
+* Outlier channels: ``outlier_channels`` latent channels, chosen by the seed,
+  are multiplied by ``outlier_mult`` for every token (before any quantisation).
+* Ragged lengths: integers uniform in ``length_range`` (inclusive).
+* Prefill queries sit at the last ``queries`` positions of each sequence.
+"""
+from dataclasses import dataclass, replace
+import math
+from typing import List, Optional
+
+import numpy as np
+
+from .configs import Workload, workload
+
+
+@dataclass
+class Inputs:
+    wl: Workload
+    lengths: np.ndarray            # int32 [b]
+    latent: Optional[np.ndarray]   # float32 [b, cap, d_c] (None when built from h)
+    hidden: Optional[np.ndarray]   # float32 [b, cap, d_model] (latent_from_hidden only)
+    W_down: Optional[np.ndarray]   # float32 [d_c, d_model]
+    W_K: List[np.ndarray]          # per layer float32 [d_k, d_c]
+    q: List[np.ndarray]            # per layer float32 [b, T, H, d_k]
+    w: List[np.ndarray]            # per layer float32 [b, T, H]
+    q_pos: Optional[np.ndarray]    # int32 [b, T] for prefill, None for decode
+    planted: List[np.ndarray]      # per sequence int64 positions
+    outlier_channels: np.ndarray   # int64 channel ids
+
+
+def shrunk(wl: Workload, capacity: int, batch: Optional[int] = None,
+           length_range=None, queries: Optional[int] = None) -> Workload:
+    """Same distributions, smaller sizes (for oracle-sized parity cases)."""
+    lr = length_range if length_range is not None else (
+        (capacity, capacity) if wl.length_range[0] == wl.length_range[1]
+        else (max(1, capacity // 2), capacity))
+    return replace(wl, capacity=capacity, batch=batch or wl.batch, length_range=lr,
+                   queries=queries or wl.queries,
+                   k=min(wl.k, capacity), B=None if wl.B is None else min(wl.B, capacity))
+
+
+def _unit(x: np.ndarray) -> np.ndarray:
+    return (x / np.linalg.norm(x)).astype(np.float32)
+
+
+def generate(wl, seed: Optional[int] = None) -> Inputs:
+    if isinstance(wl, int):
+        wl = workload(wl)
+    rng = np.random.default_rng(wl.seed if seed is None else seed)
+    b, cap, G, H, dk, dc, T = wl.batch, wl.capacity, wl.group, wl.heads, wl.d_k, wl.d_c, wl.queries
+    lo, hi = wl.length_range
+    if lo == hi:
+        lengths = np.full(b, lo, dtype=np.int32)
+    else:
+        lengths = rng.integers(lo, hi + 1, size=b).astype(np.int32)
+
+    u = _unit(rng.standard_normal(dc, dtype=np.float32))
+    W_K, q, w = [], [], []
+    for _ in range(G):
+        v = _unit(rng.standard_normal(dk, dtype=np.float32))
+        Gl = rng.standard_normal((dk, dc), dtype=np.float32)
+        W_K.append(((Gl + math.sqrt(dc) * np.outer(v, u)) / math.sqrt(dk)).astype(np.float32))
+        wl_ = (rng.standard_normal((b, T, H), dtype=np.float32) / math.sqrt(H)).astype(np.float32)
+        g = rng.standard_normal((b, T, H, dk), dtype=np.float32)
+        ql = (g + 2.0 * np.sign(wl_)[..., None] * v) / math.sqrt(dk)
+        q.append(ql.astype(np.float32))
+        w.append(wl_)
+
+    planted = []
+    for i in range(b):
+        n_p = int(math.ceil(wl.planted_frac * int(lengths[i])))
+        planted.append(np.sort(rng.choice(int(lengths[i]), size=n_p, replace=False)) if n_p else
+                       np.zeros(0, dtype=np.int64))
+
+    hidden = W_down = latent = None
+    if wl.latent_from_hidden:
+        dm = wl.d_model
+        s = 1.0 / math.sqrt(dm)
+        W_down = (rng.standard_normal((dc, dm), dtype=np.float32) * s).astype(np.float32)
+        hidden = (rng.standard_normal((b, cap, dm), dtype=np.float32) * s).astype(np.float32)
+        # unit(W_down^T u): the hidden-space direction that W_down maps closest to u.
+        dirn = _unit(W_down.T.astype(np.float64) @ u.astype(np.float64))
+        for i in range(b):
+            hidden[i, planted[i], :] += np.float32(3.0 * s * math.sqrt(dm)) * dirn
+    else:
+        s = 1.0 / math.sqrt(wl.d_model)
+        latent = rng.standard_normal((b, cap, dc), dtype=np.float32)
+        latent *= np.float32(s)
+        for i in range(b):
+            latent[i, planted[i], :] += np.float32(3.0 * s * math.sqrt(dc)) * u
+
+    outl = np.sort(rng.choice(dc, size=wl.outlier_channels, replace=False)) if wl.outlier_channels \
+        else np.zeros(0, dtype=np.int64)
+    if len(outl):
+        if latent is not None:
+            latent[:, :, outl] *= np.float32(wl.outlier_mult)
+        # (workloads built from h carry no outlier channels)
+
+    q_pos = None
+    if T > 1:
+        q_pos = np.stack([np.arange(int(L) - T, int(L), dtype=np.int32) for L in lengths])
+    return Inputs(wl=wl, lengths=lengths, latent=latent, hidden=hidden, W_down=W_down,
+                  W_K=W_K, q=q, w=w, q_pos=q_pos, planted=planted, outlier_channels=outl)
+
+
+def construction_inputs(wl: Workload, seed: Optional[int] = None):
+    """Weights and one new hidden state per sequence for the per-step key /
+    latent construction (decode step "with construction"): h_new [b, 1, d_model],
+    W_down [d_c, d_model] and one DSA key projection W_k[l] [d_k, d_model] per
+    layer, all N(0, 1/sqrt(d_model)) (std)."""
+    rng = np.random.default_rng((wl.seed if seed is None else seed) + 1000)
+    s = 1.0 / math.sqrt(wl.d_model)
+    h_new = (rng.standard_normal((wl.batch, 1, wl.d_model), dtype=np.float32) * s)
+    W_down = (rng.standard_normal((wl.d_c, wl.d_model), dtype=np.float32) * s)
+    W_k = [(rng.standard_normal((wl.d_k, wl.d_model), dtype=np.float32) * s)
+           for _ in range(wl.group)]
+    return h_new.astype(np.float32), W_down.astype(np.float32), [x.astype(np.float32) for x in W_k]
