@@ -1,0 +1,706 @@
+// api.cu -- the extern "C" entry points declared in include/li.h: argument
+// validation, workspace layout, TMA descriptor encoding and the launch
+// sequence of every operation.  Host state lives in li_ctx; the library
+// allocates no device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+using namespace li;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct ProfRec {
+  std::string name;
+  cudaEvent_t beg, end;
+  int grid, block, smem;
+};
+
+struct li_ctx {
+  int device = 0;
+  int num_sms = 0;
+  int max_smem_optin = 0;
+  EncodeTiledFn encode = nullptr;
+  std::string last_error;
+  uint64_t wait_ns = 2000000000ull;
+  bool profile = false;
+  std::vector<ProfRec> prof;
+  std::vector<cudaEvent_t> free_events;
+};
+
+namespace {
+
+li_status fail(li_ctx* ctx, li_status s, const char* fmt, ...) {
+  if (ctx) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    ctx->last_error = buf;
+  }
+  return s;
+}
+
+li_status cuda_fail(li_ctx* ctx, cudaError_t e, const char* what) {
+  return fail(ctx, LI_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elt_bytes(li_dtype d) { return d == LI_F32 ? 4 : (d == LI_BF16 ? 2 : 1); }
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ------------------------------------------------------------------ workspace
+
+struct WsLayout {
+  size_t status = 0, done = 64, hist, rowinfo, chunk_gt, chunk_off, cand, scores, cand_scores, tmp, total;
+  int n_chunks;
+};
+
+constexpr int kAppendChunkTok = 8192;
+
+WsLayout ws_layout(int64_t rows, int64_t n, int64_t B) {
+  WsLayout L;
+  size_t off = 256;
+  auto take = [&](size_t bytes) { size_t o = off; off += up256(bytes); return o; };
+  const int64_t nn = std::max<int64_t>(std::max<int64_t>(n, B), 1);
+  L.n_chunks = static_cast<int>((nn + kTopkChunk - 1) / kTopkChunk);
+  L.hist = take(rows * kHistBins * 4);
+  L.rowinfo = take(rows * 16 * 4);
+  L.chunk_gt = take(rows * L.n_chunks * 4);
+  L.chunk_off = take(rows * L.n_chunks * 4);
+  L.cand = take(rows * nn * 8);
+  L.scores = take(rows * nn * 4);
+  L.cand_scores = take(rows * std::max<int64_t>(B, 1) * 4);
+  L.tmp = take(static_cast<size_t>(kAppendChunkTok) * 256 * 4);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off); }
+
+// ------------------------------------------------------------------ profiling
+
+cudaEvent_t get_event(li_ctx* c) {
+  if (!c->free_events.empty()) {
+    cudaEvent_t e = c->free_events.back();
+    c->free_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct Launch {
+  li_ctx* c;
+  cudaStream_t st;
+  const char* name;
+  int grid, block, smem;
+  cudaEvent_t beg = nullptr;
+  Launch(li_ctx* c_, cudaStream_t st_, const char* name_, int grid_, int block_, int smem_)
+      : c(c_), st(st_), name(name_), grid(grid_), block(block_), smem(smem_) {
+    if (c->profile) {
+      beg = get_event(c);
+      cudaEventRecord(beg, st);
+    }
+  }
+  void done() {
+    if (c->profile && beg) {
+      cudaEvent_t end = get_event(c);
+      cudaEventRecord(end, st);
+      c->prof.push_back(ProfRec{name, beg, end, grid, block, smem});
+    }
+  }
+};
+
+// ------------------------------------------------------------------ validation
+
+li_status check_cache(li_ctx* ctx, const li_cache* c, const char* what) {
+  if (!c) return fail(ctx, LI_ERR_ARG, "%s: cache is NULL", what);
+  if (!c->data || !c->lengths) return fail(ctx, LI_ERR_ARG, "%s: cache data/lengths is NULL", what);
+  if (c->dtype != LI_F32 && c->dtype != LI_BF16 && c->dtype != LI_E4M3)
+    return fail(ctx, LI_ERR_DTYPE, "%s: unknown cache dtype %d", what, static_cast<int>(c->dtype));
+  if (c->dtype == LI_E4M3 && !c->scale) return fail(ctx, LI_ERR_ARG, "%s: E4M3 cache needs a scale array", what);
+  if (c->batch < 1 || c->capacity < 1) return fail(ctx, LI_ERR_SHAPE, "%s: batch and capacity must be >= 1", what);
+  if (static_cast<int64_t>(c->batch) * c->capacity >= (int64_t(1) << 31))
+    return fail(ctx, LI_ERR_SHAPE, "%s: batch * capacity must be < 2^31", what);
+  const int kmul = c->dtype == LI_F32 ? 8 : (c->dtype == LI_BF16 ? 16 : 32);
+  if (c->dim < kmul || c->dim > 256 || c->dim % kmul)
+    return fail(ctx, LI_ERR_SHAPE, "%s: dim %d must be a multiple of %d in [%d, 256]", what, c->dim, kmul, kmul);
+  if (!aligned(c->data, 16)) return fail(ctx, LI_ERR_ALIGN, "%s: cache data not 16-byte aligned", what);
+  if (c->scale && !aligned(c->scale, 4)) return fail(ctx, LI_ERR_ALIGN, "%s: scale not 4-byte aligned", what);
+  return LI_OK;
+}
+
+li_status check_query(li_ctx* ctx, const li_cache* c, const li_query* q, const char* what) {
+  if (!q) return fail(ctx, LI_ERR_ARG, "%s: query is NULL", what);
+  if (!q->q || !q->w) return fail(ctx, LI_ERR_ARG, "%s: q and w must be non-NULL", what);
+  if (q->dtype != c->dtype)
+    return fail(ctx, LI_ERR_DTYPE, "%s: query dtype %d must match the cache dtype %d", what,
+                static_cast<int>(q->dtype), static_cast<int>(c->dtype));
+  if (q->dtype == LI_E4M3 && !q->q_scale) return fail(ctx, LI_ERR_ARG, "%s: E4M3 query needs q_scale", what);
+  if (q->H < 1 || q->H > 256) return fail(ctx, LI_ERR_SHAPE, "%s: H = %d must be in [1, 256]", what, q->H);
+  if (q->T < 1) return fail(ctx, LI_ERR_SHAPE, "%s: T must be >= 1", what);
+  if (static_cast<int64_t>(c->batch) * q->T >= (int64_t(1) << 31))
+    return fail(ctx, LI_ERR_SHAPE, "%s: batch * T too large", what);
+  if (!aligned(q->q, 16)) return fail(ctx, LI_ERR_ALIGN, "%s: q not 16-byte aligned", what);
+  return LI_OK;
+}
+
+li_status check_ws(li_ctx* ctx, void* ws, size_t ws_bytes, const WsLayout& L, const char* what) {
+  if (!ws) return fail(ctx, LI_ERR_WORKSPACE, "%s: workspace is NULL", what);
+  if (!aligned(ws, 256)) return fail(ctx, LI_ERR_WORKSPACE, "%s: workspace not 256-byte aligned", what);
+  if (ws_bytes < L.total)
+    return fail(ctx, LI_ERR_WORKSPACE, "%s: workspace of %zu bytes, %zu needed", what, ws_bytes, L.total);
+  return LI_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+li_status encode_map(li_ctx* ctx, CUtensorMap* m, li_dtype dt, int rank, void* base, const cuuint64_t* dims,
+                     const cuuint64_t* strides, const cuuint32_t* box, int swz) {
+  const CUtensorMapDataType t = dt == LI_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dt == LI_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapSwizzle sw = swz == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swz == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_32B;
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = ctx->encode(m, t, rank, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ctx, LI_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LI_OK;
+}
+
+// ------------------------------------------------------------------ scan plan
+
+struct ScanPlan {
+  ScanArgs a;
+  int kind;
+  int grid;
+};
+
+li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gather, int cand_stride,
+                    ScanPlan* P, const char* what) {
+  ScanArgs& a = P->a;
+  memset(&a, 0, sizeof(a));
+  const int eb = elt_bytes(c->dtype);
+  const int64_t row_bytes = static_cast<int64_t>(c->dim) * eb;
+  const int swz = row_bytes % 128 == 0 ? 128 : (row_bytes % 64 == 0 ? 64 : 32);
+  const int H_pad = (q->H + 15) / 16 * 16;
+  const int Qg = gather ? 1 : std::max(1, std::min(256 / H_pad, q->T));
+  const int N = Qg * H_pad;
+  const int n_groups = (q->T + Qg - 1) / Qg;
+  const int n_seg = gather ? c->batch * q->T : c->batch * n_groups;
+  if (n_seg > kMaxSegments)
+    return fail(ctx, LI_ERR_UNSUPPORTED, "%s: %d segments (batch x query groups) exceed %d", what, n_seg,
+                kMaxSegments);
+  a.batch = c->batch;
+  a.capacity = c->capacity;
+  a.T = q->T;
+  a.H = q->H;
+  a.H_pad = H_pad;
+  a.Qg = Qg;
+  a.n_groups = n_groups;
+  a.N = N;
+  a.n_segments = n_seg;
+  a.swz = swz;
+  a.elt_bytes = eb;
+  a.n_kchunks = static_cast<int>(row_bytes / swz);
+  a.row_bytes = row_bytes;
+  a.cand_stride = cand_stride;
+  a.n_acc = std::min(4, 512 / N);
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(a.n_acc * N)) cols <<= 1;
+  a.tmem_cols = cols;
+  const int kind = c->dtype == LI_F32 ? kKindTF32 : (c->dtype == LI_BF16 ? kKindBF16 : kKindE4M3);
+  const uint32_t fmt = c->dtype == LI_F32 ? 2u : (c->dtype == LI_BF16 ? 1u : 0u);
+  a.idesc = make_instr_desc(fmt, kTileM, N);
+  a.a_stage_bytes = kTileM * swz;
+  a.b_slot_bytes = static_cast<uint32_t>(a.n_kchunks) * N * swz;
+  const size_t misc = 640 + 16 + (kMaxSegments + 1) * 4 + 4 * (3 * N + 16) * 4;
+  const size_t budget = static_cast<size_t>(ctx->max_smem_optin) - 1024;
+  int bslots = 2;
+  if (2 * a.b_slot_bytes + 6 * a.a_stage_bytes + misc > budget) bslots = 1;
+  const int64_t room = static_cast<int64_t>(budget) - static_cast<int64_t>(bslots) * a.b_slot_bytes -
+                       static_cast<int64_t>(misc);
+  const int stages = static_cast<int>(std::min<int64_t>(kMaxStages, room / a.a_stage_bytes));
+  if (stages < (gather ? 6 : 3))
+    return fail(ctx, LI_ERR_UNSUPPORTED, "%s: operands too large for shared memory (N=%d, dim=%d)", what, N, c->dim);
+  a.n_bslots = bslots;
+  a.n_stages = stages;
+  a.misc_offset = stages * a.a_stage_bytes + bslots * a.b_slot_bytes;
+  a.smem_bytes = static_cast<uint32_t>(std::max<size_t>(1024 + a.misc_offset + misc, 120 * 1024));
+  a.wait_ns = ctx->wait_ns;
+
+  // Tensor maps: cache rows and queries.
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c->dim),
+                                static_cast<cuuint64_t>(c->batch) * c->capacity};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(swz / eb), static_cast<cuuint32_t>(kTileM)};
+    li_status s = encode_map(ctx, &a.map_a, c->dtype, 2, c->data, dims, strides, box, swz);
+    if (s != LI_OK) return s;
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(c->dim), static_cast<cuuint64_t>(q->H),
+                                static_cast<cuuint64_t>(c->batch) * q->T};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes),
+                                   static_cast<cuuint64_t>(row_bytes) * q->H};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(swz / eb), static_cast<cuuint32_t>(H_pad),
+                               static_cast<cuuint32_t>(Qg)};
+    li_status s = encode_map(ctx, &a.map_b, c->dtype, 3, const_cast<void*>(q->q), dims, strides, box, swz);
+    if (s != LI_OK) return s;
+  }
+  a.cache = static_cast<const uint8_t*>(c->data);
+  a.cache_scale = c->dtype == LI_E4M3 ? c->scale : nullptr;
+  a.lengths = c->lengths;
+  a.q_pos = q->q_pos;
+  a.w = q->w;
+  a.q_scale = q->dtype == LI_E4M3 ? q->q_scale : nullptr;
+  a.beta = q->beta;
+  P->kind = kind;
+  const int64_t tiles_per_seg = (static_cast<int64_t>(gather ? cand_stride : c->capacity) + kTileM - 1) / kTileM;
+  P->grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ctx->num_sms, n_seg * tiles_per_seg)));
+  return LI_OK;
+}
+
+li_status run_scan(li_ctx* ctx, ScanPlan& P, bool gather, cudaStream_t st) {
+  Launch L(ctx, st, gather ? "gather" : "scan", P.grid, kScanThreads, static_cast<int>(P.a.smem_bytes));
+  const cudaError_t e = launch_scan_kernel(P.kind, gather, P.a, P.grid, st);
+  L.done();
+  if (e != cudaSuccess) return cuda_fail(ctx, e, gather ? "gather kernel launch" : "scan kernel launch");
+  return LI_OK;
+}
+
+// ------------------------------------------------------------------ selection
+
+li_status memset_async(li_ctx* ctx, void* p, size_t bytes, cudaStream_t st) {
+  Launch L(ctx, st, "memset", 0, 0, 0);
+  const cudaError_t e = cudaMemsetAsync(p, 0, bytes, st);
+  L.done();
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaMemsetAsync");
+  return LI_OK;
+}
+
+// Clears the histogram and per-row info of `rows` rows.
+li_status clear_select_state(li_ctx* ctx, void* ws, const WsLayout& L, int64_t rows, cudaStream_t st) {
+  li_status s = memset_async(ctx, at<uint8_t>(ws, L.hist), rows * kHistBins * 4, st);
+  if (s != LI_OK) return s;
+  return memset_async(ctx, at<uint8_t>(ws, L.rowinfo), rows * 16 * 4, st);
+}
+
+li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaStream_t st) {
+  t.hist = at<unsigned int>(ws, L.hist);
+  t.rowinfo = at<int>(ws, L.rowinfo);
+  t.chunk_gt = at<int>(ws, L.chunk_gt);
+  t.chunk_off = at<int>(ws, L.chunk_off);
+  t.cand = at<uint2>(ws, L.cand);
+  t.n_chunks = (t.n + kTopkChunk - 1) / kTopkChunk;
+  if (t.n_chunks < 1) t.n_chunks = 1;
+  if (t.n_chunks > kMaxTopkChunks)
+    return fail(ctx, LI_ERR_UNSUPPORTED, "selection rows longer than %d", kMaxTopkChunks * kTopkChunk);
+  if (t.rows > 65535) return fail(ctx, LI_ERR_UNSUPPORTED, "more than 65535 selection rows");
+  static const char* names[4] = {"topk_hist", "topk_filter", "topk_select", "topk_emit"};
+  for (int stage = t.hist_ready ? 1 : 0; stage < 4; ++stage) {
+    const int grid = stage == 2 ? t.rows : t.rows * t.n_chunks;
+    Launch Lc(ctx, st, names[stage], grid, stage == 2 ? 1024 : kTopkThreads, 0);
+    const cudaError_t e = launch_topk_stage(stage, t, st);
+    Lc.done();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, names[stage]);
+  }
+  return LI_OK;
+}
+
+TopkArgs topk_args(const float* scores, int64_t stride, int rows, int n, int k) {
+  TopkArgs t;
+  memset(&t, 0, sizeof(t));
+  t.scores = scores;
+  t.row_stride = stride;
+  t.rows = rows;
+  t.n = n;
+  t.k = k;
+  t.len_div = 1;
+  return t;
+}
+
+// Full-prefix scan + selection shared by li_score_topk and li_dsa_score_topk.
+li_status score_topk_impl(li_ctx* ctx, const li_cache* c, const li_query* q, int k, int32_t* out_idx,
+                          float* out_score, float* dump, void* ws, size_t ws_bytes, cudaStream_t st,
+                          const char* what) {
+  if (!ctx) return LI_ERR_ARG;
+  li_status s = check_cache(ctx, c, what);
+  if (s != LI_OK) return s;
+  if ((s = check_query(ctx, c, q, what)) != LI_OK) return s;
+  if (!out_idx) return fail(ctx, LI_ERR_ARG, "%s: out_idx is NULL", what);
+  if (k < 1 || k > c->capacity) return fail(ctx, LI_ERR_ARG, "%s: k = %d must be in [1, capacity]", what, k);
+  const int64_t rows = static_cast<int64_t>(c->batch) * q->T;
+  const WsLayout L = ws_layout(rows, c->capacity, 0);
+  if ((s = check_ws(ctx, ws, ws_bytes, L, what)) != LI_OK) return s;
+  ScanPlan P;
+  if ((s = plan_scan(ctx, c, q, false, 0, &P, what)) != LI_OK) return s;
+  float* scores = dump ? dump : at<float>(ws, L.scores);
+  P.a.scores = scores;
+  P.a.score_stride = c->capacity;
+  P.a.status = at<int>(ws, L.status);
+  P.a.hist = at<unsigned int>(ws, L.hist);
+  if ((s = clear_select_state(ctx, ws, L, rows, st)) != LI_OK) return s;
+  if ((s = run_scan(ctx, P, false, st)) != LI_OK) return s;
+  TopkArgs t = topk_args(scores, c->capacity, static_cast<int>(rows), c->capacity, k);
+  t.lengths = c->lengths;
+  t.len_div = q->T;
+  t.q_pos = q->q_pos;
+  t.out_idx = out_idx;
+  t.out_score = out_score;
+  t.hist_ready = true;
+  return run_topk(ctx, t, ws, L, st);
+}
+
+}  // namespace
+
+// ======================================================================== C ABI
+
+extern "C" {
+
+const char* li_status_string(li_status s) {
+  switch (s) {
+    case LI_OK: return "ok";
+    case LI_ERR_ARG: return "invalid argument";
+    case LI_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case LI_ERR_DTYPE: return "unsupported dtype";
+    case LI_ERR_ALIGN: return "misaligned pointer or row";
+    case LI_ERR_WORKSPACE: return "workspace missing, short or misaligned";
+    case LI_ERR_CAPACITY: return "append past the cache capacity";
+    case LI_ERR_CUDA: return "CUDA error";
+    case LI_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+    case LI_ERR_UNSUPPORTED: return "unsupported request";
+    case LI_ERR_INDEX: return "candidate index outside the valid prefix";
+  }
+  return "unknown status";
+}
+
+li_status li_create(li_ctx** out, int device) {
+  if (!out) return LI_ERR_ARG;
+  *out = nullptr;
+  li_ctx* c = new (std::nothrow) li_ctx();
+  if (!c) return LI_ERR_ARG;
+  int major = 0, minor = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&c->max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  if (e != cudaSuccess) {
+    delete c;
+    return LI_ERR_CUDA;
+  }
+  if (major != 10 || minor != 0) {
+    delete c;
+    return LI_ERR_UNSUPPORTED;
+  }
+  c->device = device;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+    delete c;
+    return LI_ERR_CUDA;
+  }
+  c->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  *out = c;
+  return LI_OK;
+}
+
+li_status li_destroy(li_ctx* c) {
+  if (!c) return LI_ERR_ARG;
+  for (auto& r : c->prof) {
+    cudaEventDestroy(r.beg);
+    cudaEventDestroy(r.end);
+  }
+  for (auto e : c->free_events) cudaEventDestroy(e);
+  delete c;
+  return LI_OK;
+}
+
+const char* li_last_error(const li_ctx* c) { return c ? c->last_error.c_str() : "null context"; }
+
+size_t li_workspace_bytes(const li_ctx* c, int batch, int T, int capacity, int H, int k, int B) {
+  (void)c;
+  (void)H;
+  (void)k;
+  const int64_t rows = static_cast<int64_t>(std::max(batch, 1)) * std::max(T, 1);
+  return ws_layout(rows, std::max(capacity, 1), std::max(B, 0)).total;
+}
+
+li_status li_device_status(li_ctx* c, const void* ws, void* stream, li_status* out) {
+  if (!c || !ws || !out) return LI_ERR_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(c, e, "li_device_status read");
+  e = cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(c, e, "li_device_status clear");
+  *out = static_cast<li_status>(v);
+  return LI_OK;
+}
+
+li_status li_set_wait_limit(li_ctx* c, uint64_t ns) {
+  if (!c) return LI_ERR_ARG;
+  c->wait_ns = ns;
+  return LI_OK;
+}
+
+li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_dtype h_dtype, int d_model,
+                           const void* W_down, int T, void* ws, size_t ws_bytes, void* stream) {
+  const char* what = "li_append_latent";
+  if (!c) return LI_ERR_ARG;
+  li_status s = check_cache(c, cache, what);
+  if (s != LI_OK) return s;
+  if (!h) return fail(c, LI_ERR_ARG, "%s: h is NULL", what);
+  if (T < 1) return fail(c, LI_ERR_SHAPE, "%s: T must be >= 1", what);
+  if (T > cache->capacity) return fail(c, LI_ERR_SHAPE, "%s: T = %d exceeds the capacity", what, T);
+  if (W_down) {
+    if (h_dtype != LI_F32 && h_dtype != LI_BF16) return fail(c, LI_ERR_DTYPE, "%s: h must be F32 or BF16", what);
+    if (d_model < 8 || d_model % 8) return fail(c, LI_ERR_SHAPE, "%s: d_model must be a multiple of 8", what);
+  } else if (h_dtype != LI_F32) {
+    return fail(c, LI_ERR_DTYPE, "%s: without W_down, h must be the F32 latent", what);
+  }
+  const WsLayout L = ws_layout(1, 1, 0);
+  if ((s = check_ws(c, ws, ws_bytes, L, what)) != LI_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int dim = cache->dim;
+  unsigned int* done = at<unsigned int>(ws, L.done);
+  int* status = at<int>(ws, L.status);
+  if (!W_down) {
+    // h already holds the fp32 rows [batch][T][dim]: quantise and store.
+    Launch Ls(c, st, "append_store", 0, 256, 0);
+    const cudaError_t e = launch_append_store(static_cast<const float*>(h), dim, cache->batch, T, 0, T, true,
+                                              cache->data, cache->scale, cache->lengths, cache->capacity, dim,
+                                              cache->dtype, done, status, st);
+    Ls.done();
+    return e == cudaSuccess ? LI_OK : cuda_fail(c, e, "append store launch");
+  }
+  // c = W_down h in chunks of tokens, staged as fp32 in the workspace.
+  float* tmp = at<float>(ws, L.tmp);
+  const int eb = elt_bytes(h_dtype);
+  const int tchunk = std::max(1, std::min(T, kAppendChunkTok / cache->batch));
+  for (int t0 = 0; t0 < T; t0 += tchunk) {
+    const int tn = std::min(tchunk, T - t0);
+    if (tn == T) {
+      // every token of the batch at once: h rows are contiguous
+      Launch Lg(c, st, "append_gemv", 0, 256, 0);
+      const cudaError_t e = launch_append_gemv(h, h_dtype, W_down, d_model, dim, cache->batch * T, tmp, st);
+      Lg.done();
+      if (e != cudaSuccess) return cuda_fail(c, e, "append gemv launch");
+    } else {
+      for (int b = 0; b < cache->batch; ++b) {
+        const uint8_t* hb = static_cast<const uint8_t*>(h) + (static_cast<int64_t>(b) * T + t0) * d_model * eb;
+        Launch Lg(c, st, "append_gemv", 0, 256, 0);
+        const cudaError_t e = launch_append_gemv(hb, h_dtype, W_down, d_model, dim, tn,
+                                                 tmp + static_cast<int64_t>(b) * tn * dim, st);
+        Lg.done();
+        if (e != cudaSuccess) return cuda_fail(c, e, "append gemv launch");
+      }
+    }
+    Launch Ls(c, st, "append_store", 0, 256, 0);
+    const cudaError_t e = launch_append_store(tmp, dim, cache->batch, tn, t0, T, t0 + tn >= T, cache->data,
+                                              cache->scale, cache->lengths, cache->capacity, dim, cache->dtype,
+                                              done, status, st);
+    Ls.done();
+    if (e != cudaSuccess) return cuda_fail(c, e, "append store launch");
+  }
+  return LI_OK;
+}
+
+li_status li_absorb_query(li_ctx* c, const void* q, li_dtype q_dtype, int n_tok, int H, int d_k, const void* W_K,
+                          int64_t W_K_head_stride, const float* b_K, int64_t b_K_head_stride, int d_c,
+                          li_dtype out_dtype, void* q_abs, float* q_abs_scale, float* beta, void* stream) {
+  const char* what = "li_absorb_query";
+  if (!c) return LI_ERR_ARG;
+  if (!q || !q_abs) return fail(c, LI_ERR_ARG, "%s: q and q_abs must be non-NULL", what);
+  if (q_dtype != LI_F32 && q_dtype != LI_BF16) return fail(c, LI_ERR_DTYPE, "%s: q must be F32 or BF16", what);
+  if (out_dtype != LI_F32 && out_dtype != LI_BF16 && out_dtype != LI_E4M3)
+    return fail(c, LI_ERR_DTYPE, "%s: unknown out dtype", what);
+  if (out_dtype == LI_E4M3 && !q_abs_scale) return fail(c, LI_ERR_ARG, "%s: E4M3 output needs q_abs_scale", what);
+  if (n_tok < 1 || H < 1 || d_k < 1 || d_k > 256 || d_c < 1 || d_c > 256)
+    return fail(c, LI_ERR_SHAPE, "%s: need n_tok, H >= 1 and d_k, d_c in [1, 256]", what);
+  if (n_tok > 65535) return fail(c, LI_ERR_SHAPE, "%s: n_tok must be <= 65535 per call", what);
+  if (!W_K && d_c != d_k) return fail(c, LI_ERR_SHAPE, "%s: identity decoder needs d_c == d_k", what);
+  if (beta && !b_K) return fail(c, LI_ERR_ARG, "%s: beta requested without b_K", what);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Launch L(c, st, "absorb", 0, 256, 0);
+  const cudaError_t e = launch_absorb(q, q_dtype, n_tok, H, d_k, W_K, W_K_head_stride, b_K, b_K_head_stride, d_c,
+                                      out_dtype, q_abs, q_abs_scale, beta, st);
+  L.done();
+  if (e != cudaSuccess) return cuda_fail(c, e, "absorb launch");
+  return LI_OK;
+}
+
+li_status li_score_topk(li_ctx* c, const li_cache* cache, const li_query* q, int k, int32_t* out_idx,
+                        float* out_score, float* scores_dump, void* ws, size_t ws_bytes, void* stream) {
+  return score_topk_impl(c, cache, q, k, out_idx, out_score, scores_dump, ws, ws_bytes,
+                         static_cast<cudaStream_t>(stream), "li_score_topk");
+}
+
+li_status li_dsa_score_topk(li_ctx* c, const li_cache* key_cache, const li_query* q, int k, int32_t* out_idx,
+                            float* out_score, float* scores_dump, void* ws, size_t ws_bytes, void* stream) {
+  return score_topk_impl(c, key_cache, q, k, out_idx, out_score, scores_dump, ws, ws_bytes,
+                         static_cast<cudaStream_t>(stream), "li_dsa_score_topk");
+}
+
+li_status li_hs_anchor_candidates(li_ctx* c, const li_cache* cache, const li_query* q, int B, int k,
+                                  int32_t* cand, int32_t* cand_n, int32_t* anchor_idx, float* anchor_score,
+                                  float* scores_dump, void* ws, size_t ws_bytes, void* stream) {
+  const char* what = "li_hs_anchor_candidates";
+  if (!c) return LI_ERR_ARG;
+  li_status s = check_cache(c, cache, what);
+  if (s != LI_OK) return s;
+  if ((s = check_query(c, cache, q, what)) != LI_OK) return s;
+  if (!cand || !cand_n || !anchor_idx) return fail(c, LI_ERR_ARG, "%s: cand, cand_n, anchor_idx required", what);
+  if (k < 1 || B < k || k > cache->capacity)
+    return fail(c, LI_ERR_ARG, "%s: need 1 <= k <= B and k <= capacity (k=%d, B=%d)", what, k, B);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t rows = static_cast<int64_t>(cache->batch) * q->T;
+  const WsLayout L = ws_layout(rows, cache->capacity, B);
+  if ((s = check_ws(c, ws, ws_bytes, L, what)) != LI_OK) return s;
+  ScanPlan P;
+  if ((s = plan_scan(c, cache, q, false, 0, &P, what)) != LI_OK) return s;
+  float* scores = scores_dump ? scores_dump : at<float>(ws, L.scores);
+  P.a.scores = scores;
+  P.a.score_stride = cache->capacity;
+  P.a.status = at<int>(ws, L.status);
+  P.a.hist = at<unsigned int>(ws, L.hist);
+  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
+  if ((s = run_scan(c, P, false, st)) != LI_OK) return s;
+  // candidates: top-B of the full prefix, with their scores
+  float* cscores = at<float>(ws, L.cand_scores);
+  TopkArgs t = topk_args(scores, cache->capacity, static_cast<int>(rows), cache->capacity, B);
+  t.lengths = cache->lengths;
+  t.len_div = q->T;
+  t.q_pos = q->q_pos;
+  t.out_idx = cand;
+  t.out_score = cscores;
+  t.out_count = cand_n;
+  t.hist_ready = true;
+  if ((s = run_topk(c, t, ws, L, st)) != LI_OK) return s;
+  // the anchor's own selection: top-k of the candidates (the top-k of the
+  // prefix under the same order is a prefix of its top-B)
+  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
+  TopkArgs t2 = topk_args(cscores, B, static_cast<int>(rows), B, k);
+  t2.lengths = cand_n;
+  t2.len_div = 1;
+  t2.idx_map = cand;
+  t2.map_stride = B;
+  t2.out_idx = anchor_idx;
+  t2.out_score = anchor_score;
+  return run_topk(c, t2, ws, L, st);
+}
+
+li_status li_hs_follower_refine(li_ctx* c, const li_cache* cache, const li_query* q, const int32_t* cand,
+                                const int32_t* cand_n, int B, int k, int32_t* out_idx, float* out_score,
+                                float* scores_dump, void* ws, size_t ws_bytes, void* stream) {
+  const char* what = "li_hs_follower_refine";
+  if (!c) return LI_ERR_ARG;
+  li_status s = check_cache(c, cache, what);
+  if (s != LI_OK) return s;
+  if ((s = check_query(c, cache, q, what)) != LI_OK) return s;
+  if (!cand || !cand_n || !out_idx) return fail(c, LI_ERR_ARG, "%s: cand, cand_n, out_idx required", what);
+  if (k < 1 || B < k) return fail(c, LI_ERR_ARG, "%s: need 1 <= k <= B (k=%d, B=%d)", what, k, B);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t rows = static_cast<int64_t>(cache->batch) * q->T;
+  const WsLayout L = ws_layout(rows, B, B);
+  if ((s = check_ws(c, ws, ws_bytes, L, what)) != LI_OK) return s;
+  ScanPlan P;
+  if ((s = plan_scan(c, cache, q, true, B, &P, what)) != LI_OK) return s;
+  float* scores = scores_dump ? scores_dump : at<float>(ws, L.scores);
+  P.a.scores = scores;
+  P.a.score_stride = B;
+  P.a.status = at<int>(ws, L.status);
+  P.a.hist = at<unsigned int>(ws, L.hist);
+  P.a.cand = cand;
+  P.a.cand_n = cand_n;
+  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
+  if ((s = run_scan(c, P, true, st)) != LI_OK) return s;
+  TopkArgs t = topk_args(scores, B, static_cast<int>(rows), B, k);
+  t.lengths = cand_n;
+  t.len_div = 1;
+  t.idx_map = cand;
+  t.map_stride = B;
+  t.out_idx = out_idx;
+  t.out_score = out_score;
+  t.hist_ready = true;
+  return run_topk(c, t, ws, L, st);
+}
+
+li_status li_topk(li_ctx* c, const float* scores, int rows, int n, int64_t row_stride, const int32_t* lengths,
+                  int k, int32_t* out_idx, float* out_score, void* ws, size_t ws_bytes, void* stream) {
+  const char* what = "li_topk";
+  if (!c) return LI_ERR_ARG;
+  if (!scores || !out_idx) return fail(c, LI_ERR_ARG, "%s: scores and out_idx must be non-NULL", what);
+  if (rows < 1 || n < 1 || k < 1 || row_stride < n)
+    return fail(c, LI_ERR_SHAPE, "%s: need rows, n, k >= 1 and row_stride >= n", what);
+  const WsLayout L = ws_layout(rows, n, 0);
+  li_status s = check_ws(c, ws, ws_bytes, L, what);
+  if (s != LI_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
+  TopkArgs t = topk_args(scores, row_stride, rows, n, k);
+  t.lengths = lengths;
+  t.out_idx = out_idx;
+  t.out_score = out_score;
+  return run_topk(c, t, ws, L, st);
+}
+
+li_status li_profile_enable(li_ctx* c, int enable) {
+  if (!c) return LI_ERR_ARG;
+  c->profile = enable != 0;
+  return LI_OK;
+}
+
+li_status li_profile_read(li_ctx* c, li_profile_record* out, int max, int* count) {
+  if (!c || !count) return LI_ERR_ARG;
+  *count = static_cast<int>(c->prof.size());
+  for (int i = 0; i < *count && i < max && out; ++i) {
+    const ProfRec& r = c->prof[i];
+    cudaError_t e = cudaEventSynchronize(r.end);
+    if (e != cudaSuccess) return cuda_fail(c, e, "li_profile_read");
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, r.beg, r.end);
+    memset(&out[i], 0, sizeof(out[i]));
+    snprintf(out[i].kernel, sizeof(out[i].kernel), "%s", r.name.c_str());
+    out[i].ms = ms;
+    out[i].grid = r.grid;
+    out[i].block = r.block;
+    out[i].smem = r.smem;
+  }
+  return LI_OK;
+}
+
+li_status li_profile_reset(li_ctx* c) {
+  if (!c) return LI_ERR_ARG;
+  for (auto& r : c->prof) {
+    c->free_events.push_back(r.beg);
+    c->free_events.push_back(r.end);
+  }
+  c->prof.clear();
+  return LI_OK;
+}
+
+}  // extern "C"

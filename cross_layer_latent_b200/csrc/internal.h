@@ -1,0 +1,102 @@
+// internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/li.h"
+
+namespace li {
+
+constexpr int kTileM = 128;          // cache rows per MMA tile (UMMA M)
+constexpr int kScanThreads = 192;    // warp 0 loads, warp 1 issues MMAs, warps 2..5 epilogue
+constexpr int kMaxSegments = 1024;   // (sequence, query group) segments per scan launch
+constexpr int kMaxStages = 32;
+constexpr int kHistBins = 2048;      // first radix digit: key bits 31..21
+
+// Arguments of the scoring kernel (scan of whole prefixes, or gather of
+// candidate rows).  Tensor maps first: they must stay 64-byte aligned.
+struct alignas(64) ScanArgs {
+  CUtensorMap map_a;          // cache rows: dims {dim, batch*capacity}, box {swz/elt, 128}
+  CUtensorMap map_b;          // queries: dims {dim, H, batch*T}, box {swz/elt, H_pad, Qg}
+  const uint8_t* cache;       // cache data (gather loads)
+  const float* cache_scale;   // [batch*capacity] or null
+  const int* lengths;         // [batch]
+  const int* q_pos;           // [batch*T] or null
+  const float* w;             // [batch*T*H]
+  const float* q_scale;       // [batch*T*H] or null
+  const float* beta;          // [batch*T*H] or null
+  const int* cand;            // gather: [batch*T][cand_stride]
+  const int* cand_n;          // gather: [batch*T]
+  float* scores;              // [batch*T][score_stride]
+  unsigned int* hist;         // fused first-digit histogram [batch*T][2048] or null
+  int* status;
+  int64_t score_stride;
+  int64_t row_bytes;
+  uint64_t wait_ns;
+  int batch, capacity, T, H, H_pad, Qg, n_groups, N;
+  int cand_stride;
+  int swz, n_kchunks, elt_bytes;
+  int n_stages, n_bslots, n_acc;
+  uint32_t tmem_cols, idesc;
+  uint32_t a_stage_bytes, b_slot_bytes, misc_offset, smem_bytes;
+  int n_segments;
+};
+
+// Kernel families (for the launch profile).
+enum KernelKind { kKScan = 0, kKGather, kKTopkHist, kKTopkFilter, kKTopkSelect, kKTopkEmit,
+                  kKAppendGemv, kKAppendStore, kKAbsorb, kKMemset };
+
+cudaError_t launch_scan_kernel(int kind, bool gather, const ScanArgs& a, int grid, cudaStream_t st);
+
+// ---- top-k
+
+struct TopkArgs {
+  const float* scores;
+  int64_t row_stride;
+  int rows, n, k;
+  // per-row valid length: n_r = min(n, lengths ? lengths[r / len_div] : n),
+  // further capped by q_pos[r] + 1 when q_pos is given; negatives -> 0.
+  const int* lengths;
+  int len_div;
+  const int* q_pos;
+  const int* idx_map;         // output index = idx_map[r * map_stride + pos], or pos
+  int64_t map_stride;
+  int32_t* out_idx;
+  float* out_score;
+  int32_t* out_count;         // k_eff per row, or null
+  // workspace
+  unsigned int* hist;         // [rows][2048]
+  int* rowinfo;               // [rows][16]
+  int* chunk_gt;              // [rows][n_chunks]
+  int* chunk_off;             // [rows][n_chunks]
+  uint2* cand;                // [rows][n]
+  int n_chunks;
+  bool hist_ready;            // first-digit histogram already accumulated (fused)
+};
+
+constexpr int kTopkChunk = 4096;
+constexpr int kTopkThreads = 256;
+constexpr int kMaxTopkChunks = 8192;
+
+// The four stages of a selection, launched in order on one stream:
+// 0 first-digit histogram (skipped when hist_ready), 1 filter (boundary
+// bucket candidates and per-chunk counts), 2 select (exact threshold, tie
+// cut and output offsets, one CTA per row), 3 emit (ordered output).
+cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st);
+
+// ---- construction
+
+cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_model, int dim,
+                               int n_tok, float* out, cudaStream_t st);
+cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int batch, int T_chunk, int t0,
+                                int T_total, bool bump, void* data, float* scale, int32_t* lengths,
+                                int capacity, int dim, int dtype, unsigned int* done_counter,
+                                int* status, cudaStream_t st);
+cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
+                          int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
+                          int out_dtype, void* q_abs, float* q_abs_scale, float* beta,
+                          cudaStream_t st);
+
+}  // namespace li

@@ -1,0 +1,277 @@
+/*
+ * li.h -- C ABI of libli, the B200 (sm_100a) LatentIndex decode indexer.
+ *
+ * What it computes.  LatentIndex (paperlayer summary of arXiv 2610.04635,
+ * "LatentIndex: Cross-Layer Sharing with Layer-Specific Selection for Sparse
+ * Attention") keeps ONE indexer cache per group of G layers: a latent c_s
+ * built by the group's first ("anchor") layer from its hidden state (Sec. 3.1).
+ * Every layer l of the group owns a decoder W_K^l; at inference the decoder is
+ * absorbed into the layer's query, qt_{t,h} = W_K^{l T} q_{t,h}, so the layer
+ * scores the shared latent directly (Sec. 3.1, Sec. B.2).  The score is the
+ * DSA-style head-weighted ReLU form
+ *
+ *     score(t, s) = sum_h w_{t,h} * max(0, qt_{t,h} . c_s + beta_{t,h})
+ *
+ * (beta = q . b_K for decoders with an output bias, Sec. A.3; NULL otherwise),
+ * and each layer keeps its own top-k tokens (Sec. 3.1, up to 2048 per query,
+ * Sec. 4.1).  In hierarchical selection (HS) the anchor proposes its top-B
+ * candidates and each follower rescores only those (Sec. 3.2, Sec. C.4).  A
+ * DSA-style comparison path scores per-layer key caches with the raw query.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.  Every pointer argument is a DEVICE pointer unless marked "host".
+ *   The caller owns all memory, including the workspace; the library never
+ *   allocates device memory.  A workspace must be at least
+ *   li_workspace_bytes(...) bytes, 256-byte aligned, and zero-filled once
+ *   before its first use; after that the library keeps it consistent.  Its
+ *   first 4 bytes are the device status word (see li_device_status).
+ * Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every
+ *   call only enqueues work on that stream and returns; none synchronises,
+ *   except li_device_status.  A li_ctx must not be used by two host threads
+ *   at once.  Two calls that share a workspace must be ordered on the GPU.
+ * Errors.  Host-detected errors (bad arguments, shapes, dtypes, alignment, a
+ *   short workspace) return before anything is enqueued and leave every
+ *   output untouched; li_last_error(ctx) then describes the problem.  A
+ *   failing CUDA call returns LI_ERR_CUDA.  Errors found on the device (an
+ *   append past capacity, a candidate index outside the valid prefix, a
+ *   bounded wait that ran out) are recorded in the workspace's status word
+ *   and reported by li_device_status.  No C++ exception crosses this ABI.
+ * Selections.  A selection of budget k over n valid positions returns the
+ *   k_eff = min(k, n) positions with the largest scores, ordered by (score
+ *   descending, position ascending) to decide who is in, and written in
+ *   ascending position order; slots k_eff..k-1 hold -1 (indices) and -inf
+ *   (scores).  -0.0 ranks equal to +0.0.  NaN scores are invalid input.
+ * Valid prefix.  In decode (q_pos == NULL) the query of sequence b sees
+ *   positions [0, lengths[b]) -- the current token is appended before it
+ *   scores.  With q_pos, query (b, t) sees [0, min(lengths[b], q_pos[b][t]+1)).
+ */
+#ifndef LI_H
+#define LI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LI_API __attribute__((visibility("default")))
+#else
+#define LI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LI_OK = 0,
+  LI_ERR_ARG = 1,              /* null pointer or out-of-range scalar          */
+  LI_ERR_SHAPE = 2,            /* unsupported or inconsistent sizes            */
+  LI_ERR_DTYPE = 3,            /* dtype not supported for this operand         */
+  LI_ERR_ALIGN = 4,            /* pointer or row not 16-byte aligned           */
+  LI_ERR_WORKSPACE = 5,        /* workspace missing, short or misaligned       */
+  LI_ERR_CAPACITY = 6,         /* (device) append past the cache capacity      */
+  LI_ERR_CUDA = 7,             /* a CUDA runtime / driver call failed          */
+  LI_ERR_DEVICE_TIMEOUT = 8,   /* (device) a bounded wait ran out              */
+  LI_ERR_UNSUPPORTED = 9,      /* valid request this build does not implement  */
+  LI_ERR_INDEX = 10            /* (device) candidate index outside the prefix  */
+} li_status;
+
+typedef enum { LI_F32 = 0, LI_BF16 = 1, LI_E4M3 = 2 } li_dtype;
+
+/* Opaque host-side context: device properties, cached driver entry points,
+ * the last error message, the wait limit and the optional launch profile.
+ * It owns no device memory. */
+typedef struct li_ctx li_ctx;
+
+/* A per-group latent cache (LatentIndex) or a per-layer key cache (DSA path).
+ * data    [batch][capacity][dim] elements of `dtype`, row-major; each row must
+ *         be a multiple of 16 bytes and `data` 16-byte aligned.
+ * scale   [batch][capacity] fp32 per-token dequantisation scale (LI_E4M3
+ *         only, NULL otherwise): element value = scale[b][s] * e4m3 code.
+ * lengths [batch] int32 valid rows per sequence (read and advanced on the
+ *         device by li_append_latent).
+ * dim: multiple of 8 (F32), 16 (BF16) or 32 (E4M3), at most 256.           */
+typedef struct {
+  void* data;
+  float* scale;
+  int32_t* lengths;
+  int32_t batch;
+  int32_t capacity;
+  int32_t dim;
+  li_dtype dtype;
+} li_cache;
+
+/* The queries of one layer for every sequence of the batch.
+ * q       [batch][T][H][dim] of `dtype`: the absorbed query qt for LatentIndex
+ *         (li_absorb_query output) or the raw query for the DSA path.  dtype
+ *         must match the cache: F32 with F32 (tf32 tensor cores), BF16 with
+ *         BF16, E4M3 with E4M3.  16-byte aligned.
+ * q_scale [batch][T][H] fp32 per-(token, head) dequantisation scale of an
+ *         E4M3 query; NULL otherwise.
+ * beta    [batch][T][H] fp32 decoder-bias term added before the ReLU, or NULL.
+ * w       [batch][T][H] fp32 head weights.
+ * T       query tokens per sequence (1 = decode).  H heads, 1..256.
+ * q_pos   [batch][T] int32 causal positions, or NULL for decode.           */
+typedef struct {
+  const void* q;
+  li_dtype dtype;
+  const float* q_scale;
+  const float* beta;
+  const float* w;
+  int32_t T;
+  int32_t H;
+  const int32_t* q_pos;
+} li_query;
+
+/* ------------------------------------------------------------------ setup */
+
+/* Create a context bound to CUDA device `device` (host-side state only).
+ * Fails with LI_ERR_UNSUPPORTED unless the device is compute capability 10.0. */
+LI_API li_status li_create(li_ctx** ctx, int device);
+LI_API li_status li_destroy(li_ctx* ctx);
+/* Message of the last host-detected error on this context ("" if none).
+ * The string is owned by the context and valid until its next call. */
+LI_API const char* li_last_error(const li_ctx* ctx);
+LI_API const char* li_status_string(li_status s);
+
+/* Bytes of workspace any call on caches of `batch` sequences with `T` query
+ * tokens each, `capacity` rows, budget k and HS budget B (0 if unused) needs.
+ * A workspace of this size serves every entry point for those sizes. */
+LI_API size_t li_workspace_bytes(const li_ctx* ctx, int batch, int T, int capacity, int H, int k, int B);
+
+/* Reads the device status word of `ws` after synchronising `stream`, stores
+ * it in *out (host) and clears it.  Returns LI_OK or LI_ERR_CUDA. */
+LI_API li_status li_device_status(li_ctx* ctx, const void* ws, void* stream, li_status* out);
+
+/* Upper bound, in nanoseconds, of every wait inside the library's kernels
+ * (default 2e9 = 2 s).  When a wait runs out the kernel records
+ * LI_ERR_DEVICE_TIMEOUT, drains its own copies in flight, frees its tensor
+ * memory and returns. */
+LI_API li_status li_set_wait_limit(li_ctx* ctx, uint64_t ns);
+
+/* ------------------------------------------------------------- a1: append */
+
+/* Latent (or key) construction and append (LatentIndex summary, Sec. 3.1:
+ * the anchor's hidden states build the shared latent once per token; the
+ * DSA path builds one key per layer the same way).  For every sequence b and
+ * new token t < T: c = W_down h[b][t] (fp32 accumulation), stored as the
+ * cache dtype (F32 as is; BF16 round-to-nearest-even; E4M3 with
+ * scale = amax|c| / 448 in fp32 division (1 if amax = 0) and codes
+ * e4m3_satfinite(c_i / scale)), into row lengths[b] + t; then
+ * lengths[b] += T.
+ * h       [batch][T][d_model] of h_dtype (F32 or BF16).
+ * W_down  [cache->dim][d_model] of h_dtype, row-major; or NULL, in which case
+ *         h is already [batch][T][cache->dim] fp32 and is stored as is.
+ * If lengths[b] + T > capacity nothing is written for b, lengths[b] is left
+ * unchanged and the status word records LI_ERR_CAPACITY. */
+LI_API li_status li_append_latent(li_ctx* ctx, const li_cache* cache, const void* h, li_dtype h_dtype,
+                           int d_model, const void* W_down, int T, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* ------------------------------------------------------------- a2: absorb */
+
+/* Query-side decoder absorption (LatentIndex summary, Sec. 3.1, Sec. A.2,
+ * Sec. B.2): for each of n_tok query tokens and H heads,
+ * qt[t][h][i] = sum_j W_K[h][j][i] * q[t][h][j]  (fp32 accumulation) and, if
+ * b_K is given, beta[t][h] = sum_j q[t][h][j] * b_K[h][j].
+ * q       [n_tok][H][d_k] of q_dtype (F32 or BF16).
+ * W_K     decoder of layer l, [d_k][d_c] of q_dtype, row-major (key = W_K c),
+ *         head h at W_K + h * W_K_head_stride elements (0 = shared by all
+ *         heads); or NULL for the identity (d_c == d_k: plain conversion).
+ * b_K     [d_k] fp32 per head at b_K + h * b_K_head_stride, or NULL.
+ * out_dtype F32, BF16 (round-to-nearest-even) or E4M3: then q_abs_scale
+ *         [n_tok][H] receives scale = amax_i |qt| / 448 (1 if 0) and q_abs the
+ *         codes e4m3_satfinite(qt_i / scale).
+ * q_abs   [n_tok][H][d_c] of out_dtype.  beta [n_tok][H] fp32 or NULL.     */
+LI_API li_status li_absorb_query(li_ctx* ctx, const void* q, li_dtype q_dtype, int n_tok, int H, int d_k,
+                          const void* W_K, int64_t W_K_head_stride, const float* b_K,
+                          int64_t b_K_head_stride, int d_c, li_dtype out_dtype, void* q_abs,
+                          float* q_abs_scale, float* beta, void* stream);
+
+/* ------------------------------------------------ a3 + a4: scan and select */
+
+/* Full-prefix LatentIndex scoring and per-layer selection (Sec. 3.1): scores
+ * every valid position of every query with the head-weighted ReLU form, on
+ * tensor cores, without per-head scores leaving the chip, then selects the
+ * top-k per query row.
+ * out_idx   [batch][T][k] int32 (see "Selections").
+ * out_score [batch][T][k] fp32 selected scores, or NULL.
+ * scores_dump [batch][T][capacity] fp32, or NULL: receives every valid score
+ *           (positions past the valid prefix are not written).            */
+LI_API li_status li_score_topk(li_ctx* ctx, const li_cache* cache, const li_query* q, int k,
+                        int32_t* out_idx, float* out_score, float* scores_dump, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------- a5: HS anchor */
+
+/* HS step 1 (Sec. 3.2, Sec. C.4): the anchor scores its full prefix and
+ * proposes cand = its top-B_eff positions, B_eff = min(B, valid length),
+ * ascending, -1 padded, with cand_n = B_eff; anchor_idx = its own top-k of
+ * the same scores (a subset of cand).  Requires B >= k.
+ * cand [batch][T][B], cand_n [batch][T], anchor_idx [batch][T][k] int32;
+ * anchor_score [batch][T][k] fp32 or NULL; scores_dump as li_score_topk. */
+LI_API li_status li_hs_anchor_candidates(li_ctx* ctx, const li_cache* cache, const li_query* q, int B,
+                                  int k, int32_t* cand, int32_t* cand_n, int32_t* anchor_idx,
+                                  float* anchor_score, float* scores_dump, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------- a6: HS follower */
+
+/* HS step 2 (Sec. 3.2, Sec. C.4): a follower layer gathers only the latent
+ * rows cand[b][t][0 .. cand_n[b][t]) (ascending token positions from
+ * li_hs_anchor_candidates of the same step), scores them with its own
+ * absorbed query and selects its own top-min(k, cand_n) by (score desc,
+ * token position asc), written as token positions ascending, -1 padded.
+ * A candidate outside [0, lengths[b]) records LI_ERR_INDEX on the device
+ * and is scored -inf.
+ * scores_dump [batch][T][B] fp32 or NULL: score of candidate j at [..][j]. */
+LI_API li_status li_hs_follower_refine(li_ctx* ctx, const li_cache* cache, const li_query* q,
+                                const int32_t* cand, const int32_t* cand_n, int B, int k,
+                                int32_t* out_idx, float* out_score, float* scores_dump, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------ a7: DSA-style path */
+
+/* DSA-style per-layer comparison path (Sec. 1 and Sec. B.3: native DSA keeps a
+ * key cache per layer and scans the full prefix at every layer): scores the
+ * layer's own key cache (dim = d_k) with the raw query and selects top-k.
+ * Arguments as li_score_topk; key caches are filled with li_append_latent
+ * (W_down = the layer's key projection). */
+LI_API li_status li_dsa_score_topk(li_ctx* ctx, const li_cache* key_cache, const li_query* q, int k,
+                            int32_t* out_idx, float* out_score, float* scores_dump, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------- a4: plain selection */
+
+/* Top-k of `rows` fp32 rows: row r is scores[r * row_stride + 0 .. n_r),
+ * n_r = lengths ? lengths[r] : n (lengths[r] is clamped to [0, n]).
+ * out_idx [rows][k] int32, out_score [rows][k] fp32 or NULL. */
+LI_API li_status li_topk(li_ctx* ctx, const float* scores, int rows, int n, int64_t row_stride,
+                  const int32_t* lengths, int k, int32_t* out_idx, float* out_score, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- profiling */
+
+/* Launch profile: when enabled, every kernel launch (and workspace clear) of
+ * the library is bracketed by CUDA events on the launching stream.
+ * li_profile_read synchronises the recorded events and copies up to `max`
+ * records into the host array `out` (in launch order), returning the number
+ * of records in *count; li_profile_reset clears them.  Profiling adds two
+ * event records per launch and is off by default. */
+typedef struct {
+  char kernel[48];       /* "scan", "gather", "topk_filter", "append_gemv", ...  */
+  float ms;              /* event-timed duration of the launch                   */
+  int32_t grid;          /* CTAs launched (0 when not tracked)                   */
+  int32_t block;         /* threads per CTA                                      */
+  int32_t smem;          /* dynamic shared memory bytes per CTA                  */
+} li_profile_record;
+
+LI_API li_status li_profile_enable(li_ctx* ctx, int enable);
+LI_API li_status li_profile_read(li_ctx* ctx, li_profile_record* out, int max, int* count);
+LI_API li_status li_profile_reset(li_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LI_H */

@@ -1,0 +1,74 @@
+"""li_topk on identical fp32 arrays must match the oracle's sort bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import indexer
+
+pytestmark = pytest.mark.gpu
+li = pytest.importorskip("cross_layer_latent_b200")
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    c = li.Context(0)
+    yield c
+    c.close()
+
+
+def _rows(kind, rows, n, rng):
+    if kind == "gauss":
+        return rng.standard_normal((rows, n)).astype(np.float32)
+    if kind == "ties":        # few distinct values: many ties at the boundary
+        return (rng.integers(-3, 4, (rows, n)) * 0.5).astype(np.float32)
+    if kind == "zeros":       # +0 and -0 everywhere
+        return np.where(rng.random((rows, n)) < 0.5, np.float32(0.0), np.float32(-0.0)).astype(np.float32)
+    if kind == "const":
+        return np.full((rows, n), 1.25, np.float32)
+    if kind == "wide":        # magnitudes across the whole exponent range, both signs, infinities
+        x = rng.standard_normal((rows, n)) * 10.0 ** rng.integers(-30, 30, (rows, n))
+        x[:, ::97] = np.inf
+        x[:, 5::101] = -np.inf
+        return x.astype(np.float32)
+    if kind == "neg":
+        return -np.abs(rng.standard_normal((rows, n))).astype(np.float32)
+    raise ValueError(kind)
+
+
+def _check(ctx, x, k, lengths=None):
+    rows, n = x.shape
+    xd = torch.from_numpy(x).to(DEV)
+    idx = torch.full((rows, k), -7, dtype=torch.int32, device=DEV)
+    val = torch.zeros(rows, k, device=DEV)
+    ws = li.workspace(ctx, rows, 1, n, 1, k)
+    ld = None if lengths is None else torch.from_numpy(lengths.astype(np.int32)).to(DEV)
+    li.li_topk(ctx, xd, k, idx, val, ws, lengths=ld)
+    torch.cuda.synchronize()
+    gi, gv = idx.cpu().numpy(), val.cpu().numpy()
+    for r in range(rows):
+        nr = n if lengths is None else int(np.clip(lengths[r], 0, n))
+        ei, ev = indexer.topk(x[r], k, nr)
+        assert np.array_equal(gi[r], ei), f"row {r}: first difference at {np.argmax(gi[r] != ei)}"
+        keep = ei >= 0
+        assert np.array_equal(gv[r][keep].view(np.uint32), x[r][ei[keep]].view(np.uint32))
+        assert np.all(np.isneginf(gv[r][~keep]))
+
+
+@pytest.mark.parametrize("kind", ["gauss", "ties", "zeros", "const", "wide", "neg"])
+@pytest.mark.parametrize("rows,n,k", [(1, 8192, 2048), (4, 131072, 2048), (3, 1000, 64), (5, 4097, 4097),
+                                      (64, 5000, 100)])
+def test_topk_bit_exact(ctx, kind, rows, n, k):
+    rng = np.random.default_rng(hash((kind, rows, n, k)) % 2 ** 32)
+    _check(ctx, _rows(kind, rows, n, rng), k)
+
+
+def test_topk_ragged_lengths_and_short_rows(ctx):
+    rng = np.random.default_rng(1)
+    x = _rows("ties", 9, 20000, rng)
+    lengths = np.array([0, 1, 5, 63, 64, 65, 4096, 12345, 20000])
+    _check(ctx, x, 64, lengths)
+    _check(ctx, x, 2048, lengths)
