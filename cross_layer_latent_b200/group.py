@@ -57,6 +57,37 @@ class GroupIndexer:
             self.cand_n = torch.zeros(batch, T, dtype=torch.int32, device=dev)
         self.ws = workspace(ctx, batch, T, capacity, H, k, B or 0, device=dev)
 
+    # ------------------------------------------------------------ loading a prefix
+    def load(self, lengths, W_K, q, w, latent=None, hidden=None, W_down=None, q_pos=None, dsa_keys=True):
+        """Fill the caches with a prefix and set every layer's queries.
+
+        lengths [batch] valid rows; latent [batch, >= max(lengths), d_c] fp32
+        (or hidden [batch, ..., d_model] with W_down [d_c, d_model], built into
+        the latent by the library); W_K per layer [d_k, d_c]; q per layer
+        [batch, T, H, d_k]; w per layer [batch, T, H]; q_pos [batch, T] for
+        prefill queries.  Arrays may be NumPy or torch; the DSA key caches (if
+        any) receive key = W_K c, built by the library from the fp32 latent."""
+        dev = self.device
+        as_t = lambda x: torch.as_tensor(x).to(dev)  # noqa: E731
+        lengths = as_t(lengths).to(torch.int32)
+        maxlen = int(lengths.max().item())
+        if hidden is not None:
+            self.append(as_t(hidden)[:, :maxlen].contiguous(), as_t(W_down))
+            c_src = self.latent.data[:, :maxlen].float().contiguous() if self.keys else None
+        else:
+            c_src = as_t(latent)[:, :maxlen].float().contiguous()
+            self.append(c_src)
+        self.set_lengths(lengths)
+        for l, kc in enumerate(self.keys if dsa_keys else []):
+            kc.lengths.zero_()
+            li_append_latent(self.ctx, kc, c_src, as_t(W_K[l]).float().contiguous(), maxlen, self.ws)
+            kc.lengths.copy_(lengths)
+        if q_pos is not None:
+            self.q_pos = as_t(q_pos).to(torch.int32).contiguous()
+        for l in range(self.G):
+            self.set_queries(l, as_t(q[l]).float().contiguous(), as_t(W_K[l]).float().contiguous(),
+                             as_t(w[l]).float().contiguous())
+
     # ------------------------------------------------------------ construction (a1)
     def append(self, h: torch.Tensor, W_down: Optional[torch.Tensor] = None, stream=None):
         """Append T new tokens per sequence to the shared latent cache:

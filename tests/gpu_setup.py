@@ -14,30 +14,8 @@ def build_group(ctx, inp: Inputs, dsa: bool = True, device="cuda:0") -> li.Group
     wl = inp.wl
     g = li.GroupIndexer(ctx, batch=wl.batch, capacity=wl.capacity, d_c=wl.d_c, H=wl.heads, d_k=wl.d_k, G=wl.group,
                         dtype=DTYPE[wl.cache_dtype], k=wl.k, B=wl.B, T=wl.queries, dsa=dsa, device=device)
-    maxlen = int(inp.lengths.max())
-    if inp.hidden is not None:
-        h = torch.from_numpy(inp.hidden[:, :maxlen]).to(device)
-        g.append(h, torch.from_numpy(inp.W_down).to(device))
-    else:
-        g.append(torch.from_numpy(inp.latent[:, :maxlen]).to(device))
-    lengths = torch.from_numpy(inp.lengths).to(device)
-    g.set_lengths(lengths)
-    if dsa:
-        # DSA key caches: key = W_K c from the fp32 latent (the exact one, or the
-        # cache itself when the latent is built from h in fp32)
-        c_src = (g.latent.data[:, :maxlen].float() if inp.hidden is not None
-                 else torch.from_numpy(inp.latent[:, :maxlen]).to(device))
-        for l in range(wl.group):
-            kc = g.keys[l]
-            kc.lengths.zero_()
-            li.li_append_latent(ctx, kc, c_src.contiguous(), torch.from_numpy(inp.W_K[l]).to(device), maxlen,
-                                g.ws)
-            kc.lengths.copy_(lengths)
-    if wl.queries > 1:
-        g.q_pos = torch.from_numpy(inp.q_pos).to(device)
-    for l in range(wl.group):
-        g.set_queries(l, torch.from_numpy(inp.q[l]).to(device), torch.from_numpy(inp.W_K[l]).to(device),
-                      torch.from_numpy(inp.w[l]).to(device))
+    g.load(inp.lengths, inp.W_K, inp.q, inp.w, latent=inp.latent, hidden=inp.hidden, W_down=inp.W_down,
+           q_pos=inp.q_pos)
     torch.cuda.synchronize()
     return g
 
