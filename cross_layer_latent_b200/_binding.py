@@ -77,6 +77,7 @@ _sigs = {
     "li_dsa_score_topk": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _I, _P, _P, _P, _P,
                                _SZ, _P]),
     "li_topk": (_I, [_P, _P, _I, _I, _I64, _P, _I, _P, _P, _P, _SZ, _P]),
+    "li_set_trace": (_I, [_P, _P, _SZ]),
     "li_profile_enable": (_I, [_P, _I]),
     "li_profile_read": (_I, [_P, ctypes.POINTER(c_li_profile_record), _I, ctypes.POINTER(_I)]),
     "li_profile_reset": (_I, [_P]),
@@ -263,6 +264,12 @@ def li_topk(ctx: Context, scores: torch.Tensor, k: int, out_idx: torch.Tensor, o
     n = stride if n is None else n
     ctx.check(_lib.li_topk(ctx.handle, _ptr(scores), rows, int(n), int(scores.stride(0)), _ptr(lengths), int(k),
                            _ptr(out_idx), _ptr(out_score), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def li_set_trace(ctx: Context, buf: Optional[torch.Tensor]):
+    """Diagnostic per-tile trace of the scoring kernels into buf (uint8/int64
+    device tensor of >= 32768 bytes, viewed as [8, 64, 8] int64), or None."""
+    ctx.check(_lib.li_set_trace(ctx.handle, _ptr(buf), 0 if buf is None else buf.numel() * buf.element_size()))
 
 
 def li_profile_enable(ctx: Context, enable: bool = True):

@@ -1,6 +1,7 @@
 """Build libli.so (the sm_100a indexer library) in-tree with nvcc.
 
-Usage: python -m cross_layer_latent_b200.build [--force]
+Usage: python cross_layer_latent_b200/build.py [--force] [--ptxas]
+(run as a script: importing the package loads the library being built)
 Objects go to cross_layer_latent_b200/_build/; the shared library to
 cross_layer_latent_b200/libli.so.  The CUDA runtime is linked statically so
 the library does not depend on the runtime version a host process loads.

@@ -35,6 +35,7 @@ struct li_ctx {
   std::string last_error;
   uint64_t wait_ns = 2000000000ull;
   bool profile = false;
+  uint64_t* trace = nullptr;
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> free_events;
 };
@@ -143,7 +144,8 @@ li_status check_cache(li_ctx* ctx, const li_cache* c, const char* what) {
   if (c->dim < kmul || c->dim > 256 || c->dim % kmul)
     return fail(ctx, LI_ERR_SHAPE, "%s: dim %d must be a multiple of %d in [%d, 256]", what, c->dim, kmul, kmul);
   if (!aligned(c->data, 16)) return fail(ctx, LI_ERR_ALIGN, "%s: cache data not 16-byte aligned", what);
-  if (c->scale && !aligned(c->scale, 4)) return fail(ctx, LI_ERR_ALIGN, "%s: scale not 4-byte aligned", what);
+  if (c->scale && !aligned(c->scale, 16)) return fail(ctx, LI_ERR_ALIGN, "%s: scale not 16-byte aligned", what);
+
   return LI_OK;
 }
 
@@ -224,37 +226,62 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   a.n_kchunks = static_cast<int>(row_bytes / swz);
   a.row_bytes = row_bytes;
   a.cand_stride = cand_stride;
-  a.n_acc = std::min(4, 512 / N);
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(a.n_acc * N)) cols <<= 1;
-  a.tmem_cols = cols;
   const int kind = c->dtype == LI_F32 ? kKindTF32 : (c->dtype == LI_BF16 ? kKindBF16 : kKindE4M3);
   const uint32_t fmt = c->dtype == LI_F32 ? 2u : (c->dtype == LI_BF16 ? 1u : 0u);
-  a.idesc = make_instr_desc(fmt, kTileM, N);
-  a.a_stage_bytes = kTileM * swz;
+  a.idesc = make_instr_desc(fmt, 128, N);
   a.b_slot_bytes = static_cast<uint32_t>(a.n_kchunks) * N * swz;
-  const size_t misc = 640 + 16 + (kMaxSegments + 1) * 4 + 4 * (3 * N + 16) * 4;
+  // Work item of R rows (two M=128 blocks when both accumulators of every
+  // in-flight item fit tensor memory), stage of KS K-chunks: the largest
+  // stage that still leaves a pipeline of several stages.
+  const bool has_meta = gather || c->dtype == LI_E4M3;
+  const size_t fixed_misc = 1024 + 16 + (kMaxSegments + 1) * 4 + 16 + kEpiWarps * (3 * N + 16) * 4;
   const size_t budget = static_cast<size_t>(ctx->max_smem_optin) - 1024;
-  int bslots = 2;
-  if (2 * a.b_slot_bytes + 6 * a.a_stage_bytes + misc > budget) bslots = 1;
-  const int64_t room = static_cast<int64_t>(budget) - static_cast<int64_t>(bslots) * a.b_slot_bytes -
-                       static_cast<int64_t>(misc);
-  const int stages = static_cast<int>(std::min<int64_t>(kMaxStages, room / a.a_stage_bytes));
-  if (stages < (gather ? 6 : 3))
+  const size_t kStageCap = 48 * 1024;
+  bool planned = false;
+  for (int R = (2 * N <= 256 && !gather) ? 256 : 128; R >= 128 && !planned; R -= 128) {
+    const size_t meta = has_meta ? static_cast<size_t>(kMetaSlots) * 8 * R : 0;
+    for (int KS = a.n_kchunks; KS >= 1 && !planned; --KS) {
+      if (a.n_kchunks % KS) continue;
+      const size_t stage = static_cast<size_t>(R) * swz * KS;
+      if (stage > kStageCap && KS > 1) continue;
+      for (int bslots = 2; bslots >= 1 && !planned; --bslots) {
+        const int64_t room = static_cast<int64_t>(budget) - static_cast<int64_t>(bslots) * a.b_slot_bytes -
+                             static_cast<int64_t>(meta + fixed_misc);
+        const int stages = room > 0 ? static_cast<int>(std::min<int64_t>(kMaxStages, room / stage)) : 0;
+        const int need = gather ? 6 : (KS < a.n_kchunks ? 4 : 3);
+        if (stages < need) continue;
+        a.R = R;
+        a.MB = R / 128;
+        a.KS = KS;
+        a.stages_per_item = a.n_kchunks / KS;
+        a.n_stages = stages;
+        a.n_bslots = bslots;
+        a.a_stage_bytes = static_cast<uint32_t>(stage);
+        a.meta_bytes = static_cast<uint32_t>(8 * R);
+        a.misc_offset = static_cast<uint32_t>(stages * stage + bslots * a.b_slot_bytes + meta);
+        a.smem_bytes = static_cast<uint32_t>(std::max<size_t>(1024 + a.misc_offset + fixed_misc, 120 * 1024));
+        planned = true;
+      }
+    }
+  }
+  if (!planned || a.smem_bytes > static_cast<uint32_t>(ctx->max_smem_optin))
     return fail(ctx, LI_ERR_UNSUPPORTED, "%s: operands too large for shared memory (N=%d, dim=%d)", what, N, c->dim);
-  a.n_bslots = bslots;
-  a.n_stages = stages;
-  a.misc_offset = stages * a.a_stage_bytes + bslots * a.b_slot_bytes;
-  a.smem_bytes = static_cast<uint32_t>(std::max<size_t>(1024 + a.misc_offset + misc, 120 * 1024));
+  a.n_acc = std::min(4, 512 / (a.MB * N));
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(a.n_acc * a.MB * N)) cols <<= 1;
+  a.tmem_cols = cols;
   a.wait_ns = ctx->wait_ns;
+  a.trace = ctx->trace;
 
-  // Tensor maps: cache rows and queries.
+  // Tensor maps: cache rows as {chunk elements, rows, chunks} so that one
+  // box carries all KS chunks of R rows in [chunk][row] order, and queries.
   {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c->dim),
-                                static_cast<cuuint64_t>(c->batch) * c->capacity};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(swz / eb), static_cast<cuuint32_t>(kTileM)};
-    li_status s = encode_map(ctx, &a.map_a, c->dtype, 2, c->data, dims, strides, box, swz);
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(swz / eb), static_cast<cuuint64_t>(c->batch) * c->capacity,
+                                static_cast<cuuint64_t>(a.n_kchunks)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(swz)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(swz / eb), static_cast<cuuint32_t>(a.R),
+                               static_cast<cuuint32_t>(a.KS)};
+    li_status s = encode_map(ctx, &a.map_a, c->dtype, 3, c->data, dims, strides, box, swz);
     if (s != LI_OK) return s;
   }
   {
@@ -267,6 +294,10 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
     li_status s = encode_map(ctx, &a.map_b, c->dtype, 3, const_cast<void*>(q->q), dims, strides, box, swz);
     if (s != LI_OK) return s;
   }
+  if (c->dtype == LI_E4M3 && !gather && c->capacity % 4)
+    // the loader copies each tile's 128 scales in 16-byte pieces
+    return fail(ctx, LI_ERR_SHAPE, "%s: scanning an E4M3 cache needs capacity %% 4 == 0 (got %d)", what,
+                c->capacity);
   a.cache = static_cast<const uint8_t*>(c->data);
   a.cache_scale = c->dtype == LI_E4M3 ? c->scale : nullptr;
   a.lengths = c->lengths;
@@ -275,12 +306,13 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   a.q_scale = q->dtype == LI_E4M3 ? q->q_scale : nullptr;
   a.beta = q->beta;
   P->kind = kind;
-  const int64_t tiles_per_seg = (static_cast<int64_t>(gather ? cand_stride : c->capacity) + kTileM - 1) / kTileM;
+  const int64_t tiles_per_seg = (static_cast<int64_t>(gather ? cand_stride : c->capacity) + a.R - 1) / a.R;
   P->grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ctx->num_sms, n_seg * tiles_per_seg)));
   return LI_OK;
 }
 
 li_status run_scan(li_ctx* ctx, ScanPlan& P, bool gather, cudaStream_t st) {
+  (void)cudaGetLastError();   // do not blame this launch for an earlier, unrelated error
   Launch L(ctx, st, gather ? "gather" : "scan", P.grid, kScanThreads, static_cast<int>(P.a.smem_bytes));
   const cudaError_t e = launch_scan_kernel(P.kind, gather, P.a, P.grid, st);
   L.done();
@@ -305,7 +337,7 @@ li_status clear_select_state(li_ctx* ctx, void* ws, const WsLayout& L, int64_t r
   return memset_async(ctx, at<uint8_t>(ws, L.rowinfo), rows * 16 * 4, st);
 }
 
-li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaStream_t st) {
+li_status run_topk_chunked(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaStream_t st) {
   t.hist = at<unsigned int>(ws, L.hist);
   t.rowinfo = at<int>(ws, L.rowinfo);
   t.chunk_gt = at<int>(ws, L.chunk_gt);
@@ -323,6 +355,44 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
     const cudaError_t e = launch_topk_stage(stage, t, st);
     Lc.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, names[stage]);
+  }
+  return LI_OK;
+}
+
+// One selection (and optionally a second budget k2 <= k over the same rows):
+// the single-launch cluster kernel when the rows fit it, else the chunked
+// multi-kernel path (which needs its histogram and row state cleared).
+li_status run_topk(li_ctx* ctx, TopkArgs& t, const TopkOut2& o2, void* ws, const WsLayout& L, cudaStream_t st) {
+  // workspace regions used by either path (the cluster kernel compacts its
+  // boundary-bucket keys into `cand`)
+  t.hist = at<unsigned int>(ws, L.hist);
+  t.rowinfo = at<int>(ws, L.rowinfo);
+  t.chunk_gt = at<int>(ws, L.chunk_gt);
+  t.chunk_off = at<int>(ws, L.chunk_off);
+  t.cand = at<uint2>(ws, L.cand);
+  if (static_cast<int64_t>(t.rows) * t.n > static_cast<int64_t>((L.scores - L.cand) / 8))
+    return fail(ctx, LI_ERR_WORKSPACE, "selection of %d x %d exceeds the workspace candidate buffer", t.rows, t.n);
+  if (t.n <= kClusterMaxN && t.rows <= 65535) {
+    int cs = 0;
+    Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);
+    const cudaError_t e = launch_topk_cluster(t, o2, st, &cs);
+    Lc.grid = cs * t.rows;
+    Lc.done();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster");
+    return LI_OK;
+  }
+  li_status s = clear_select_state(ctx, ws, L, t.rows, st);
+  if (s != LI_OK) return s;
+  t.hist_ready = false;
+  if ((s = run_topk_chunked(ctx, t, ws, L, st)) != LI_OK) return s;
+  if (o2.k2 > 0) {
+    TopkArgs t2 = t;
+    t2.k = o2.k2;
+    t2.out_idx = o2.out_idx2;
+    t2.out_score = o2.out_score2;
+    t2.out_count = nullptr;
+    if ((s = clear_select_state(ctx, ws, L, t.rows, st)) != LI_OK) return s;
+    return run_topk_chunked(ctx, t2, ws, L, st);
   }
   return LI_OK;
 }
@@ -358,8 +428,6 @@ li_status score_topk_impl(li_ctx* ctx, const li_cache* c, const li_query* q, int
   P.a.scores = scores;
   P.a.score_stride = c->capacity;
   P.a.status = at<int>(ws, L.status);
-  P.a.hist = at<unsigned int>(ws, L.hist);
-  if ((s = clear_select_state(ctx, ws, L, rows, st)) != LI_OK) return s;
   if ((s = run_scan(ctx, P, false, st)) != LI_OK) return s;
   TopkArgs t = topk_args(scores, c->capacity, static_cast<int>(rows), c->capacity, k);
   t.lengths = c->lengths;
@@ -367,8 +435,7 @@ li_status score_topk_impl(li_ctx* ctx, const li_cache* c, const li_query* q, int
   t.q_pos = q->q_pos;
   t.out_idx = out_idx;
   t.out_score = out_score;
-  t.hist_ready = true;
-  return run_topk(ctx, t, ws, L, st);
+  return run_topk(ctx, t, TopkOut2{0, nullptr, nullptr}, ws, L, st);
 }
 
 }  // namespace
@@ -479,6 +546,7 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
   if (W_down) {
     if (h_dtype != LI_F32 && h_dtype != LI_BF16) return fail(c, LI_ERR_DTYPE, "%s: h must be F32 or BF16", what);
     if (d_model < 8 || d_model % 8) return fail(c, LI_ERR_SHAPE, "%s: d_model must be a multiple of 8", what);
+    if (!aligned(h, 16) || !aligned(W_down, 16)) return fail(c, LI_ERR_ALIGN, "%s: h and W_down must be 16-byte aligned", what);
   } else if (h_dtype != LI_F32) {
     return fail(c, LI_ERR_DTYPE, "%s: without W_down, h must be the F32 latent", what);
   }
@@ -491,7 +559,7 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
   if (!W_down) {
     // h already holds the fp32 rows [batch][T][dim]: quantise and store.
     Launch Ls(c, st, "append_store", 0, 256, 0);
-    const cudaError_t e = launch_append_store(static_cast<const float*>(h), dim, cache->batch, T, 0, T, true,
+    const cudaError_t e = launch_append_store(static_cast<const float*>(h), dim, 0, 1, cache->batch, T, 0, T, true,
                                               cache->data, cache->scale, cache->lengths, cache->capacity, dim,
                                               cache->dtype, done, status, st);
     Ls.done();
@@ -503,24 +571,28 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
   const int tchunk = std::max(1, std::min(T, kAppendChunkTok / cache->batch));
   for (int t0 = 0; t0 < T; t0 += tchunk) {
     const int tn = std::min(tchunk, T - t0);
+    int splits = 1;
     if (tn == T) {
       // every token of the batch at once: h rows are contiguous
       Launch Lg(c, st, "append_gemv", 0, 256, 0);
-      const cudaError_t e = launch_append_gemv(h, h_dtype, W_down, d_model, dim, cache->batch * T, tmp, st);
+      splits = gemv_splits(d_model, cache->batch * T);
+      const cudaError_t e = launch_append_gemv(h, h_dtype, W_down, d_model, dim, cache->batch * T, splits, tmp, st);
       Lg.done();
       if (e != cudaSuccess) return cuda_fail(c, e, "append gemv launch");
     } else {
       for (int b = 0; b < cache->batch; ++b) {
         const uint8_t* hb = static_cast<const uint8_t*>(h) + (static_cast<int64_t>(b) * T + t0) * d_model * eb;
         Launch Lg(c, st, "append_gemv", 0, 256, 0);
-        const cudaError_t e = launch_append_gemv(hb, h_dtype, W_down, d_model, dim, tn,
+        splits = 1;
+        const cudaError_t e = launch_append_gemv(hb, h_dtype, W_down, d_model, dim, tn, 1,
                                                  tmp + static_cast<int64_t>(b) * tn * dim, st);
         Lg.done();
         if (e != cudaSuccess) return cuda_fail(c, e, "append gemv launch");
       }
     }
     Launch Ls(c, st, "append_store", 0, 256, 0);
-    const cudaError_t e = launch_append_store(tmp, dim, cache->batch, tn, t0, T, t0 + tn >= T, cache->data,
+    const cudaError_t e = launch_append_store(tmp, dim, static_cast<int64_t>(cache->batch) * tn * dim, splits,
+                                              cache->batch, tn, t0, T, t0 + tn >= T, cache->data,
                                               cache->scale, cache->lengths, cache->capacity, dim, cache->dtype,
                                               done, status, st);
     Ls.done();
@@ -586,31 +658,16 @@ li_status li_hs_anchor_candidates(li_ctx* c, const li_cache* cache, const li_que
   P.a.scores = scores;
   P.a.score_stride = cache->capacity;
   P.a.status = at<int>(ws, L.status);
-  P.a.hist = at<unsigned int>(ws, L.hist);
-  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
   if ((s = run_scan(c, P, false, st)) != LI_OK) return s;
-  // candidates: top-B of the full prefix, with their scores
-  float* cscores = at<float>(ws, L.cand_scores);
+  // candidates = top-B of the full prefix, and in the same selection launch
+  // the anchor's own top-k (the top-k under the same order is a subset)
   TopkArgs t = topk_args(scores, cache->capacity, static_cast<int>(rows), cache->capacity, B);
   t.lengths = cache->lengths;
   t.len_div = q->T;
   t.q_pos = q->q_pos;
   t.out_idx = cand;
-  t.out_score = cscores;
   t.out_count = cand_n;
-  t.hist_ready = true;
-  if ((s = run_topk(c, t, ws, L, st)) != LI_OK) return s;
-  // the anchor's own selection: top-k of the candidates (the top-k of the
-  // prefix under the same order is a prefix of its top-B)
-  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
-  TopkArgs t2 = topk_args(cscores, B, static_cast<int>(rows), B, k);
-  t2.lengths = cand_n;
-  t2.len_div = 1;
-  t2.idx_map = cand;
-  t2.map_stride = B;
-  t2.out_idx = anchor_idx;
-  t2.out_score = anchor_score;
-  return run_topk(c, t2, ws, L, st);
+  return run_topk(c, t, TopkOut2{k, anchor_idx, anchor_score}, ws, L, st);
 }
 
 li_status li_hs_follower_refine(li_ctx* c, const li_cache* cache, const li_query* q, const int32_t* cand,
@@ -633,10 +690,8 @@ li_status li_hs_follower_refine(li_ctx* c, const li_cache* cache, const li_query
   P.a.scores = scores;
   P.a.score_stride = B;
   P.a.status = at<int>(ws, L.status);
-  P.a.hist = at<unsigned int>(ws, L.hist);
   P.a.cand = cand;
   P.a.cand_n = cand_n;
-  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
   if ((s = run_scan(c, P, true, st)) != LI_OK) return s;
   TopkArgs t = topk_args(scores, B, static_cast<int>(rows), B, k);
   t.lengths = cand_n;
@@ -645,8 +700,7 @@ li_status li_hs_follower_refine(li_ctx* c, const li_cache* cache, const li_query
   t.map_stride = B;
   t.out_idx = out_idx;
   t.out_score = out_score;
-  t.hist_ready = true;
-  return run_topk(c, t, ws, L, st);
+  return run_topk(c, t, TopkOut2{0, nullptr, nullptr}, ws, L, st);
 }
 
 li_status li_topk(li_ctx* c, const float* scores, int rows, int n, int64_t row_stride, const int32_t* lengths,
@@ -660,12 +714,20 @@ li_status li_topk(li_ctx* c, const float* scores, int rows, int n, int64_t row_s
   li_status s = check_ws(c, ws, ws_bytes, L, what);
   if (s != LI_OK) return s;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = clear_select_state(c, ws, L, rows, st)) != LI_OK) return s;
   TopkArgs t = topk_args(scores, row_stride, rows, n, k);
   t.lengths = lengths;
   t.out_idx = out_idx;
   t.out_score = out_score;
-  return run_topk(c, t, ws, L, st);
+  return run_topk(c, t, TopkOut2{0, nullptr, nullptr}, ws, L, st);
+}
+
+li_status li_set_trace(li_ctx* c, void* buf, size_t bytes) {
+  if (!c) return LI_ERR_ARG;
+  if (buf && bytes < static_cast<size_t>(kTraceCtas) * kTraceTiles * kTraceEvents * 8)
+    return fail(c, LI_ERR_WORKSPACE, "li_set_trace: buffer of %zu bytes, %zu needed", bytes,
+                static_cast<size_t>(kTraceCtas) * kTraceTiles * kTraceEvents * 8);
+  c->trace = static_cast<uint64_t*>(buf);
+  return LI_OK;
 }
 
 li_status li_profile_enable(li_ctx* c, int enable) {

@@ -19,44 +19,65 @@ namespace li {
 
 namespace {
 
-__device__ __forceinline__ float load_elt(const void* p, int64_t i, int dtype) {
-  return dtype == LI_BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i])
-                          : reinterpret_cast<const float*>(p)[i];
-}
-
 __device__ __forceinline__ uint8_t to_e4m3(float x) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
 }
 
 constexpr int kGemvTok = 8;    // tokens per warp task
+constexpr int kMaxSplits = 32; // reduction splits of the construction GEMV
 constexpr int kGemvWarps = 8;
 
-// out[m][j] = sum_i W[j][i] * h[m][i]; one warp per output j and 8 tokens.
-// Lanes stride the reduction dimension by 8 elements (16 B of bf16), then a
-// fixed butterfly sums the lanes.
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(b[e]);
+    v[2 * e] = f.x;
+    v[2 * e + 1] = f.y;
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Split-K GEMV: partial[s][m][j] = sum_{i in split s} W[j][i] * h[m][i].  One
+// warp per (output j, split s, 8 tokens); lanes take 8 consecutive elements
+// (16-byte loads) at a stride of 256, then a fixed butterfly sums the lanes.
+// The store kernel adds the splits in order, so results are deterministic.
 template <typename T>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const T* __restrict__ h,
                                                                const T* __restrict__ W, int d_model,
-                                                               int dim, int n_tok, float* __restrict__ out) {
+                                                               int dim, int n_tok, int splits,
+                                                               float* __restrict__ out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * kGemvWarps + warp;
+  const int task = blockIdx.x * kGemvWarps + warp;
+  if (task >= dim * splits) return;
+  const int j = task / splits, sp = task % splits;
   const int m0 = blockIdx.y * kGemvTok;
-  if (j >= dim) return;
   const int nm = min(kGemvTok, n_tok - m0);
+  const int len = d_model / splits;
+  const int i0 = sp * len, i1 = i0 + len;
   float acc[kGemvTok];
 #pragma unroll
   for (int t = 0; t < kGemvTok; ++t) acc[t] = 0.f;
   const T* wrow = W + static_cast<int64_t>(j) * d_model;
-  for (int i = lane * 8; i < d_model; i += 256) {
+  for (int i = i0 + lane * 8; i < i1; i += 256) {
     float wv[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) wv[e] = static_cast<float>(wrow[i + e]);
+    load8<T>(wrow + i, wv);
 #pragma unroll
     for (int t = 0; t < kGemvTok; ++t) {
       if (t < nm) {
-        const T* hr = h + static_cast<int64_t>(m0 + t) * d_model + i;
+        float hv[8];
+        load8<T>(h + static_cast<int64_t>(m0 + t) * d_model + i, hv);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[t] = fmaf(wv[e], static_cast<float>(hr[e]), acc[t]);
+        for (int e = 0; e < 8; ++e) acc[t] = fmaf(wv[e], hv[e], acc[t]);
       }
     }
   }
@@ -66,13 +87,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const T* __restri
     for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
   }
   if (lane == 0)
-    for (int t = 0; t < nm; ++t) out[static_cast<int64_t>(m0 + t) * dim + j] = acc[t];
+    for (int t = 0; t < nm; ++t)
+      out[(static_cast<int64_t>(sp) * n_tok + m0 + t) * dim + j] = acc[t];
 }
 
 // One warp per new token: write c (fp32 rows) into the cache at row
 // lengths[b] + t0 + t in the cache dtype.  The last block to finish advances
 // lengths[b] by T_total when `bump` is set (all blocks read lengths first).
 __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c, int64_t c_tok_stride,
+                                                    int64_t split_stride, int splits,
                                                     int batch, int T_chunk, int t0, int T_total, int bump,
                                                     void* data, float* scale, int32_t* lengths,
                                                     int capacity, int dim, int dtype,
@@ -92,7 +115,18 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int i = lane + 32 * e;
-        v[e] = i < dim ? src[i] : 0.f;
+        float x = 0.f;
+        if (i < dim) {
+          // all partial sums in flight at once, then added in split order
+          float part[kMaxSplits];
+#pragma unroll
+          for (int sp = 0; sp < kMaxSplits; ++sp) part[sp] = sp < splits ? src[sp * split_stride + i] : 0.f;
+          x = part[0];
+#pragma unroll
+          for (int sp = 1; sp < kMaxSplits; ++sp)
+            if (sp < splits) x += part[sp];
+        }
+        v[e] = x;
         amax = fmaxf(amax, fabsf(v[e]));
       }
       if (dtype == LI_F32) {
@@ -134,12 +168,19 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
   }
 }
 
-constexpr int kAbsorbHeads = 8;
+constexpr int kAbsorbHeads = 2;
 
-// Block per (token, 8 heads); thread i computes output element i of the 8
+template <typename T>
+__device__ __forceinline__ float to_f(T x) { return static_cast<float>(x); }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Block per (token, 2 heads); thread i computes output element i of both
 // absorbed heads: qt[h][i] = sum_j W[h][j][i] q[h][j] (j ascending, fp32).
-__global__ void __launch_bounds__(256) absorb_kernel(const void* __restrict__ q, int q_dtype, int H, int d_k,
-                                                     const void* __restrict__ W, int64_t W_hs,
+// The decoder is read in column order (coalesced over i), 8 rows per step.
+template <typename T>
+__global__ void __launch_bounds__(256) absorb_kernel(const T* __restrict__ q, int H, int d_k,
+                                                     const T* __restrict__ W, int64_t W_hs,
                                                      const float* __restrict__ bK, int64_t b_hs, int d_c,
                                                      int out_dtype, void* q_abs, float* q_abs_scale,
                                                      float* beta) {
@@ -149,7 +190,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(const void* __restrict__ q,
   const int nh = min(kAbsorbHeads, H - h0);
   for (int x = threadIdx.x; x < kAbsorbHeads * d_k; x += blockDim.x) {
     const int hh = x / d_k, jj = x % d_k;
-    qs[hh][jj] = hh < nh ? load_elt(q, (static_cast<int64_t>(t) * H + h0 + hh) * d_k + jj, q_dtype) : 0.f;
+    qs[hh][jj] = hh < nh ? to_f(q[(static_cast<int64_t>(t) * H + h0 + hh) * d_k + jj]) : 0.f;
   }
   __syncthreads();
   const int i = threadIdx.x;
@@ -160,18 +201,33 @@ __global__ void __launch_bounds__(256) absorb_kernel(const void* __restrict__ q,
     if (W == nullptr) {
 #pragma unroll
       for (int hh = 0; hh < kAbsorbHeads; ++hh) acc[hh] = qs[hh][i];
-    } else if (W_hs == 0) {
-      for (int j = 0; j < d_k; ++j) {
-        const float wv = load_elt(W, static_cast<int64_t>(j) * d_c + i, q_dtype);
-#pragma unroll
-        for (int hh = 0; hh < kAbsorbHeads; ++hh) acc[hh] = fmaf(wv, qs[hh][j], acc[hh]);
-      }
     } else {
-      for (int j = 0; j < d_k; ++j) {
 #pragma unroll
-        for (int hh = 0; hh < kAbsorbHeads; ++hh) {
-          if (hh < nh) {
-            const float wv = load_elt(W, (h0 + hh) * W_hs + static_cast<int64_t>(j) * d_c + i, q_dtype);
+      for (int hh = 0; hh < kAbsorbHeads; ++hh) {
+        if (hh >= nh) break;
+        if (hh > 0 && W_hs == 0) break;      // shared decoder: handled below with one read
+        const T* Wh = W + (h0 + hh) * W_hs + i;
+        int j = 0;
+        for (; j + 8 <= d_k; j += 8) {
+          float wv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) wv[u] = to_f(Wh[static_cast<int64_t>(j + u) * d_c]);
+          if (W_hs == 0) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+              for (int h2 = 0; h2 < kAbsorbHeads; ++h2) acc[h2] = fmaf(wv[u], qs[h2][j + u], acc[h2]);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[hh] = fmaf(wv[u], qs[hh][j + u], acc[hh]);
+          }
+        }
+        for (; j < d_k; ++j) {
+          const float wv = to_f(Wh[static_cast<int64_t>(j) * d_c]);
+          if (W_hs == 0) {
+#pragma unroll
+            for (int h2 = 0; h2 < kAbsorbHeads; ++h2) acc[h2] = fmaf(wv, qs[h2][j], acc[h2]);
+          } else {
             acc[hh] = fmaf(wv, qs[hh][j], acc[hh]);
           }
         }
@@ -215,28 +271,38 @@ __global__ void __launch_bounds__(256) absorb_kernel(const void* __restrict__ q,
 
 }  // namespace
 
+int gemv_splits(int d_model, int n_tok) {
+  // decode: enough warps that each reads one 256-element slice of a W row
+  if (n_tok > 64) return 1;
+  for (int sp = kMaxSplits; sp > 1; --sp)
+    if (d_model % (8 * sp) == 0 && d_model / sp >= 256 && (d_model / sp) % 256 == 0) return sp;
+  for (int sp = kMaxSplits; sp > 1; --sp)
+    if (d_model % (8 * sp) == 0 && d_model / sp >= 256) return sp;
+  return 1;
+}
+
 cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_model, int dim, int n_tok,
-                               float* out, cudaStream_t st) {
-  const dim3 grid((dim + kGemvWarps - 1) / kGemvWarps, (n_tok + kGemvTok - 1) / kGemvTok);
+                               int splits, float* out, cudaStream_t st) {
+  const dim3 grid((dim * splits + kGemvWarps - 1) / kGemvWarps, (n_tok + kGemvTok - 1) / kGemvTok);
   if (h_dtype == LI_BF16)
     gemv_kernel<__nv_bfloat16><<<grid, kGemvWarps * 32, 0, st>>>(
         reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim,
-        n_tok, out);
+        n_tok, splits, out);
   else
     gemv_kernel<float><<<grid, kGemvWarps * 32, 0, st>>>(reinterpret_cast<const float*>(h),
                                                           reinterpret_cast<const float*>(W), d_model, dim,
-                                                          n_tok, out);
+                                                          n_tok, splits, out);
   return cudaGetLastError();
 }
 
-cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int batch, int T_chunk, int t0,
-                                int T_total, bool bump, void* data, float* scale, int32_t* lengths,
-                                int capacity, int dim, int dtype, unsigned int* done_counter, int* status,
-                                cudaStream_t st) {
+cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits, int batch,
+                                int T_chunk, int t0, int T_total, bool bump, void* data, float* scale,
+                                int32_t* lengths, int capacity, int dim, int dtype, unsigned int* done_counter,
+                                int* status, cudaStream_t st) {
   const int n_tok = batch * T_chunk;
   const int grid = (n_tok + 7) / 8;
-  store_kernel<<<grid, 256, 0, st>>>(c, c_tok_stride, batch, T_chunk, t0, T_total, bump ? 1 : 0, data, scale,
-                                     lengths, capacity, dim, dtype, done_counter, status);
+  store_kernel<<<grid, 256, 0, st>>>(c, c_tok_stride, split_stride, splits, batch, T_chunk, t0, T_total,
+                                     bump ? 1 : 0, data, scale, lengths, capacity, dim, dtype, done_counter, status);
   return cudaGetLastError();
 }
 
@@ -244,8 +310,14 @@ cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
                           int out_dtype, void* q_abs, float* q_abs_scale, float* beta, cudaStream_t st) {
   const dim3 grid((H + kAbsorbHeads - 1) / kAbsorbHeads, n_tok);
-  absorb_kernel<<<grid, 256, 0, st>>>(q, q_dtype, H, d_k, W, W_head_stride, b, b_head_stride, d_c, out_dtype,
-                                      q_abs, q_abs_scale, beta);
+  if (q_dtype == LI_BF16)
+    absorb_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), H, d_k,
+                                                       reinterpret_cast<const __nv_bfloat16*>(W), W_head_stride, b,
+                                                       b_head_stride, d_c, out_dtype, q_abs, q_abs_scale, beta);
+  else
+    absorb_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(q), H, d_k,
+                                               reinterpret_cast<const float*>(W), W_head_stride, b, b_head_stride,
+                                               d_c, out_dtype, q_abs, q_abs_scale, beta);
   return cudaGetLastError();
 }
 

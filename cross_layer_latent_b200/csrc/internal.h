@@ -10,7 +10,10 @@
 namespace li {
 
 constexpr int kTileM = 128;          // cache rows per MMA tile (UMMA M)
-constexpr int kScanThreads = 192;    // warp 0 loads, warp 1 issues MMAs, warps 2..5 epilogue
+constexpr int kEpiWarps = 8;         // two epilogue warpgroups, alternating tiles
+constexpr int kScanThreads = 64 + 32 * kEpiWarps;   // warp 0 loads, warp 1 issues MMAs
+constexpr int kMetaSlots = 8;        // ring of per-item row metadata (fp8 scales, gathered rows)
+constexpr int kMaxItemRows = 256;    // rows of one work item (two M=128 MMA blocks)
 constexpr int kMaxSegments = 1024;   // (sequence, query group) segments per scan launch
 constexpr int kMaxStages = 32;
 constexpr int kHistBins = 2048;      // first radix digit: key bits 31..21
@@ -18,7 +21,7 @@ constexpr int kHistBins = 2048;      // first radix digit: key bits 31..21
 // Arguments of the scoring kernel (scan of whole prefixes, or gather of
 // candidate rows).  Tensor maps first: they must stay 64-byte aligned.
 struct alignas(64) ScanArgs {
-  CUtensorMap map_a;          // cache rows: dims {dim, batch*capacity}, box {swz/elt, 128}
+  CUtensorMap map_a;          // cache rows: dims {swz/elt, batch*capacity, n_kchunks}, box {swz/elt, R, KS}
   CUtensorMap map_b;          // queries: dims {dim, H, batch*T}, box {swz/elt, H_pad, Qg}
   const uint8_t* cache;       // cache data (gather loads)
   const float* cache_scale;   // [batch*capacity] or null
@@ -30,7 +33,6 @@ struct alignas(64) ScanArgs {
   const int* cand;            // gather: [batch*T][cand_stride]
   const int* cand_n;          // gather: [batch*T]
   float* scores;              // [batch*T][score_stride]
-  unsigned int* hist;         // fused first-digit histogram [batch*T][2048] or null
   int* status;
   int64_t score_stride;
   int64_t row_bytes;
@@ -38,11 +40,21 @@ struct alignas(64) ScanArgs {
   int batch, capacity, T, H, H_pad, Qg, n_groups, N;
   int cand_stride;
   int swz, n_kchunks, elt_bytes;
+  int R, MB;                  // rows per work item (128 or 256) and M=128 blocks per item
+  int KS, stages_per_item;    // K-chunks per stage, stages per item
   int n_stages, n_bslots, n_acc;
   uint32_t tmem_cols, idesc;
-  uint32_t a_stage_bytes, b_slot_bytes, misc_offset, smem_bytes;
+  uint32_t a_stage_bytes, b_slot_bytes, meta_bytes, misc_offset, smem_bytes;
   int n_segments;
+  uint64_t* trace;            // per-tile event times of the first kTraceCtas CTAs, or null
 };
+
+// Diagnostic tile trace: [kTraceCtas][kTraceTiles][kTraceEvents] SM clock
+// cycles (comparable within one CTA).  Events: 0 producer has the first stage of the tile, 1 producer issued
+// the last stage, 2 MMA saw the first stage full, 3 MMA committed the tile,
+// 4 epilogue saw the accumulator full, 5 epilogue released it, 6 MMA issuer
+// started waiting for the first stage, 7 epilogue finished its head sums.
+constexpr int kTraceCtas = 8, kTraceTiles = 64, kTraceEvents = 8;
 
 // Kernel families (for the launch profile).
 enum KernelKind { kKScan = 0, kKGather, kKTopkHist, kKTopkFilter, kKTopkSelect, kKTopkEmit,
@@ -76,6 +88,20 @@ struct TopkArgs {
   bool hist_ready;            // first-digit histogram already accumulated (fused)
 };
 
+// Single-launch selection for rows of up to kClusterMaxN positions: one
+// thread-block cluster per row, keys held in registers, digit histograms
+// summed across the cluster in distributed shared memory.  A second budget
+// k2 <= k (out_idx2 / out_score2) can be selected in the same launch.
+constexpr int kClusterThreads = 512;
+constexpr int kClusterMaxSize = 8;
+constexpr int kClusterMaxN = kClusterThreads * 32 * kClusterMaxSize;   // 131072
+struct TopkOut2 {
+  int k2;                     // 0: no second selection
+  int32_t* out_idx2;
+  float* out_score2;
+};
+cudaError_t launch_topk_cluster(const TopkArgs& a, const TopkOut2& o2, cudaStream_t st, int* cluster_size);
+
 constexpr int kTopkChunk = 4096;
 constexpr int kTopkThreads = 256;
 constexpr int kMaxTopkChunks = 8192;
@@ -88,12 +114,14 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st);
 
 // ---- construction
 
+// Split count of the construction GEMV for n_tok tokens of width d_model.
+int gemv_splits(int d_model, int n_tok);
 cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_model, int dim,
-                               int n_tok, float* out, cudaStream_t st);
-cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int batch, int T_chunk, int t0,
-                                int T_total, bool bump, void* data, float* scale, int32_t* lengths,
-                                int capacity, int dim, int dtype, unsigned int* done_counter,
-                                int* status, cudaStream_t st);
+                               int n_tok, int splits, float* out, cudaStream_t st);
+cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits,
+                                int batch, int T_chunk, int t0, int T_total, bool bump, void* data,
+                                float* scale, int32_t* lengths, int capacity, int dim, int dtype,
+                                unsigned int* done_counter, int* status, cudaStream_t st);
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
                           int out_dtype, void* q_abs, float* q_abs_scale, float* beta,

@@ -5,19 +5,29 @@
 //     score(t, s) = sum_h w_{t,h} * max(0, qt_{t,h} . c_s + beta_{t,h})
 // (LatentIndex summary, Sec. 3.1: absorbed queries score the shared latent
 // directly; Sec. 3.2 / C.4: HS followers rescore only the anchor's
-// candidates).  The per-head dot products are one tensor-core contraction
-// per 128-row tile: A = 128 cache rows x dim (K-major, swizzled smem, loaded
-// by TMA or gathered by cp.async), B = Qg queries x H_pad heads x dim, D =
-// 128 x N fp32 in tensor memory.  An epilogue warpgroup reads D lane by lane
-// (one cached row per thread), applies ReLU, the head weights and the
-// per-token / per-head fp8 scales, reduces over heads and writes one fp32
-// score per (query, row); per-head scores never leave the SM.
+// candidates).  The per-head dot products are tensor-core contractions:
+// A = 128 cache rows x dim (K-major, swizzled smem), B = Qg queries x H_pad
+// heads x dim, D = 128 x N fp32 in tensor memory.  Epilogue warps read D lane
+// by lane (one cached row per thread), apply ReLU, the head weights and the
+// per-token / per-head fp8 scales, reduce over heads and write one fp32 score
+// per (query, row); per-head scores never leave the SM.
 //
-// Warp roles (192 threads): warp 0 loads (TMA, or 32-lane cp.async gather),
-// warp 1 allocates tensor memory and issues the MMAs, warps 2..5 run the
-// epilogue.  Each CTA is persistent over a contiguous range of work items
-// (segment, tile); a segment is one (sequence, query group) of the scan or
-// one (sequence, query) of the gather.  All waits are bounded.
+// Work is cut into items of R = 128 or 256 rows (one or two M=128 MMA
+// blocks).  A pipeline stage holds KS K-chunks of an item's R rows, loaded by
+// ONE 3-D TMA box ({chunk bytes, rows, chunks}, smem order [chunk][row]) or
+// gathered by cp.async; decode items use one stage per item.  The control
+// paths are single-lane dependency chains whose every step (mbarrier wait,
+// MMA issue, shared load) costs on the order of 100 cycles, so each step is
+// made to move as many bytes as the shared-memory budget allows.
+//
+// Warp roles (64 + 32 * kEpiWarps threads): warp 0 loads (one lane issues
+// TMA; all 32 lanes gather), warp 1 allocates tensor memory and one lane
+// issues the MMAs, and two epilogue warpgroups take the two M blocks of an
+// item (R = 256) or alternate items (R = 128).  Per-item row metadata (fp8
+// per-token scales, gathered token ids) travels through its own ring.  Each
+// CTA is persistent over a contiguous range of items; a segment is one
+// (sequence, query group) of the scan or one (sequence, query) of the gather.
+// Every wait is bounded; ring positions advance without integer division.
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -30,23 +40,27 @@ constexpr uint64_t kDrainNs = 200ull * 1000ull * 1000ull;   // 0.2 s
 struct ScanSmem {
   uint8_t* a_stages;
   uint8_t* b_slots;
+  uint8_t* meta;        // kMetaSlots x meta_bytes: scale[R] then tok[R]
   uint64_t* full;
   uint64_t* empty;
   uint64_t* bfull;
   uint64_t* bempty;
   uint64_t* accfull;
   uint64_t* accempty;
+  uint64_t* mfull;
+  uint64_t* mempty;
   uint64_t* drain;
   uint32_t* tmem_base;
   int* abort_flag;
   int* prefix;          // [kMaxSegments + 1]
-  float* ep;            // 4 warps x (3 * N + 16) floats
+  float* ep;            // kEpiWarps x (3 * N + 16) floats
 };
 
 __device__ __forceinline__ ScanSmem carve(uint8_t* base, const ScanArgs& a) {
   ScanSmem s;
   s.a_stages = base;
   s.b_slots = base + static_cast<size_t>(a.n_stages) * a.a_stage_bytes;
+  s.meta = s.b_slots + static_cast<size_t>(a.n_bslots) * a.b_slot_bytes;
   uint8_t* p = base + a.misc_offset;
   s.full = reinterpret_cast<uint64_t*>(p);
   s.empty = s.full + kMaxStages;
@@ -54,21 +68,24 @@ __device__ __forceinline__ ScanSmem carve(uint8_t* base, const ScanArgs& a) {
   s.bempty = s.bfull + 2;
   s.accfull = s.bempty + 2;
   s.accempty = s.accfull + 4;
-  s.drain = s.accempty + 4;
+  s.mfull = s.accempty + 4;
+  s.mempty = s.mfull + kMetaSlots;
+  s.drain = s.mempty + kMetaSlots;
   s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 1);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
-  s.prefix = s.abort_flag + 3;
-  s.ep = reinterpret_cast<float*>(s.prefix + kMaxSegments + 1);
+  s.prefix = s.abort_flag + 2;
+  // 16-byte aligned parameter arrays (read four at a time)
+  s.ep = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s.prefix + kMaxSegments + 1) + 15) & ~uintptr_t(15));
   return s;
 }
 
-// Number of 128-row tiles a segment needs.
+// Number of R-row items a segment needs.
 template <bool GATHER>
-__device__ __forceinline__ int segment_tiles(const ScanArgs& a, int seg) {
+__device__ __forceinline__ int segment_items(const ScanArgs& a, int seg) {
   if (GATHER) {
     int n = a.cand_n[seg];
     n = n < 0 ? 0 : (n > a.cand_stride ? a.cand_stride : n);
-    return (n + kTileM - 1) / kTileM;
+    return (n + a.R - 1) / a.R;
   }
   const int b = seg / a.n_groups, g = seg % a.n_groups;
   int len = a.lengths[b];
@@ -84,14 +101,37 @@ __device__ __forceinline__ int segment_tiles(const ScanArgs& a, int seg) {
       L = v > L ? v : L;
     }
   }
-  return (L + kTileM - 1) / kTileM;
+  return (L + a.R - 1) / a.R;
 }
 
-struct ItemCursor {
+// Position in a ring of n barriers/buffers: index and the parity of the
+// current pass.  Advancing never divides (integer division costs ~50 cycles
+// on the issuing warp, and these loops run once per item).
+struct Ring {
+  uint32_t i = 0, ph = 0;
+  __device__ __forceinline__ void step(uint32_t n) {
+    if (++i == n) { i = 0; ph ^= 1u; }
+  }
+  __device__ __forceinline__ void step_by(uint32_t k, uint32_t n) {   // k <= n
+    i += k;
+    if (i >= n) { i -= n; ph ^= 1u; }
+  }
+};
+
+// Walks the segments of an item range in order, keeping (b, g) without
+// division: segment seg = b * n_groups + g.
+struct SegWalk {
   const int* prefix;
-  int seg;
-  __device__ __forceinline__ void seek(int item) {
-    while (prefix[seg + 1] <= item) ++seg;
+  int n_groups;
+  int seg = 0, b = 0, g = 0;
+  __device__ __forceinline__ bool to(int item) {
+    bool moved = false;
+    while (prefix[seg + 1] <= item) {
+      ++seg;
+      if (++g == n_groups) { g = 0; ++b; }
+      moved = true;
+    }
+    return moved;
   }
 };
 
@@ -100,17 +140,114 @@ __device__ __forceinline__ uint32_t swizzle(uint32_t off, uint32_t swz) {
   return off ^ (((off >> 7) & ((swz >> 4) - 1u)) << 4);
 }
 
+// 16-byte cp.async reading src_bytes (0..16) and zero-filling the rest.
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst_smem, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// 4-byte cp.async reading src_bytes (0 or 4).
+__device__ __forceinline__ void cp_async_4_zfill(uint32_t dst_smem, const void* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// Bulk (non-tensor) global -> shared copy completing on an mbarrier;
+// addresses and size must be multiples of 16 bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// sum_h wq_h * max(v_h, 0) over 16 columns, in 4 interleaved partial sums;
+// the weights are read four at a time.
+__device__ __forceinline__ void relu_dot16(const float* v, const float* wq, float (&acc)[4]) {
+#pragma unroll
+  for (int e = 0; e < 16; e += 4) {
+    const float4 w4 = *reinterpret_cast<const float4*>(wq + e);
+    acc[0] = fmaf(w4.x, fmaxf(v[e], 0.f), acc[0]);
+    acc[1] = fmaf(w4.y, fmaxf(v[e + 1], 0.f), acc[1]);
+    acc[2] = fmaf(w4.z, fmaxf(v[e + 2], 0.f), acc[2]);
+    acc[3] = fmaf(w4.w, fmaxf(v[e + 3], 0.f), acc[3]);
+  }
+}
+
+__device__ __forceinline__ void relu_dot16_beta(const float* v, const float* w, const float* qs,
+                                                const float* be, float cs, float (&acc)[4]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float x = fmaf(v[e], qs[e] * cs, be[e]);
+    acc[e & 3] = fmaf(w[e], fmaxf(x, 0.f), acc[e & 3]);
+  }
+}
+
+// The MMAs of one K-chunk of a stage: KSTEPS steps of 32 bytes along K, each
+// for MB row blocks (separate accumulators N columns apart).  Unrolled: the
+// issuing thread is a single dependency chain, so loop control and address
+// arithmetic per MMA would otherwise cost as much as the MMA itself.
+template <int KIND, int KSTEPS, int MB>
+__device__ __forceinline__ void issue_chunk(uint32_t d0, uint32_t a_c, uint32_t b_c, uint64_t desc_hi,
+                                            uint32_t m_stride, uint32_t n_cols, uint32_t idesc, bool first_chunk) {
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS; ++ks) {
+    const uint64_t bdesc = desc_hi | ((b_c + ks * 32u) >> 4);
+#pragma unroll
+    for (int mb = 0; mb < MB; ++mb) {
+      const uint64_t adesc = desc_hi | ((a_c + mb * m_stride + ks * 32u) >> 4);
+      umma<KIND>(d0 + mb * n_cols, adesc, bdesc, idesc, (first_chunk && ks == 0) ? 0u : 1u);
+    }
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ void issue_chunk_rt(int ksteps, int mbs, uint32_t d0, uint32_t a_c, uint32_t b_c,
+                                               uint64_t desc_hi, uint32_t m_stride, uint32_t n_cols, uint32_t idesc,
+                                               bool first_chunk) {
+  switch (ksteps * 4 + mbs) {
+    case 1 * 4 + 1: issue_chunk<KIND, 1, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 1 * 4 + 2: issue_chunk<KIND, 1, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 2 * 4 + 1: issue_chunk<KIND, 2, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 2 * 4 + 2: issue_chunk<KIND, 2, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 4 * 4 + 1: issue_chunk<KIND, 4, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    default: issue_chunk<KIND, 4, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+  }
+}
+
+__device__ __forceinline__ void trace_event(uint64_t* trace, uint32_t lt, int ev) {
+  if (trace && blockIdx.x < kTraceCtas && lt < kTraceTiles)
+    trace[(static_cast<size_t>(blockIdx.x) * kTraceTiles + lt) * kTraceEvents + ev] = cycles();
+}
+
+// Wait for the last pass of every slot of a ring used `uses` times (only
+// after an abort; divisions are fine here).
+__device__ __forceinline__ void drain_ring(uint64_t* bars, uint32_t n, uint32_t uses) {
+  const uint32_t m = uses < n ? uses : n;
+  for (uint32_t i = 0; i < m; ++i) {
+    const uint32_t last = uses - 1 - ((uses - 1 - i) % n);
+    drain_wait(&bars[i], (last / n) & 1u, kDrainNs);
+  }
+}
+
 template <int KIND, bool GATHER>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_constant__ ScanArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   ScanSmem s = carve(base, a);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool e4 = a.cache_scale != nullptr;
+  const bool has_meta = GATHER || e4;
 
   if (tid == 0) {
     for (int i = 0; i < a.n_stages; ++i) { mbar_init(&s.full[i], GATHER ? 32 : 1); mbar_init(&s.empty[i], 1); }
     for (int i = 0; i < a.n_bslots; ++i) { mbar_init(&s.bfull[i], 1); mbar_init(&s.bempty[i], 1); }
-    for (int i = 0; i < a.n_acc; ++i) { mbar_init(&s.accfull[i], 1); mbar_init(&s.accempty[i], 4); }
+    for (int i = 0; i < a.n_acc; ++i) { mbar_init(&s.accfull[i], 1); mbar_init(&s.accempty[i], 4 * a.MB); }
+    for (int i = 0; i < kMetaSlots; ++i) {
+      mbar_init(&s.mfull[i], GATHER ? 32 : 1);
+      mbar_init(&s.mempty[i], 4 * a.MB);
+    }
     mbar_init(s.drain, 1);
     *s.abort_flag = 0;
     fence_barrier_init();
@@ -119,8 +256,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     tmem_alloc(s.tmem_base, a.tmem_cols);
     tmem_relinquish();
   }
-  // Tiles per segment, then an exclusive prefix over segments.
-  for (int i = tid; i < a.n_segments; i += blockDim.x) s.prefix[i + 1] = segment_tiles<GATHER>(a, i);
+  // Items per segment, then an exclusive prefix over segments.
+  for (int i = tid; i < a.n_segments; i += blockDim.x) s.prefix[i + 1] = segment_items<GATHER>(a, i);
   __syncthreads();
   if (warp == 0) {
     int carry = 0;
@@ -141,188 +278,252 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
 
+  // Every scalar argument is copied into registers once: the argument block
+  // is addressable (the tensor maps are read through their addresses), so a
+  // field read after an asm statement with a memory clobber would otherwise
+  // be reloaded from parameter memory.
+  const int k_capacity = a.capacity, k_T = a.T, k_H = a.H, k_H_pad = a.H_pad, k_Qg = a.Qg, k_N = a.N;
+  const int k_cand_stride = a.cand_stride, k_swz = a.swz, k_n_kchunks = a.n_kchunks;
+  const int k_R = a.R, k_MB = a.MB, k_KS = a.KS, k_spi = a.stages_per_item;
+  const uint32_t k_a_stage_bytes = a.a_stage_bytes, k_b_slot_bytes = a.b_slot_bytes, k_idesc = a.idesc;
+  const uint32_t k_meta_bytes = a.meta_bytes;
+  const int64_t k_row_bytes = a.row_bytes, k_score_stride = a.score_stride;
+  const uint8_t* const k_cache = a.cache;
+  const float* const k_cache_scale = a.cache_scale;
+  const int* const k_lengths = a.lengths;
+  const int* const k_q_pos = a.q_pos;
+  const float* const k_w = a.w;
+  const float* const k_q_scale = a.q_scale;
+  const float* const k_beta = a.beta;
+  const int* const k_cand = a.cand;
+  const int* const k_cand_n = a.cand_n;
+  float* const k_scores = a.scores;
+  int* const k_status = a.status;
+  uint64_t* const k_trace = a.trace;
+
   const int total = s.prefix[a.n_segments];
   const int begin = static_cast<int>((static_cast<int64_t>(total) * blockIdx.x) / gridDim.x);
   const int end = static_cast<int>((static_cast<int64_t>(total) * (blockIdx.x + 1)) / gridDim.x);
-  const WaitCtl wc{s.abort_flag, a.status, a.wait_ns};
+  const WaitCtl wc{s.abort_flag, k_status, a.wait_ns};
   const uint32_t tmem = *s.tmem_base;
-  const int S = a.n_stages;
-  const int elt_per_chunk = a.swz / a.elt_bytes;
+  const uint32_t S = static_cast<uint32_t>(a.n_stages);
+  const uint32_t NB = static_cast<uint32_t>(a.n_bslots);
+  const uint32_t NA = static_cast<uint32_t>(a.n_acc);
+  const int elt_per_chunk = k_swz / a.elt_bytes;
+  const int n_groups = GATHER ? k_T : a.n_groups;
+  const uint32_t chunk_region = static_cast<uint32_t>(k_R * k_swz);   // one K-chunk of a stage
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    uint32_t kcount = 0, b_use = 0;
-    int cur_seg = -1;
-    ItemCursor cur{s.prefix, 0};
-    if (!GATHER) {
-      if (lane == 0) {
-        tma_prefetch_desc(&a.map_a);
-        tma_prefetch_desc(&a.map_b);
-        for (int item = begin; item < end && !*s.abort_flag; ++item) {
-          cur.seek(item);
-          const int seg = cur.seg, tile = item - s.prefix[seg];
-          if (seg != cur_seg) {
-            const int slot = b_use % a.n_bslots;
-            if (!bounded_wait(&s.bempty[slot], ((b_use / a.n_bslots) & 1u) ^ 1u, wc)) break;
-            mbar_arrive_expect_tx(&s.bfull[slot], a.b_slot_bytes);
-            const int b = seg / a.n_groups, g = seg % a.n_groups;
-            uint8_t* dst = s.b_slots + static_cast<size_t>(slot) * a.b_slot_bytes;
-            for (int kc = 0; kc < a.n_kchunks; ++kc)
-              tma_load_3d(dst + static_cast<size_t>(kc) * a.N * a.swz, &a.map_b, &s.bfull[slot],
-                          kc * elt_per_chunk, 0, b * a.T + g * a.Qg);
-            ++b_use;
-            cur_seg = seg;
-          }
-          const int b = seg / a.n_groups;
-          const int row0 = b * a.capacity + tile * kTileM;
-          bool ok = true;
-          for (int kc = 0; kc < a.n_kchunks; ++kc) {
-            const int st = kcount % S;
-            if (!bounded_wait(&s.empty[st], ((kcount / S) & 1u) ^ 1u, wc)) { ok = false; break; }
-            mbar_arrive_expect_tx(&s.full[st], a.a_stage_bytes);
-            tma_load_2d(s.a_stages + static_cast<size_t>(st) * a.a_stage_bytes, &a.map_a, &s.full[st],
-                        kc * elt_per_chunk, row0);
-            ++kcount;
-          }
-          if (!ok) break;
+  if (warp == 0 && !GATHER) {
+    // ------------------------------------------------------------ loader (TMA), one lane
+    if (lane == 0) {
+      tma_prefetch_desc(&a.map_a);
+      tma_prefetch_desc(&a.map_b);
+      Ring st, bs, ms;
+      uint32_t n_st = 0, n_bs = 0, n_ms = 0;
+      SegWalk w{s.prefix, n_groups};
+      bool first = true;
+      uint32_t lt = 0;
+      for (int item = begin; item < end; ++item, ++lt) {
+        if (*s.abort_flag) break;
+        const bool moved = w.to(item) || first;
+        first = false;
+        const int it = item - s.prefix[w.seg];   // item index within the segment
+        if (moved) {
+          if (!bounded_wait(&s.bempty[bs.i], bs.ph ^ 1u, wc)) break;
+          mbar_arrive_expect_tx(&s.bfull[bs.i], k_b_slot_bytes);
+          uint8_t* dst = s.b_slots + static_cast<size_t>(bs.i) * k_b_slot_bytes;
+          const int z = w.b * k_T + w.g * k_Qg;
+          for (int kc = 0; kc < k_n_kchunks; ++kc)
+            tma_load_3d(dst + static_cast<size_t>(kc) * k_N * k_swz, &a.map_b, &s.bfull[bs.i],
+                        kc * elt_per_chunk, 0, z);
+          bs.step(NB);
+          ++n_bs;
         }
-        if (*s.abort_flag) {
-          // Let every copy already issued land before the CTA exits.
-          const uint32_t nst = kcount < static_cast<uint32_t>(S) ? kcount : S;
-          for (uint32_t i = 0; i < nst; ++i) {
-            const uint32_t last = kcount - 1 - ((kcount - 1 - i) % S);   // last use of stage i
-            drain_wait(&s.full[i], (last / S) & 1u, kDrainNs);
-          }
-          const uint32_t nb = b_use < static_cast<uint32_t>(a.n_bslots) ? b_use : a.n_bslots;
-          for (uint32_t i = 0; i < nb; ++i) {
-            const uint32_t last = b_use - 1 - ((b_use - 1 - i) % a.n_bslots);
-            drain_wait(&s.bfull[i], (last / a.n_bslots) & 1u, kDrainNs);
-          }
+        if (e4) {
+          // the item's per-token scales, one bulk copy (rows past the
+          // capacity are not read: the epilogue ignores them)
+          if (!bounded_wait(&s.mempty[ms.i], ms.ph ^ 1u, wc)) break;
+          const int rows = min(k_R, k_capacity - it * k_R);
+          const uint32_t bytes = static_cast<uint32_t>(rows) * 4u;
+          mbar_arrive_expect_tx(&s.mfull[ms.i], bytes);
+          bulk_load(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes,
+                    k_cache_scale + static_cast<int64_t>(w.b) * k_capacity + it * k_R, bytes, &s.mfull[ms.i]);
+          ms.step(kMetaSlots);
+          ++n_ms;
         }
-      }
-    } else {
-      // Gather: 32 lanes copy candidate rows with 16-byte cp.async into the
-      // same swizzled layout TMA would produce; a stage is signalled full
-      // once every lane's copies for it have landed (4 stages in flight).
-      constexpr int kDepth = 4;
-      uint32_t pend[kDepth];
-      int inflight = 0;
-      const int chunks16 = a.swz >> 4;
-      for (int item = begin; item < end && !*s.abort_flag; ++item) {
-        cur.seek(item);
-        const int seg = cur.seg, tile = item - s.prefix[seg];
-        if (seg != cur_seg) {
-          bool ok = true;
-          if (lane == 0) {
-            const int slot = b_use % a.n_bslots;
-            ok = bounded_wait(&s.bempty[slot], ((b_use / a.n_bslots) & 1u) ^ 1u, wc);
-            if (ok) {
-              mbar_arrive_expect_tx(&s.bfull[slot], a.b_slot_bytes);
-              uint8_t* dst = s.b_slots + static_cast<size_t>(slot) * a.b_slot_bytes;
-              for (int kc = 0; kc < a.n_kchunks; ++kc)
-                tma_load_3d(dst + static_cast<size_t>(kc) * a.N * a.swz, &a.map_b, &s.bfull[slot],
-                            kc * elt_per_chunk, 0, seg);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-          ++b_use;
-          cur_seg = seg;
-        }
-        const int b = seg / a.T;
-        int len = a.lengths[b];
-        len = len < 0 ? 0 : (len > a.capacity ? a.capacity : len);
-        int cn = a.cand_n[seg];
-        cn = cn < 0 ? 0 : (cn > a.cand_stride ? a.cand_stride : cn);
-        int tok[kTileM / 32];
-#pragma unroll
-        for (int i = 0; i < kTileM / 32; ++i) {
-          const int j = tile * kTileM + lane + 32 * i;
-          const int t = j < cn ? a.cand[static_cast<int64_t>(seg) * a.cand_stride + j] : -1;
-          tok[i] = (t >= 0 && t < len) ? t : -1;
-        }
+        const int row0 = w.b * k_capacity + it * k_R;
         bool ok = true;
-        for (int kc = 0; kc < a.n_kchunks; ++kc) {
-          const int st = kcount % S;
-          // One lane waits; the whole warp follows its verdict so the lanes
-          // never diverge around the warp-synchronous calls.
-          int got = 1;
-          if (lane == 0) got = bounded_wait(&s.empty[st], ((kcount / S) & 1u) ^ 1u, wc) ? 1 : 0;
-          got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) { ok = false; break; }
-          const uint32_t dst = smem_addr(s.a_stages + static_cast<size_t>(st) * a.a_stage_bytes);
-#pragma unroll
-          for (int i = 0; i < kTileM / 32; ++i) {
-            if (tok[i] < 0) continue;
-            const int r = lane + 32 * i;
-            const uint8_t* src = a.cache + (static_cast<int64_t>(b) * a.capacity + tok[i]) * a.row_bytes +
-                                 static_cast<int64_t>(kc) * a.swz;
-            for (int c = 0; c < chunks16; ++c)
-              cp_async_16(dst + swizzle(static_cast<uint32_t>(r * a.swz + c * 16), a.swz), src + c * 16);
-          }
-          cp_async_commit();
-          pend[kcount % kDepth] = st;
-          ++kcount;
-          if (++inflight == kDepth) {
-            cp_async_wait_group<kDepth - 1>();
-            fence_proxy_async_smem();
-            mbar_arrive(&s.full[pend[(kcount - kDepth) % kDepth]]);
-            --inflight;
-          }
+        for (int sp = 0; sp < k_spi; ++sp) {
+          if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
+          if (sp == 0) trace_event(k_trace, lt, 0);
+          mbar_arrive_expect_tx(&s.full[st.i], k_a_stage_bytes);
+          tma_load_3d(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes, &a.map_a, &s.full[st.i], 0, row0,
+                      sp * k_KS);
+          st.step(S);
+          ++n_st;
         }
         if (!ok) break;
+        trace_event(k_trace, lt, 1);
       }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      if (!*s.abort_flag) {
-        for (; inflight > 0; --inflight) mbar_arrive(&s.full[pend[(kcount - inflight) % kDepth]]);
-      } else if (lane == 0) {
-        const uint32_t nb = b_use < static_cast<uint32_t>(a.n_bslots) ? b_use : a.n_bslots;
-        for (uint32_t i = 0; i < nb; ++i) {
-          const uint32_t last = b_use - 1 - ((b_use - 1 - i) % a.n_bslots);
-          drain_wait(&s.bfull[i], (last / a.n_bslots) & 1u, kDrainNs);
-        }
+      if (*s.abort_flag) {
+        // let every copy already issued land before the CTA exits
+        drain_ring(s.full, S, n_st);
+        drain_ring(s.bfull, NB, n_bs);
+        drain_ring(s.mfull, kMetaSlots, n_ms);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t kcount = 0, b_use = 0, acc_use = 0;
-      int cur_seg = -1, slot = -1;
-      ItemCursor cur{s.prefix, 0};
-      for (int item = begin; item < end && !*s.abort_flag; ++item) {
-        cur.seek(item);
-        const int seg = cur.seg;
-        if (seg != cur_seg) {
-          if (slot >= 0) umma_commit(&s.bempty[slot]);
-          slot = b_use % a.n_bslots;
-          if (!bounded_wait(&s.bfull[slot], (b_use / a.n_bslots) & 1u, wc)) break;
-          tc_fence_after();
-          ++b_use;
-          cur_seg = seg;
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ loader (gather), 32 lanes
+    // Each lane copies R/32 candidate rows with 16-byte cp.async into the
+    // [chunk][row] swizzled layout the 3-D TMA box would produce, plus the
+    // rows' token ids and fp8 scales into the item's metadata slot.  A stage
+    // (and the metadata with an item's first stage) is signalled once every
+    // lane's copies for it have landed; kDepth stages stay in flight.  All
+    // waits are warp-uniform.
+    constexpr int kDepth = 4;
+    uint32_t pend[kDepth];     // stage | (meta slot + 1) << 16
+    uint32_t issued = 0, retired = 0, n_bs = 0;
+    const int chunks16 = k_swz >> 4;
+    const int rows_per_lane = k_R >> 5;
+    Ring st, bs, ms;
+    SegWalk w{s.prefix, n_groups};
+    bool first = true;
+    for (int item = begin; item < end; ++item) {
+      if (*s.abort_flag) break;
+      const bool moved = w.to(item) || first;
+      first = false;
+      const int seg = w.seg, it = item - s.prefix[seg];
+      if (moved) {
+        if (!bounded_wait(&s.bempty[bs.i], bs.ph ^ 1u, wc)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&s.bfull[bs.i], k_b_slot_bytes);
+          uint8_t* dst = s.b_slots + static_cast<size_t>(bs.i) * k_b_slot_bytes;
+          for (int kc = 0; kc < k_n_kchunks; ++kc)
+            tma_load_3d(dst + static_cast<size_t>(kc) * k_N * k_swz, &a.map_b, &s.bfull[bs.i],
+                        kc * elt_per_chunk, 0, seg);
         }
-        const int acc = acc_use % a.n_acc;
-        if (!bounded_wait(&s.accempty[acc], ((acc_use / a.n_acc) & 1u) ^ 1u, wc)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * a.N);
-        const uint32_t b_base = smem_addr(s.b_slots + static_cast<size_t>(slot) * a.b_slot_bytes);
-        bool ok = true;
-        for (int kc = 0; kc < a.n_kchunks; ++kc) {
-          const int st = kcount % S;
-          if (!bounded_wait(&s.full[st], (kcount / S) & 1u, wc)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_base = smem_addr(s.a_stages + static_cast<size_t>(st) * a.a_stage_bytes);
-          const uint32_t bk = b_base + static_cast<uint32_t>(kc * a.N * a.swz);
-          for (int ks = 0; ks < (a.swz >> 5); ++ks) {
-            umma<KIND>(d_tmem, make_smem_desc(a_base + ks * 32, a.swz), make_smem_desc(bk + ks * 32, a.swz),
-                       a.idesc, (kc | ks) != 0 ? 1u : 0u);
+        bs.step(NB);
+        ++n_bs;
+      }
+      int len = k_lengths[w.b];
+      len = len < 0 ? 0 : (len > k_capacity ? k_capacity : len);
+      int cn = k_cand_n[seg];
+      cn = cn < 0 ? 0 : (cn > k_cand_stride ? k_cand_stride : cn);
+      if (!bounded_wait(&s.mempty[ms.i], ms.ph ^ 1u, wc)) break;
+      float* mscale = reinterpret_cast<float*>(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes);
+      int* mtok = reinterpret_cast<int*>(mscale + k_R);
+      const int64_t seq_row = static_cast<int64_t>(w.b) * k_capacity;
+      int tok[kMaxItemRows / 32];
+#pragma unroll
+      for (int i = 0; i < kMaxItemRows / 32; ++i) {
+        tok[i] = -1;
+        if (i < rows_per_lane) {
+          const int r = lane + 32 * i;
+          const int j = it * k_R + r;
+          int t = j < cn ? k_cand[static_cast<int64_t>(seg) * k_cand_stride + j] : -1;
+          if (j < cn && (t < 0 || t >= len)) t = -2;     // invalid candidate
+          tok[i] = t;
+          mtok[r] = t;
+          if (e4) cp_async_4_zfill(smem_addr(mscale + r), k_cache_scale + seq_row + (t >= 0 ? t : 0), t >= 0 ? 4 : 0);
+        }
+      }
+      const uint32_t mslot = ms.i;
+      ms.step(kMetaSlots);
+      bool ok = true;
+      for (int sp = 0; sp < k_spi; ++sp) {
+        if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
+        const uint32_t dst = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
+#pragma unroll
+        for (int i = 0; i < kMaxItemRows / 32; ++i) {
+          if (i >= rows_per_lane) break;
+          const int r = lane + 32 * i;
+          const int t = tok[i] >= 0 ? tok[i] : 0;
+          const int nbytes = tok[i] >= 0 ? 16 : 0;
+          for (int c = 0; c < k_KS; ++c) {
+            const int kc = sp * k_KS + c;
+            const uint8_t* src = k_cache + (seq_row + t) * k_row_bytes + static_cast<int64_t>(kc) * k_swz;
+            const uint32_t rowdst = dst + static_cast<uint32_t>(c) * chunk_region;
+            for (int q = 0; q < chunks16; ++q)
+              cp_async_16_zfill(rowdst + swizzle(static_cast<uint32_t>(r * k_swz + q * 16), k_swz), src + q * 16,
+                                nbytes);
           }
-          umma_commit(&s.empty[st]);
-          ++kcount;
+        }
+        cp_async_commit();
+        pend[issued & (kDepth - 1)] = st.i | (sp == 0 ? (mslot + 1u) << 16 : 0u);
+        ++issued;
+        st.step(S);
+        if (issued - retired == kDepth) {
+          cp_async_wait_group<kDepth - 1>();
+          fence_proxy_async_smem();
+          const uint32_t p = pend[retired & (kDepth - 1)];
+          mbar_arrive(&s.full[p & 0xFFFFu]);
+          if (p >> 16) mbar_arrive(&s.mfull[(p >> 16) - 1]);
+          ++retired;
+        }
+      }
+      if (!ok) break;
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    if (!*s.abort_flag) {
+      while (retired < issued) {
+        const uint32_t p = pend[retired & (kDepth - 1)];
+        mbar_arrive(&s.full[p & 0xFFFFu]);
+        if (p >> 16) mbar_arrive(&s.mfull[(p >> 16) - 1]);
+        ++retired;
+      }
+    } else if (lane == 0) {
+      // B slots were loaded by TMA: let them land (the cp.async rows are done)
+      drain_ring(s.bfull, NB, n_bs);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer, one lane
+    if (lane == 0) {
+      Ring st, bs, acc;
+      SegWalk w{s.prefix, n_groups};
+      bool first = true;
+      int slot = -1;
+      uint32_t lt = 0;
+      // K-major swizzled descriptors: everything but the start address is
+      // fixed, so only the address field is added per MMA.
+      const uint64_t desc_hi = make_smem_desc(0, static_cast<uint32_t>(k_swz));
+      const uint32_t m_stride = static_cast<uint32_t>(128 * k_swz);     // next M block in a chunk
+      const uint32_t ksteps = static_cast<uint32_t>(k_swz >> 5);
+      for (int item = begin; item < end; ++item, ++lt) {
+        if (*s.abort_flag) break;
+        const bool moved = w.to(item) || first;
+        first = false;
+        if (moved) {
+          if (slot >= 0) umma_commit(&s.bempty[slot]);
+          if (!bounded_wait(&s.bfull[bs.i], bs.ph, wc)) break;
+          tc_fence_after();
+          slot = static_cast<int>(bs.i);
+          bs.step(NB);
+        }
+        if (!bounded_wait(&s.accempty[acc.i], acc.ph ^ 1u, wc)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem + acc.i * static_cast<uint32_t>(k_MB * k_N);
+        const uint32_t b_base = smem_addr(s.b_slots + static_cast<size_t>(slot) * k_b_slot_bytes);
+        bool ok = true;
+        for (int sp = 0; sp < k_spi; ++sp) {
+          if (sp == 0) trace_event(k_trace, lt, 6);
+          if (!bounded_wait(&s.full[st.i], st.ph, wc)) { ok = false; break; }
+          if (sp == 0) trace_event(k_trace, lt, 2);
+          tc_fence_after();
+          const uint32_t a_base = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
+          for (int c = 0; c < k_KS; ++c) {
+            const int kc = sp * k_KS + c;
+            issue_chunk_rt<KIND>(static_cast<int>(ksteps), k_MB, d0, a_base + static_cast<uint32_t>(c) * chunk_region,
+                                 b_base + static_cast<uint32_t>(kc * k_N * k_swz), desc_hi, m_stride,
+                                 static_cast<uint32_t>(k_N), k_idesc, kc == 0);
+          }
+          umma_commit(&s.empty[st.i]);
+          st.step(S);
         }
         if (!ok) break;
-        umma_commit(&s.accfull[acc]);
-        ++acc_use;
+        umma_commit(&s.accfull[acc.i]);
+        trace_event(k_trace, lt, 3);
+        acc.step(NA);
       }
       if (*s.abort_flag) {
         umma_commit(s.drain);
@@ -331,53 +532,64 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;                 // 0..3
+    // Two warpgroups.  With two M blocks per item (R = 256) warpgroup g takes
+    // block g of every item; with one (R = 128) they take alternate items.
+    const int ew = warp - 2;                 // 0 .. kEpiWarps-1
+    const int wg = ew >> 2;
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-    const int r = quad * 32 + lane;          // row of the tile = TMEM lane
-    float* ep_w = s.ep + ew * (3 * a.N + 16);
-    float* ep_qs = ep_w + a.N;
-    float* ep_beta = ep_qs + a.N;
-    int* ep_len = reinterpret_cast<int*>(ep_beta + a.N);
-    uint32_t acc_use = 0;
-    int cur_seg = -1;
-    ItemCursor cur{s.prefix, 0};
-    const bool has_beta = a.beta != nullptr;
-    for (int item = begin; item < end && !*s.abort_flag; ++item) {
-      cur.seek(item);
-      const int seg = cur.seg, tile = item - s.prefix[seg];
-      const int b = GATHER ? seg / a.T : seg / a.n_groups;
-      const int g = GATHER ? seg % a.T : seg % a.n_groups;
-      int len = a.lengths[b];
-      len = len < 0 ? 0 : (len > a.capacity ? a.capacity : len);
-      if (seg != cur_seg) {
+    const int mb = k_MB == 2 ? wg : 0;
+    const int istep = k_MB == 2 ? 1 : 2;
+    const int r = mb * 128 + quad * 32 + lane;   // row of the item
+    float* ep_w = s.ep + ew * (3 * k_N + 16);
+    float* ep_qs = ep_w + k_N;
+    float* ep_beta = ep_qs + k_N;
+    int* ep_len = reinterpret_cast<int*>(ep_beta + k_N);
+    const bool has_beta = k_beta != nullptr;
+    Ring acc, ms;
+    const uint32_t first_item = k_MB == 2 ? 0u : static_cast<uint32_t>(wg);
+    acc.i = first_item;                      // n_acc, kMetaSlots >= 2
+    ms.i = first_item;
+    SegWalk w{s.prefix, n_groups};
+    bool first = true;
+    uint32_t lt = first_item;
+    for (int item = begin + static_cast<int>(first_item); item < end; item += istep, lt += istep) {
+      if (*s.abort_flag) break;
+      const bool moved = w.to(item) || first;
+      first = false;
+      const int seg = w.seg, it = item - s.prefix[seg];
+      const int b = w.b, g = w.g;
+      if (moved) {
+        int len = k_lengths[b];
+        len = len < 0 ? 0 : (len > k_capacity ? k_capacity : len);
         __syncwarp();
-        for (int i = lane; i < a.N; i += 32) {
-          const int qi = i / a.H_pad, h = i % a.H_pad;
-          const int t = g * a.Qg + qi;
-          float wv = 0.f, qs = 1.f, be = 0.f;
-          if (h < a.H && t < a.T) {
-            const int64_t o = (static_cast<int64_t>(b) * a.T + t) * a.H + h;
-            wv = a.w[o];
-            if (a.q_scale) qs = a.q_scale[o];
-            if (has_beta) be = a.beta[o];
+        for (int qi = 0, i0 = 0; qi < k_Qg; ++qi, i0 += k_H_pad) {
+          const int t = g * k_Qg + qi;
+          for (int h = lane; h < k_H_pad; h += 32) {
+            float wv = 0.f, qs = 1.f, be = 0.f;
+            if (h < k_H && t < k_T) {
+              const int64_t o = (static_cast<int64_t>(b) * k_T + t) * k_H + h;
+              wv = k_w[o];
+              if (k_q_scale) qs = k_q_scale[o];
+              if (has_beta) be = k_beta[o];
+            }
+            // Without a bias, fold the query scale into the weight (ReLU is
+            // positively homogeneous and the scales are positive).
+            ep_w[i0 + h] = has_beta ? wv : wv * qs;
+            ep_qs[i0 + h] = qs;
+            ep_beta[i0 + h] = be;
           }
-          // Without a bias, fold the query scale into the weight (ReLU is
-          // positively homogeneous and the scales are positive).
-          ep_w[i] = has_beta ? wv : wv * qs;
-          ep_qs[i] = qs;
-          ep_beta[i] = be;
         }
         if (lane < 16) {
-          const int t = g * a.Qg + lane;
+          const int t = g * k_Qg + lane;
           int v = 0;
-          if (lane < a.Qg && t < a.T) {
+          if (lane < k_Qg && t < k_T) {
             if (GATHER) {
-              v = a.cand_n[seg];
-              v = v < 0 ? 0 : (v > a.cand_stride ? a.cand_stride : v);
+              v = k_cand_n[seg];
+              v = v < 0 ? 0 : (v > k_cand_stride ? k_cand_stride : v);
             } else {
               v = len;
-              if (a.q_pos) {
-                int p = a.q_pos[b * a.T + t] + 1;
+              if (k_q_pos) {
+                int p = k_q_pos[b * k_T + t] + 1;
                 v = p < 0 ? 0 : (p > len ? len : p);
               }
             }
@@ -385,74 +597,68 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           ep_len[lane] = v;
         }
         __syncwarp();
-        cur_seg = seg;
       }
-      const int acc = acc_use % a.n_acc;
-      if (!bounded_wait(&s.accfull[acc], (acc_use / a.n_acc) & 1u, wc)) break;
+      const int j = it * k_R + r;           // position (scan) or candidate slot (gather)
+      int tok = j;
+      float cs = 1.f;
+      if (has_meta) {
+        if (!bounded_wait(&s.mfull[ms.i], ms.ph, wc)) break;
+        const float* mscale = reinterpret_cast<const float*>(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes);
+        if (GATHER) tok = reinterpret_cast<const int*>(mscale + k_R)[r];
+        if (e4 && tok >= 0) cs = mscale[r];    // rows past the valid prefix read a stale value, unused
+      }
+      if (!bounded_wait(&s.accfull[acc.i], acc.ph, wc)) break;
+      if (lane == 0 && (ew & 3) == 0) trace_event(k_trace, lt, 4);
       tc_fence_after();
 
-      const int j = tile * kTileM + r;      // position (scan) or candidate slot (gather)
-      int tok = j;
-      bool tok_ok = true;
-      if (GATHER) {
-        tok = j < ep_len[0] ? a.cand[static_cast<int64_t>(seg) * a.cand_stride + j] : -1;
-        tok_ok = tok >= 0 && tok < len;
-      }
-      float cs = 1.f;
-      if (a.cache_scale && tok_ok && j < (GATHER ? ep_len[0] : len))
-        cs = a.cache_scale[static_cast<int64_t>(b) * a.capacity + tok];
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * a.N);
-      for (int qi = 0; qi < a.Qg; ++qi) {
-        const int t = g * a.Qg + qi;
-        if (t >= a.T) break;
-        float sc = 0.f;
-        const float* wq = ep_w + qi * a.H_pad;
-        const float* qs = ep_qs + qi * a.H_pad;
-        const float* be = ep_beta + qi * a.H_pad;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                             (acc.i * static_cast<uint32_t>(k_MB) + static_cast<uint32_t>(mb)) * static_cast<uint32_t>(k_N);
+      for (int qi = 0; qi < k_Qg; ++qi) {
+        const int t = g * k_Qg + qi;
+        if (t >= k_T) break;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* wq = ep_w + qi * k_H_pad;
+        const float* qs = ep_qs + qi * k_H_pad;
+        const float* be = ep_beta + qi * k_H_pad;
         int h0 = 0;
-        for (; h0 + 32 <= a.H_pad; h0 += 32) {
+        for (; h0 + 32 <= k_H_pad; h0 += 32) {
           float v[32];
-          tmem_load32_sync(tbase + static_cast<uint32_t>(qi * a.H_pad + h0), v);
+          tmem_load32_sync(tbase + static_cast<uint32_t>(qi * k_H_pad + h0), v);
           if (!has_beta) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sc = fmaf(wq[h0 + e], fmaxf(v[e], 0.f), sc);
+            relu_dot16(v, wq + h0, part);
+            relu_dot16(v + 16, wq + h0 + 16, part);
           } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float x = fmaf(v[e], qs[h0 + e] * cs, be[h0 + e]);
-              sc = fmaf(wq[h0 + e], fmaxf(x, 0.f), sc);
-            }
+            relu_dot16_beta(v, wq + h0, qs + h0, be + h0, cs, part);
+            relu_dot16_beta(v + 16, wq + h0 + 16, qs + h0 + 16, be + h0 + 16, cs, part);
           }
         }
-        if (h0 < a.H_pad) {   // H_pad % 32 == 16
+        if (h0 < k_H_pad) {   // H_pad % 32 == 16
           float v[16];
-          tmem_load16_sync(tbase + static_cast<uint32_t>(qi * a.H_pad + h0), v);
-          if (!has_beta) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) sc = fmaf(wq[h0 + e], fmaxf(v[e], 0.f), sc);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x = fmaf(v[e], qs[h0 + e] * cs, be[h0 + e]);
-              sc = fmaf(wq[h0 + e], fmaxf(x, 0.f), sc);
-            }
-          }
+          tmem_load16_sync(tbase + static_cast<uint32_t>(qi * k_H_pad + h0), v);
+          if (!has_beta) relu_dot16(v, wq + h0, part);
+          else relu_dot16_beta(v, wq + h0, qs + h0, be + h0, cs, part);
         }
-        if (!has_beta && a.cache_scale) sc *= cs;
+        if (qi == 0 && lane == 0 && (ew & 3) == 0) trace_event(k_trace, lt, 7);
+        float sc = (part[0] + part[1]) + (part[2] + part[3]);
+        if (!has_beta && e4) sc *= cs;
         if (j < ep_len[qi]) {
-          if (!tok_ok) {
+          if (GATHER && tok < 0) {
             sc = -INFINITY;
-            record_status(a.status, kStatusIndex);
+            record_status(k_status, kStatusIndex);
           }
-          const int64_t row = static_cast<int64_t>(b) * a.T + t;
-          a.scores[row * a.score_stride + j] = sc;
-          if (a.hist) atomicAdd(&a.hist[row * kHistBins + (radix_key(sc) >> 21)], 1u);
+          const int64_t row = static_cast<int64_t>(b) * k_T + t;
+          k_scores[row * k_score_stride + j] = sc;
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.accempty[acc]);
-      ++acc_use;
+      if (lane == 0) {
+        if ((ew & 3) == 0) trace_event(k_trace, lt, 5);
+        mbar_arrive(&s.accempty[acc.i]);
+        if (has_meta) mbar_arrive(&s.mempty[ms.i]);
+      }
+      acc.step_by(static_cast<uint32_t>(istep), NA);
+      if (has_meta) ms.step_by(static_cast<uint32_t>(istep), kMetaSlots);
     }
   }
 
@@ -466,7 +672,10 @@ template <int KIND, bool GATHER>
 cudaError_t launch_one(const ScanArgs& a, int grid, cudaStream_t st) {
   auto k = scan_kernel<KIND, GATHER>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return e;
+  }
   k<<<grid, kScanThreads, a.smem_bytes, st>>>(a);
   return cudaGetLastError();
 }

@@ -24,6 +24,12 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// SM cycle counter: cheap to read, used to bound waits.  Limits given in ns
+// are converted at kCyclesPerNs (above the 1.965 GHz maximum SM clock, so a
+// bound in cycles never ends a wait early in real time).
+constexpr uint64_t kCyclesPerNs = 2;
+__device__ __forceinline__ uint64_t cycles() { return clock64(); }
+
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
@@ -60,6 +66,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep up to `ns` waiting
+// for the phase (and is woken when it completes) instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Per-CTA wait control: a shared abort flag and the global status word.
 struct WaitCtl {
   volatile int* abort_flag;  // shared memory
@@ -72,11 +92,27 @@ struct WaitCtl {
 // limit_ns, in which case it records the timeout and raises the abort flag.
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const uint64_t t0 = cycles();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*w.abort_flag) return false;
-    if ((it & 7u) == 0 && global_timer_ns() - t0 > w.limit_ns) {
+    if ((it & 7u) == 0 && cycles() - t0 > w.limit_ns * kCyclesPerNs) {
+      *w.abort_flag = 1;
+      record_status(w.status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// bounded_wait for a waiter that is not on the critical issue path: it
+// sleeps between polls so that it does not crowd the barrier unit.
+__device__ __forceinline__ bool bounded_wait_sleep(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = cycles();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
+    if (*w.abort_flag) return false;
+    if (cycles() - t0 > w.limit_ns * kCyclesPerNs) {
       *w.abort_flag = 1;
       record_status(w.status, kStatusTimeout);
       return false;
@@ -88,9 +124,9 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, con
 // flight to land (they always do), bounded by a fixed limit.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return;
-  const uint64_t t0 = global_timer_ns();
+  const uint64_t t0 = cycles();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > limit_ns) return;
+    if (cycles() - t0 > limit_ns * kCyclesPerNs) return;
   }
 }
 

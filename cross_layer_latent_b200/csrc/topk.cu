@@ -350,3 +350,291 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
 }
 
 }  // namespace li
+
+// ============================================================================
+// Single-launch cluster selection.
+//
+// One thread-block cluster (CS <= 8 CTAs of 512 threads) per row; CTA c owns
+// positions [c*E, (c+1)*E), E = 512 * PT, as register-resident keys (warp w
+// holds a contiguous run of 32*PT positions, lane l position j*32 + l).  Four
+// cluster barriers:
+//   1. first-digit (top 11 bits) histograms are complete; every CTA sums the
+//      cluster's histograms through distributed shared memory and finds the
+//      boundary bucket b1 of each budget;
+//   2. each CTA has compacted the keys of its elements in the boundary
+//      bucket(s) to its own region of the workspace; every CTA then resolves
+//      the two remaining digits (11 + 10 bits) over all of them, redundantly,
+//      giving the exact k-th key T and how many elements equal to T are taken;
+//   3. per-CTA counts of (key > T, key == T) are published; an element's
+//      output rank is #greater before it + min(#equal before it, taken);
+//   4. no CTA leaves while another may still read its counts.
+// Up to two budgets (k and k2 <= k) are selected from the same keys.
+// ============================================================================
+#include <cooperative_groups.h>
+
+namespace li {
+namespace {
+
+namespace cg = cooperative_groups;
+
+struct SelState {
+  int keff;          // min(k, n)
+  unsigned b1;       // boundary bucket of the first digit
+  int above1;        // elements in higher first-digit buckets
+  unsigned T;        // exact key of the keff-th element
+  int n_gt;          // elements with key > T
+  int need_eq;       // elements equal to T that are taken (lowest positions first)
+};
+
+// Find the boundary bucket of `need` counting from the top in a 2048-bin
+// histogram whose per-thread bins are held in loc[0..3] (bins hi-1..hi-4).
+__device__ __forceinline__ void find_from_loc(const unsigned (&loc)[4], int hi, int need, int* scratch,
+                                              int* out) {
+  const int sum = static_cast<int>(loc[0] + loc[1] + loc[2] + loc[3]);
+  if (threadIdx.x == 0) { out[0] = 0; out[1] = 0; }
+  const int before = block_excl_scan(sum, scratch, nullptr);
+  if (before < need && need <= before + sum) {
+    int cum = before;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (cum + static_cast<int>(loc[i]) >= need) { out[0] = hi - 1 - i; out[1] = cum; break; }
+      cum += static_cast<int>(loc[i]);
+    }
+  }
+  __syncthreads();
+}
+
+// Remaining two digits over the candidate keys of all CTAs (each CTA's
+// candidates at cand_base + c*E, counts in cnt[c]).
+__device__ void resolve_low_digits(SelState& st, const unsigned* cand_base, int64_t E, const int* cnt, int CS,
+                                   int offset_in_region_sel, unsigned* hist, int* scratch, int* res,
+                                   const int* cnt_other) {
+  int need = st.keff - st.above1;
+  unsigned prefix2 = 0;
+#pragma unroll 1
+  for (int d = 0; d < 2; ++d) {
+    const int nb = d == 0 ? 2048 : 1024;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int rk = 0; rk < CS; ++rk) {
+      const unsigned* src = cand_base + static_cast<int64_t>(rk) * E + (offset_in_region_sel ? cnt_other[rk] : 0);
+      const int m = cnt[rk];
+      for (int i = threadIdx.x; i < m; i += blockDim.x) {
+        const unsigned key = src[i];
+        if (d == 0) atomicAdd(&hist[(key >> 10) & 2047u], 1u);
+        else if (((key >> 10) & 2047u) == prefix2) atomicAdd(&hist[key & 1023u], 1u);
+      }
+    }
+    __syncthreads();
+    find_bucket_desc(hist, nb, need, scratch, res);
+    const unsigned bin = static_cast<unsigned>(res[0]);
+    const int above = res[1];
+    __syncthreads();
+    need -= above;
+    st.n_gt += above;
+    if (d == 0) prefix2 = bin;
+    else st.T = (st.b1 << 21) | (prefix2 << 10) | bin;
+  }
+  st.need_eq = need;
+}
+
+template <int PT>
+__global__ void __launch_bounds__(kClusterThreads) topk_cluster_kernel(const TopkArgs a, const TopkOut2 o2) {
+  __shared__ __align__(16) unsigned hist[kHistBins];
+  __shared__ int scratch[32];
+  __shared__ int res[2];
+  __shared__ int cnt_local[2];                  // candidates of this CTA per budget
+  __shared__ int cnt_all[2][kClusterMaxSize];   // every CTA's, per budget
+  __shared__ int wtot[4][kClusterThreads / 32];
+  __shared__ int ctot[4];                       // (gt, eq) per budget of this CTA
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CS = static_cast<int>(cluster.num_blocks());
+  const int c = static_cast<int>(cluster.block_rank());
+  const int r = blockIdx.y;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int n = row_len(a, r);
+  const int nsel = o2.k2 > 0 ? 2 : 1;
+  SelState sel[2];
+  sel[0].keff = min(a.k, n);
+  sel[1].keff = min(o2.k2, n);
+  int32_t* oidx[2] = {a.out_idx + static_cast<int64_t>(r) * a.k,
+                      o2.k2 ? o2.out_idx2 + static_cast<int64_t>(r) * o2.k2 : nullptr};
+  float* osc[2] = {a.out_score ? a.out_score + static_cast<int64_t>(r) * a.k : nullptr,
+                   (o2.k2 && o2.out_score2) ? o2.out_score2 + static_cast<int64_t>(r) * o2.k2 : nullptr};
+  const int kk[2] = {a.k, o2.k2};
+  if (c == 0) {
+    for (int sidx = 0; sidx < nsel; ++sidx)
+      for (int j = max(sel[sidx].keff, 0) + threadIdx.x; j < kk[sidx]; j += blockDim.x) {
+        oidx[sidx][j] = -1;
+        if (osc[sidx]) osc[sidx][j] = -INFINITY;
+      }
+    if (a.out_count && threadIdx.x == 0) a.out_count[r] = max(sel[0].keff, 0);
+  }
+  if (sel[0].keff <= 0) return;   // uniform over the cluster (depends on the row only)
+
+  const int64_t E = static_cast<int64_t>(kClusterThreads) * PT;
+  const int64_t base_w = static_cast<int64_t>(c) * E + static_cast<int64_t>(wid) * 32 * PT;
+  const float* row = a.scores + static_cast<int64_t>(r) * a.row_stride;
+  unsigned key[PT];
+  unsigned vmask = 0;
+#pragma unroll
+  for (int j = 0; j < PT; ++j) {
+    const int64_t pos = base_w + static_cast<int64_t>(j) * 32 + lane;
+    key[j] = 0;
+    if (pos < n) {
+      key[j] = radix_key(row[pos]);
+      vmask |= 1u << j;
+    }
+  }
+
+  // ---- 1. first digit
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < PT; ++j)
+    if ((vmask >> j) & 1u) atomicAdd(&hist[key[j] >> 21], 1u);
+  cluster.sync();
+  const int hi = kHistBins - static_cast<int>(threadIdx.x) * 4;
+  unsigned loc[4] = {0, 0, 0, 0};
+  {
+    uint4 parts[kClusterMaxSize];
+#pragma unroll
+    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+      if (rk < CS) parts[rk] = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, rk) + hi - 4);
+#pragma unroll
+    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+      if (rk < CS) { loc[3] += parts[rk].x; loc[2] += parts[rk].y; loc[1] += parts[rk].z; loc[0] += parts[rk].w; }
+  }
+  for (int sidx = 0; sidx < nsel; ++sidx) {
+    find_from_loc(loc, hi, sel[sidx].keff, scratch, res);
+    sel[sidx].b1 = static_cast<unsigned>(res[0]);
+    sel[sidx].above1 = res[1];
+    sel[sidx].n_gt = res[1];
+    __syncthreads();
+  }
+
+  // ---- 2. compact this CTA's boundary-bucket keys (budget 0, then budget 1
+  //         if its bucket differs) into its workspace region
+  unsigned* region = reinterpret_cast<unsigned*>(a.cand) + static_cast<int64_t>(r) * a.n + static_cast<int64_t>(c) * E;
+  const bool two_buckets = nsel == 2 && sel[1].b1 != sel[0].b1;
+  int written = 0;
+  for (int sidx = 0; sidx < (two_buckets ? 2 : 1); ++sidx) {
+    const unsigned b1 = sel[sidx].b1;
+    int mine = 0;
+#pragma unroll
+    for (int j = 0; j < PT; ++j) mine += (((vmask >> j) & 1u) && (key[j] >> 21) == b1) ? 1 : 0;
+    int tot = 0;
+    int off = block_excl_scan(mine, scratch, &tot);
+#pragma unroll
+    for (int j = 0; j < PT; ++j)
+      if (((vmask >> j) & 1u) && (key[j] >> 21) == b1) region[written + off++] = key[j];
+    if (threadIdx.x == 0) cnt_local[sidx] = tot;
+    written += tot;
+    __syncthreads();
+  }
+  if (!two_buckets && threadIdx.x == 0) cnt_local[1] = 0;
+  cluster.sync();
+  if (threadIdx.x < CS) {
+    const int* rc = cluster.map_shared_rank(cnt_local, static_cast<int>(threadIdx.x));
+    cnt_all[0][threadIdx.x] = rc[0];
+    cnt_all[1][threadIdx.x] = rc[1];
+  }
+  __syncthreads();
+  const unsigned* cand_base = reinterpret_cast<const unsigned*>(a.cand) + static_cast<int64_t>(r) * a.n;
+  resolve_low_digits(sel[0], cand_base, E, cnt_all[0], CS, 0, hist, scratch, res, cnt_all[0]);
+  if (nsel == 2) {
+    if (two_buckets)
+      resolve_low_digits(sel[1], cand_base, E, cnt_all[1], CS, 1, hist, scratch, res, cnt_all[0]);
+    else
+      resolve_low_digits(sel[1], cand_base, E, cnt_all[0], CS, 0, hist, scratch, res, cnt_all[0]);
+  }
+
+  // ---- 3. ordered output
+  int gtw[2] = {0, 0}, eqw[2] = {0, 0};
+#pragma unroll
+  for (int j = 0; j < PT; ++j) {
+    const bool v = (vmask >> j) & 1u;
+    for (int sidx = 0; sidx < nsel; ++sidx) {
+      gtw[sidx] += __popc(__ballot_sync(0xffffffffu, v && key[j] > sel[sidx].T));
+      eqw[sidx] += __popc(__ballot_sync(0xffffffffu, v && key[j] == sel[sidx].T));
+    }
+  }
+  if (lane == 0)
+    for (int sidx = 0; sidx < nsel; ++sidx) { wtot[2 * sidx][wid] = gtw[sidx]; wtot[2 * sidx + 1][wid] = eqw[sidx]; }
+  __syncthreads();
+  if (threadIdx.x < 2 * nsel) {
+    int acc = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int t = wtot[threadIdx.x][w];
+      wtot[threadIdx.x][w] = acc;
+      acc += t;
+    }
+    ctot[threadIdx.x] = acc;
+  }
+  cluster.sync();
+  const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int sidx = 0; sidx < nsel; ++sidx) {
+    int gt_before = wtot[2 * sidx][wid], eq_before = wtot[2 * sidx + 1][wid];
+    for (int rk = 0; rk < c; ++rk) {
+      const int* rt = cluster.map_shared_rank(ctot, rk);
+      gt_before += rt[2 * sidx];
+      eq_before += rt[2 * sidx + 1];
+    }
+    const SelState& s = sel[sidx];
+#pragma unroll
+    for (int j = 0; j < PT; ++j) {
+      const bool v = (vmask >> j) & 1u;
+      const bool gt = v && key[j] > s.T;
+      const bool eq = v && key[j] == s.T;
+      const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+      const int g_here = gt_before + __popc(bg & lt_mask);
+      const int e_here = eq_before + __popc(be & lt_mask);
+      if (gt || (eq && e_here < s.need_eq)) {
+        const int rank = g_here + min(e_here, s.need_eq);
+        if (rank < kk[sidx]) {
+          const int64_t pos = base_w + static_cast<int64_t>(j) * 32 + lane;
+          oidx[sidx][rank] = map ? map[pos] : static_cast<int32_t>(pos);
+          if (osc[sidx]) osc[sidx][rank] = row[pos];
+        }
+      }
+      gt_before += __popc(bg);
+      eq_before += __popc(be);
+    }
+  }
+  cluster.sync();   // the counts of this CTA may be read until everyone is past here
+}
+
+template <int PT>
+cudaError_t launch_cluster_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, a.rows, 1);
+  cfg.blockDim = dim3(kClusterThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<PT>, a, o2);
+}
+
+}  // namespace
+
+cudaError_t launch_topk_cluster(const TopkArgs& a, const TopkOut2& o2, cudaStream_t st, int* cluster_size) {
+  const int64_t n = a.n;
+  int cs = static_cast<int>((n + kClusterThreads * 16 - 1) / (kClusterThreads * 16));
+  cs = cs < 1 ? 1 : (cs > kClusterMaxSize ? kClusterMaxSize : cs);
+  const int64_t per_thread = (n + static_cast<int64_t>(cs) * kClusterThreads - 1) / (static_cast<int64_t>(cs) * kClusterThreads);
+  if (cluster_size) *cluster_size = cs;
+  if (per_thread <= 4) return launch_cluster_pt<4>(a, o2, cs, st);
+  if (per_thread <= 8) return launch_cluster_pt<8>(a, o2, cs, st);
+  if (per_thread <= 16) return launch_cluster_pt<16>(a, o2, cs, st);
+  if (per_thread <= 32) return launch_cluster_pt<32>(a, o2, cs, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace li

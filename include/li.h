@@ -90,7 +90,9 @@ typedef struct li_ctx li_ctx;
  *         only, NULL otherwise): element value = scale[b][s] * e4m3 code.
  * lengths [batch] int32 valid rows per sequence (read and advanced on the
  *         device by li_append_latent).
- * dim: multiple of 8 (F32), 16 (BF16) or 32 (E4M3), at most 256.           */
+ * dim: multiple of 8 (F32), 16 (BF16) or 32 (E4M3), at most 256.  Scanning
+ * an E4M3 cache (li_score_topk, li_hs_anchor_candidates, li_dsa_score_topk)
+ * needs capacity % 4 == 0 and a 16-byte aligned scale array.                */
 typedef struct {
   void* data;
   float* scale;
@@ -265,6 +267,15 @@ typedef struct {
   int32_t block;         /* threads per CTA                                      */
   int32_t smem;          /* dynamic shared memory bytes per CTA                  */
 } li_profile_record;
+
+/* Diagnostic tile trace of the scoring kernels: when `buf` (device, at least
+ * 8 * 64 * 8 * 8 = 32768 bytes) is set, every later scan / gather launch
+ * writes, for each of its first 8 CTAs and their first 64 tiles, 8 uint64
+ * SM clock-cycle stamps [cta][tile][event] (comparable within one CTA): 0 the loader got the tile's first
+ * stage, 1 it issued the last one, 2 the MMA issuer saw the first stage
+ * full, 3 it committed the tile, 4 the epilogue saw the accumulator full, 5
+ * the epilogue released it.  NULL turns tracing off. */
+LI_API li_status li_set_trace(li_ctx* ctx, void* buf, size_t bytes);
 
 LI_API li_status li_profile_enable(li_ctx* ctx, int enable);
 LI_API li_status li_profile_read(li_ctx* ctx, li_profile_record* out, int max, int* count);

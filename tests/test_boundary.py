@@ -20,8 +20,8 @@ def declared_symbols():
 @pytest.fixture(scope="module")
 def lib():
     if not os.path.exists(LIB):
-        from cross_layer_latent_b200 import build as b
-        b.build()
+        import __graft_entry__
+        __graft_entry__._builder().build()
     return ctypes.CDLL(LIB)
 
 
