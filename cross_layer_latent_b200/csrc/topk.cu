@@ -386,6 +386,8 @@ struct SelState {
   int need_eq;       // elements equal to T that are taken (lowest positions first)
 };
 
+constexpr int kCandCap = 16384;   // boundary-bucket keys a CTA stages in shared memory
+
 // Find the boundary bucket of `need` counting from the top in a 2048-bin
 // histogram whose per-thread bins are held in loc[0..3] (bins hi-1..hi-4).
 __device__ __forceinline__ void find_from_loc(const unsigned (&loc)[4], int hi, int need, int* scratch,
@@ -404,26 +406,20 @@ __device__ __forceinline__ void find_from_loc(const unsigned (&loc)[4], int hi, 
   __syncthreads();
 }
 
-// Remaining two digits over the candidate keys of all CTAs (each CTA's
-// candidates at cand_base + c*E, counts in cnt[c]).
-__device__ void resolve_low_digits(SelState& st, const unsigned* cand_base, int64_t E, const int* cnt, int CS,
-                                   int offset_in_region_sel, unsigned* hist, int* scratch, int* res,
-                                   const int* cnt_other) {
+// Remaining two digits over `m` candidate keys (shared memory).
+__device__ __forceinline__ void resolve_low_digits(SelState& st, const unsigned* cand, int m, unsigned* hist,
+                                                   int* scratch, int* res) {
   int need = st.keff - st.above1;
   unsigned prefix2 = 0;
-#pragma unroll 1
+#pragma unroll
   for (int d = 0; d < 2; ++d) {
     const int nb = d == 0 ? 2048 : 1024;
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int rk = 0; rk < CS; ++rk) {
-      const unsigned* src = cand_base + static_cast<int64_t>(rk) * E + (offset_in_region_sel ? cnt_other[rk] : 0);
-      const int m = cnt[rk];
-      for (int i = threadIdx.x; i < m; i += blockDim.x) {
-        const unsigned key = src[i];
-        if (d == 0) atomicAdd(&hist[(key >> 10) & 2047u], 1u);
-        else if (((key >> 10) & 2047u) == prefix2) atomicAdd(&hist[key & 1023u], 1u);
-      }
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+      const unsigned key = cand[i];
+      if (d == 0) atomicAdd(&hist[(key >> 10) & 2047u], 1u);
+      else if (((key >> 10) & 2047u) == prefix2) atomicAdd(&hist[key & 1023u], 1u);
     }
     __syncthreads();
     find_bucket_desc(hist, nb, need, scratch, res);
@@ -438,56 +434,66 @@ __device__ void resolve_low_digits(SelState& st, const unsigned* cand_base, int6
   st.need_eq = need;
 }
 
-template <int PT>
-__global__ void __launch_bounds__(kClusterThreads) topk_cluster_kernel(const TopkArgs a, const TopkOut2 o2) {
+// Thread t of CTA c owns positions [c*E + t*PT, +PT), E = 512 * PT, as
+// register keys; NSEL budgets (k, and k2 <= k) are selected from them.
+template <int PT, int NSEL>
+__global__ void __launch_bounds__(kClusterThreads, 1) topk_cluster_kernel(const TopkArgs a, const TopkOut2 o2) {
+  extern __shared__ __align__(16) unsigned cand_smem[];   // kCandCap keys
   __shared__ __align__(16) unsigned hist[kHistBins];
   __shared__ int scratch[32];
   __shared__ int res[2];
-  __shared__ int cnt_local[2];                  // candidates of this CTA per budget
-  __shared__ int cnt_all[2][kClusterMaxSize];   // every CTA's, per budget
-  __shared__ int wtot[4][kClusterThreads / 32];
-  __shared__ int ctot[4];                       // (gt, eq) per budget of this CTA
+  __shared__ int cnt_local[2];                  // candidates of this CTA per bucket
+  __shared__ int ctot[2 * NSEL];                // (gt, eq) per budget of this CTA
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = static_cast<int>(cluster.num_blocks());
   const int c = static_cast<int>(cluster.block_rank());
   const int r = blockIdx.y;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int n = row_len(a, r);
-  const int nsel = o2.k2 > 0 ? 2 : 1;
-  SelState sel[2];
+  SelState sel[NSEL];
   sel[0].keff = min(a.k, n);
-  sel[1].keff = min(o2.k2, n);
-  int32_t* oidx[2] = {a.out_idx + static_cast<int64_t>(r) * a.k,
-                      o2.k2 ? o2.out_idx2 + static_cast<int64_t>(r) * o2.k2 : nullptr};
-  float* osc[2] = {a.out_score ? a.out_score + static_cast<int64_t>(r) * a.k : nullptr,
-                   (o2.k2 && o2.out_score2) ? o2.out_score2 + static_cast<int64_t>(r) * o2.k2 : nullptr};
-  const int kk[2] = {a.k, o2.k2};
+  if (NSEL == 2) sel[NSEL - 1].keff = min(o2.k2, n);
   if (c == 0) {
-    for (int sidx = 0; sidx < nsel; ++sidx)
-      for (int j = max(sel[sidx].keff, 0) + threadIdx.x; j < kk[sidx]; j += blockDim.x) {
-        oidx[sidx][j] = -1;
-        if (osc[sidx]) osc[sidx][j] = -INFINITY;
+#pragma unroll
+    for (int si = 0; si < NSEL; ++si) {
+      const int kk = si == 0 ? a.k : o2.k2;
+      int32_t* oi = (si == 0 ? a.out_idx : o2.out_idx2) + static_cast<int64_t>(r) * kk;
+      float* osv = si == 0 ? a.out_score : o2.out_score2;
+      for (int j = max(sel[si].keff, 0) + threadIdx.x; j < kk; j += blockDim.x) {
+        oi[j] = -1;
+        if (osv) osv[static_cast<int64_t>(r) * kk + j] = -INFINITY;
       }
+    }
     if (a.out_count && threadIdx.x == 0) a.out_count[r] = max(sel[0].keff, 0);
   }
   if (sel[0].keff <= 0) return;   // uniform over the cluster (depends on the row only)
 
   const int64_t E = static_cast<int64_t>(kClusterThreads) * PT;
-  const int64_t base_w = static_cast<int64_t>(c) * E + static_cast<int64_t>(wid) * 32 * PT;
+  const int64_t p0 = static_cast<int64_t>(c) * E + static_cast<int64_t>(threadIdx.x) * PT;
   const float* row = a.scores + static_cast<int64_t>(r) * a.row_stride;
   unsigned key[PT];
   unsigned vmask = 0;
+  if ((a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0 && p0 + PT <= n) {
 #pragma unroll
-  for (int j = 0; j < PT; ++j) {
-    const int64_t pos = base_w + static_cast<int64_t>(j) * 32 + lane;
-    key[j] = 0;
-    if (pos < n) {
-      key[j] = radix_key(row[pos]);
-      vmask |= 1u << j;
+    for (int j = 0; j < PT; j += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(row + p0 + j);
+      key[j] = radix_key(f.x);
+      key[j + 1] = radix_key(f.y);
+      key[j + 2] = radix_key(f.z);
+      key[j + 3] = radix_key(f.w);
+    }
+    vmask = PT == 32 ? 0xffffffffu : ((1u << PT) - 1u);
+  } else {
+#pragma unroll
+    for (int j = 0; j < PT; ++j) {
+      key[j] = 0;
+      if (p0 + j < n) {
+        key[j] = radix_key(row[p0 + j]);
+        vmask |= 1u << j;
+      }
     }
   }
 
-  // ---- 1. first digit
+  // ---- 1. first digit: histograms summed over the cluster
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
   __syncthreads();
 #pragma unroll
@@ -505,112 +511,160 @@ __global__ void __launch_bounds__(kClusterThreads) topk_cluster_kernel(const Top
     for (int rk = 0; rk < kClusterMaxSize; ++rk)
       if (rk < CS) { loc[3] += parts[rk].x; loc[2] += parts[rk].y; loc[1] += parts[rk].z; loc[0] += parts[rk].w; }
   }
-  for (int sidx = 0; sidx < nsel; ++sidx) {
-    find_from_loc(loc, hi, sel[sidx].keff, scratch, res);
-    sel[sidx].b1 = static_cast<unsigned>(res[0]);
-    sel[sidx].above1 = res[1];
-    sel[sidx].n_gt = res[1];
+#pragma unroll
+  for (int si = 0; si < NSEL; ++si) {
+    find_from_loc(loc, hi, sel[si].keff, scratch, res);
+    sel[si].b1 = static_cast<unsigned>(res[0]);
+    sel[si].above1 = res[1];
+    sel[si].n_gt = res[1];
     __syncthreads();
   }
 
-  // ---- 2. compact this CTA's boundary-bucket keys (budget 0, then budget 1
-  //         if its bucket differs) into its workspace region
-  unsigned* region = reinterpret_cast<unsigned*>(a.cand) + static_cast<int64_t>(r) * a.n + static_cast<int64_t>(c) * E;
-  const bool two_buckets = nsel == 2 && sel[1].b1 != sel[0].b1;
-  int written = 0;
-  for (int sidx = 0; sidx < (two_buckets ? 2 : 1); ++sidx) {
-    const unsigned b1 = sel[sidx].b1;
-    int mine = 0;
-#pragma unroll
-    for (int j = 0; j < PT; ++j) mine += (((vmask >> j) & 1u) && (key[j] >> 21) == b1) ? 1 : 0;
-    int tot = 0;
-    int off = block_excl_scan(mine, scratch, &tot);
-#pragma unroll
-    for (int j = 0; j < PT; ++j)
-      if (((vmask >> j) & 1u) && (key[j] >> 21) == b1) region[written + off++] = key[j];
-    if (threadIdx.x == 0) cnt_local[sidx] = tot;
-    written += tot;
-    __syncthreads();
-  }
-  if (!two_buckets && threadIdx.x == 0) cnt_local[1] = 0;
-  cluster.sync();
-  if (threadIdx.x < CS) {
-    const int* rc = cluster.map_shared_rank(cnt_local, static_cast<int>(threadIdx.x));
-    cnt_all[0][threadIdx.x] = rc[0];
-    cnt_all[1][threadIdx.x] = rc[1];
-  }
-  __syncthreads();
-  const unsigned* cand_base = reinterpret_cast<const unsigned*>(a.cand) + static_cast<int64_t>(r) * a.n;
-  resolve_low_digits(sel[0], cand_base, E, cnt_all[0], CS, 0, hist, scratch, res, cnt_all[0]);
-  if (nsel == 2) {
-    if (two_buckets)
-      resolve_low_digits(sel[1], cand_base, E, cnt_all[1], CS, 1, hist, scratch, res, cnt_all[0]);
-    else
-      resolve_low_digits(sel[1], cand_base, E, cnt_all[0], CS, 0, hist, scratch, res, cnt_all[0]);
-  }
-
-  // ---- 3. ordered output
-  int gtw[2] = {0, 0}, eqw[2] = {0, 0};
-#pragma unroll
-  for (int j = 0; j < PT; ++j) {
-    const bool v = (vmask >> j) & 1u;
-    for (int sidx = 0; sidx < nsel; ++sidx) {
-      gtw[sidx] += __popc(__ballot_sync(0xffffffffu, v && key[j] > sel[sidx].T));
-      eqw[sidx] += __popc(__ballot_sync(0xffffffffu, v && key[j] == sel[sidx].T));
-    }
-  }
-  if (lane == 0)
-    for (int sidx = 0; sidx < nsel; ++sidx) { wtot[2 * sidx][wid] = gtw[sidx]; wtot[2 * sidx + 1][wid] = eqw[sidx]; }
-  __syncthreads();
-  if (threadIdx.x < 2 * nsel) {
-    int acc = 0;
-    for (int w = 0; w < nw; ++w) {
-      const int t = wtot[threadIdx.x][w];
-      wtot[threadIdx.x][w] = acc;
-      acc += t;
-    }
-    ctot[threadIdx.x] = acc;
-  }
-  cluster.sync();
-  const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int sidx = 0; sidx < nsel; ++sidx) {
-    int gt_before = wtot[2 * sidx][wid], eq_before = wtot[2 * sidx + 1][wid];
-    for (int rk = 0; rk < c; ++rk) {
-      const int* rt = cluster.map_shared_rank(ctot, rk);
-      gt_before += rt[2 * sidx];
-      eq_before += rt[2 * sidx + 1];
-    }
-    const SelState& s = sel[sidx];
+  // ---- 2. this CTA's boundary-bucket keys -> its workspace region
+  //         (bucket of budget 0, then budget 1's if it differs)
+  const bool two = NSEL == 2 && sel[NSEL - 1].b1 != sel[0].b1;
+  unsigned* rowcand = reinterpret_cast<unsigned*>(a.cand) + static_cast<int64_t>(r) * a.n;
+  {
+    int m0 = 0, m1 = 0;
 #pragma unroll
     for (int j = 0; j < PT; ++j) {
       const bool v = (vmask >> j) & 1u;
-      const bool gt = v && key[j] > s.T;
-      const bool eq = v && key[j] == s.T;
-      const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
-      const int g_here = gt_before + __popc(bg & lt_mask);
-      const int e_here = eq_before + __popc(be & lt_mask);
-      if (gt || (eq && e_here < s.need_eq)) {
-        const int rank = g_here + min(e_here, s.need_eq);
-        if (rank < kk[sidx]) {
-          const int64_t pos = base_w + static_cast<int64_t>(j) * 32 + lane;
-          oidx[sidx][rank] = map ? map[pos] : static_cast<int32_t>(pos);
-          if (osc[sidx]) osc[sidx][rank] = row[pos];
+      const unsigned d = key[j] >> 21;
+      m0 += (v && d == sel[0].b1) ? 1 : 0;
+      m1 += (v && two && d == sel[NSEL - 1].b1) ? 1 : 0;
+    }
+    int tot = 0;
+    const int off = block_excl_scan(m0 | (m1 << 16), scratch, &tot);   // both counts < 2^15
+    int o0 = off & 0xFFFF, o1 = (off >> 16) + (tot & 0xFFFF);
+    unsigned* region = rowcand + static_cast<int64_t>(c) * E;
+#pragma unroll
+    for (int j = 0; j < PT; ++j) {
+      const bool v = (vmask >> j) & 1u;
+      const unsigned d = key[j] >> 21;
+      if (v && d == sel[0].b1) region[o0++] = key[j];
+      else if (v && two && d == sel[NSEL - 1].b1) region[o1++] = key[j];
+    }
+    if (threadIdx.x == 0) { cnt_local[0] = tot & 0xFFFF; cnt_local[1] = tot >> 16; }
+  }
+  cluster.sync();
+  // stage every CTA's keys of one bucket in shared memory, resolve the two
+  // remaining digits there (each CTA redundantly: no broadcast needed)
+#pragma unroll
+  for (int si = 0; si < NSEL; ++si) {
+    const int bk = (si == 1 && two) ? 1 : 0;
+    int m = 0;
+    for (int rk = 0; rk < CS; ++rk) {
+      const int* rc = cluster.map_shared_rank(cnt_local, rk);
+      const int cnt = rc[bk];
+      const unsigned* src = rowcand + static_cast<int64_t>(rk) * E + (bk ? rc[0] : 0);
+      for (int i = threadIdx.x; i < cnt; i += blockDim.x)
+        if (m + i < kCandCap) cand_smem[m + i] = src[i];
+      m += cnt;
+    }
+    __syncthreads();
+    if (m <= kCandCap) {
+      resolve_low_digits(sel[si], cand_smem, m, hist, scratch, res);
+    } else {
+      // more boundary keys than shared memory holds (heavy ties): resolve from
+      // the workspace copies, one CTA region after the other
+      int need = sel[si].keff - sel[si].above1;
+      unsigned prefix2 = 0;
+#pragma unroll 1
+      for (int d = 0; d < 2; ++d) {
+        const int nb = d == 0 ? 2048 : 1024;
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        for (int rk = 0; rk < CS; ++rk) {
+          const int* rc = cluster.map_shared_rank(cnt_local, rk);
+          const int cnt = rc[bk];
+          const unsigned* src = rowcand + static_cast<int64_t>(rk) * E + (bk ? rc[0] : 0);
+          for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+            const unsigned kq = src[i];
+            if (d == 0) atomicAdd(&hist[(kq >> 10) & 2047u], 1u);
+            else if (((kq >> 10) & 2047u) == prefix2) atomicAdd(&hist[kq & 1023u], 1u);
+          }
+        }
+        __syncthreads();
+        find_bucket_desc(hist, nb, need, scratch, res);
+        const unsigned bin = static_cast<unsigned>(res[0]);
+        const int above = res[1];
+        __syncthreads();
+        need -= above;
+        sel[si].n_gt += above;
+        if (d == 0) prefix2 = bin;
+        else sel[si].T = (sel[si].b1 << 21) | (prefix2 << 10) | bin;
+      }
+      sel[si].need_eq = need;
+    }
+    __syncthreads();
+  }
+
+  // ---- 3. ordered output: rank = #greater before + min(#equal before, need_eq)
+  int off_gt[NSEL], off_eq[NSEL];
+#pragma unroll
+  for (int si = 0; si < NSEL; ++si) {
+    int g = 0, e = 0;
+#pragma unroll
+    for (int j = 0; j < PT; ++j) {
+      const bool v = (vmask >> j) & 1u;
+      g += (v && key[j] > sel[si].T) ? 1 : 0;
+      e += (v && key[j] == sel[si].T) ? 1 : 0;
+    }
+    int tot = 0;
+    const int off = block_excl_scan(g | (e << 16), scratch, &tot);
+    off_gt[si] = off & 0xFFFF;
+    off_eq[si] = off >> 16;
+    if (threadIdx.x == 0) { ctot[2 * si] = tot & 0xFFFF; ctot[2 * si + 1] = tot >> 16; }
+  }
+  cluster.sync();
+  for (int rk = 0; rk < c; ++rk) {
+    const int* rt = cluster.map_shared_rank(ctot, rk);
+#pragma unroll
+    for (int si = 0; si < NSEL; ++si) { off_gt[si] += rt[2 * si]; off_eq[si] += rt[2 * si + 1]; }
+  }
+  const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
+#pragma unroll
+  for (int si = 0; si < NSEL; ++si) {
+    const int kk = si == 0 ? a.k : o2.k2;
+    int32_t* oi = (si == 0 ? a.out_idx : o2.out_idx2) + static_cast<int64_t>(r) * kk;
+    float* osv = si == 0 ? a.out_score : o2.out_score2;
+    if (osv) osv += static_cast<int64_t>(r) * kk;
+    int gb = off_gt[si], eb = off_eq[si];
+    const unsigned T = sel[si].T;
+    const int need_eq = sel[si].need_eq;
+#pragma unroll
+    for (int j = 0; j < PT; ++j) {
+      const bool v = (vmask >> j) & 1u;
+      const bool gt = v && key[j] > T;
+      const bool eq = v && key[j] == T;
+      if (gt || (eq && eb < need_eq)) {
+        const int rank = gb + min(eb, need_eq);
+        if (rank < kk) {
+          const int64_t pos = p0 + j;
+          oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
+          if (osv) osv[rank] = row[pos];
         }
       }
-      gt_before += __popc(bg);
-      eq_before += __popc(be);
+      gb += gt ? 1 : 0;
+      eb += eq ? 1 : 0;
     }
   }
   cluster.sync();   // the counts of this CTA may be read until everyone is past here
 }
 
-template <int PT>
+template <int PT, int NSEL>
 cudaError_t launch_cluster_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
+  auto k = topk_cluster_kernel<PT, NSEL>;
+  const int dyn = kCandCap * 4;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, a.rows, 1);
   cfg.blockDim = dim3(kClusterThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = dyn;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -619,7 +673,12 @@ cudaError_t launch_cluster_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cud
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<PT>, a, o2);
+  return cudaLaunchKernelEx(&cfg, k, a, o2);
+}
+
+template <int PT>
+cudaError_t launch_cluster_sel(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
+  return o2.k2 > 0 ? launch_cluster_pt<PT, 2>(a, o2, cs, st) : launch_cluster_pt<PT, 1>(a, o2, cs, st);
 }
 
 }  // namespace
@@ -630,10 +689,10 @@ cudaError_t launch_topk_cluster(const TopkArgs& a, const TopkOut2& o2, cudaStrea
   cs = cs < 1 ? 1 : (cs > kClusterMaxSize ? kClusterMaxSize : cs);
   const int64_t per_thread = (n + static_cast<int64_t>(cs) * kClusterThreads - 1) / (static_cast<int64_t>(cs) * kClusterThreads);
   if (cluster_size) *cluster_size = cs;
-  if (per_thread <= 4) return launch_cluster_pt<4>(a, o2, cs, st);
-  if (per_thread <= 8) return launch_cluster_pt<8>(a, o2, cs, st);
-  if (per_thread <= 16) return launch_cluster_pt<16>(a, o2, cs, st);
-  if (per_thread <= 32) return launch_cluster_pt<32>(a, o2, cs, st);
+  if (per_thread <= 4) return launch_cluster_sel<4>(a, o2, cs, st);
+  if (per_thread <= 8) return launch_cluster_sel<8>(a, o2, cs, st);
+  if (per_thread <= 16) return launch_cluster_sel<16>(a, o2, cs, st);
+  if (per_thread <= 32) return launch_cluster_sel<32>(a, o2, cs, st);
   return cudaErrorInvalidValue;
 }
 
