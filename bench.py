@@ -23,7 +23,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -48,6 +47,7 @@ def parse():
     p.add_argument("--workload", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-other-contexts", action="store_true")
     return p.parse_args()
 
 
@@ -123,67 +123,123 @@ def run_reference(args):
     return 0
 
 
-def cpu_baseline(inp, hnew, Wd, Wk, budget_s=20.0):
+def cpu_baseline(inp, hnew, Wd, Wk, budget_s=10.0):
     keys, t0 = 0, time.perf_counter()
     reps = 0
     while True:
         keys += oracle_sample_step(inp, reps % inp.wl.batch, hnew, Wd, Wk)
         reps += 1
-        if time.perf_counter() - t0 > budget_s / 2 or reps >= inp.wl.batch:
+        if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
     return {"value": keys / dt, "unit": "keys/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"{reps} of {inp.wl.batch} sequences of one step (HS + DSA-style), fp64 NumPy, {dt:.1f} s"}
+            "sample": f"{reps} sequence-steps (HS + DSA-style group step of one sequence, cycling over the "
+                      f"{inp.wl.batch} sequences), fp64 NumPy, {dt:.1f} s"}
 
 
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, power and clock-event reasons through NVML in a
+    background thread while the timed region runs."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, period_s=0.005):
         self.dev = device_index
-        self.proc = None
+        self.period = period_s
+        self.samples = []
+        self.error = None
+        self.nv = None
+        self.handle = None
+
+    def _open(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        self.nv = nv
+        props = torch.cuda.get_device_properties(self.dev)
+        h = None
+        uuid = str(getattr(props, "uuid", "") or "")
+        if uuid:
+            for cand in (uuid if uuid.startswith("GPU-") else "GPU-" + uuid, uuid):
+                try:
+                    h = nv.nvmlDeviceGetHandleByUUID(cand)
+                    break
+                except Exception:
+                    h = None
+        if h is None and hasattr(props, "pci_bus_id"):
+            bus = f"{getattr(props, 'pci_domain_id', 0):08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                h = None
+        if h is None:
+            h = nv.nvmlDeviceGetHandleByIndex(self.dev)
+        self.handle = h
+        self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+    def _sample(self):
+        nv, h = self.nv, self.handle
+        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        try:
+            reasons = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+        except Exception:
+            reasons = int(nv.nvmlDeviceGetCurrentClocksThrottleReasons(h))
+        try:
+            power = nv.nvmlDeviceGetPowerUsage(h) / 1e3
+        except Exception:
+            power = None
+        self.samples.append((sm, reasons, power))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception as e:  # keep the timing run alive; report the failure
+                self.error = repr(e)
+                return
+            self._stop.wait(self.period)
 
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self.thread = None
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+            self._open()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        except Exception as e:
+            self.error = repr(e)
         return self
 
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc:
-            self.proc.terminate()
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self._sample()
             except Exception:
-                self.proc.kill()
-                out = ""
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                pass
 
     def summary(self):
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
-            except ValueError:
-                continue
-            for nme, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nme)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
+               "samples": len(self.samples), "source": "NVML, sampled every 5 ms during the timed region"}
+        if self.samples:
+            out["sm_mhz"] = statistics.median(x[0] for x in self.samples)
+            seen = 0
+            for _, r, _ in self.samples:
+                seen |= r
+            out["reasons"] = sorted(name for name, attr in self.REASONS
+                                    if hasattr(self.nv, attr) and seen & int(getattr(self.nv, attr)))
+            pw = [x[2] for x in self.samples if x[2] is not None]
+            if pw:
+                out["power_w_max"] = max(pw)
+        if self.error:
+            out["error"] = self.error
+        return out
 
 
 # ------------------------------------------------------------------ roofline inputs
@@ -220,6 +276,147 @@ def profiled_traffic(kind):
 
 # ------------------------------------------------------------------ GPU leg
 
+class Step:
+    """One group decode step of a workload, set up on the device: the HS path
+    and the DSA-style path as callables that issue the library calls, and the
+    same two captured once as CUDA graphs."""
+
+    def __init__(self, li, ctx, wl, rank, dev):
+        self.li, self.ctx, self.wl, self.dev = li, ctx, wl, dev
+        inp = generate(wl, seed=wl.seed + 1000 * rank)
+        hnew, Wd, Wk = construction_inputs(wl, seed=wl.seed + 1000 * rank)
+        self.inp, self.hnew, self.Wd, self.Wk = inp, hnew, Wd, Wk
+        dt_code = {"f32": li.LI_F32, "bf16": li.LI_BF16, "e4m3": li.LI_E4M3}[wl.cache_dtype]
+        g = li.GroupIndexer(ctx, batch=wl.batch, capacity=wl.capacity, d_c=wl.d_c, H=wl.heads, d_k=wl.d_k,
+                            G=wl.group, dtype=dt_code, k=wl.k, B=wl.B, T=wl.queries, dsa=True, device=dev)
+        g.load(inp.lengths, inp.W_K, inp.q, inp.w, latent=inp.latent, hidden=inp.hidden, W_down=inp.W_down,
+               q_pos=inp.q_pos)
+        self.g = g
+        lengths = torch.from_numpy(inp.lengths).to(dev)
+        self.len_before = (lengths - 1).to(torch.int32)
+        bf = torch.bfloat16
+        self.h_anchor = torch.from_numpy(hnew).to(dev, bf)
+        self.h_layers = [torch.from_numpy(hnew).to(dev, bf) for _ in range(wl.group)]
+        self.W_down = torch.from_numpy(Wd).to(dev, bf)
+        self.W_k = [torch.from_numpy(x).to(dev, bf) for x in Wk]
+        self.W_K = [torch.from_numpy(x).to(dev, bf) for x in inp.W_K]
+        self.q = [torch.from_numpy(x).to(dev, bf) for x in inp.q]
+        self.w = [torch.from_numpy(x).to(dev) for x in inp.w]
+        self.hs_keys, self.dsa_keys = keys_per_step(wl, inp.lengths)
+        self.graphs = None
+
+    def reset(self):
+        """Undo the step's appends, so every step sees the same lengths."""
+        self.g.latent.lengths.copy_(self.len_before)
+        for kc in self.g.keys:
+            kc.lengths.copy_(self.len_before)
+
+    def hs_path(self):
+        li, g, wl = self.li, self.g, self.wl
+        g.append(self.h_anchor, self.W_down)
+        for l in range(wl.group):
+            g.w[l].copy_(self.w[l])
+            li.li_absorb_query(self.ctx, self.q[l], self.W_K[l], wl.d_c, g.dtype, g.q_abs[l], g.q_abs_scale[l])
+        g.hs_anchor(0)
+        for l in range(1, wl.group):
+            g.hs_follower(l)
+
+    def dsa_path(self):
+        li, g, wl = self.li, self.g, self.wl
+        for l in range(wl.group):
+            g.append_keys(l, self.h_layers[l], self.W_k[l])
+            li.li_absorb_query(self.ctx, self.q[l], None, wl.d_k, g.dtype, g.q_raw[l], g.q_raw_scale[l])
+            g.dsa_score_topk(l)
+
+    def capture(self):
+        side = torch.cuda.Stream(self.dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):       # warm the caching allocator outside capture
+            self.reset()
+            self.hs_path()
+            self.dsa_path()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.reset()
+        hs, dsa = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(hs):
+            self.hs_path()
+        with torch.cuda.graph(dsa):
+            self.dsa_path()
+        torch.cuda.synchronize()
+        self.graphs = (hs, dsa)
+
+    def status(self, when):
+        st = self.li.li_device_status(self.ctx, self.g.ws)
+        if st != "LI_OK":
+            raise RuntimeError(f"device status {when}: {st}")
+
+
+def timed_steps(step, steps, flush, stream, graphs):
+    """Times `steps` group steps with CUDA events on the launching stream;
+    L2 is flushed (a 256 MiB write) before every step, outside the events.
+    Returns per-step (hs_ms, dsa_ms)."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        step.reset()
+        ev[i][0].record(stream)
+        if graphs:
+            graphs[0].replay()
+        else:
+            step.hs_path()
+        ev[i][1].record(stream)
+        if graphs:
+            graphs[1].replay()
+        else:
+            step.dsa_path()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    return [e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev]
+
+
+def profiled_steps(step, steps, flush, stream, lead_ms=4.0):
+    """The same steps again, eager, with the library's launch profile on (a
+    CUDA event pair around every kernel). A bounded spin kernel queued ahead
+    of each step keeps the GPU busy while the host issues the whole step, so
+    no host-side launch gap falls between an event pair. Returns every launch
+    record and the per-step path times."""
+    li, ctx = step.li, step.ctx
+    cycles = int(lead_ms * 1e-3 * 2.0e9)
+    li.li_profile_reset(ctx)
+    recs, hs_ms, dsa_ms = [], [], []
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        step.reset()
+        torch.cuda._sleep(cycles)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        li.li_profile_enable(ctx, True)
+        e[0].record(stream)
+        step.hs_path()
+        e[1].record(stream)
+        step.dsa_path()
+        e[2].record(stream)
+        li.li_profile_enable(ctx, False)
+        torch.cuda.synchronize()
+        hs_ms.append(e[0].elapsed_time(e[1]))
+        dsa_ms.append(e[1].elapsed_time(e[2]))
+        recs += li.li_profile_read(ctx)
+        li.li_profile_reset(ctx)
+    return recs, hs_ms, dsa_ms
+
+
+def max_over_ranks(x, dist, dev):
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def row_bytes(wl, dim):
+    el = {"e4m3": 1, "bf16": 2, "f32": 4}[wl.cache_dtype]
+    return dim * el + (4 if wl.cache_dtype == "e4m3" else 0)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -236,107 +433,55 @@ def main():
 
     import cross_layer_latent_b200 as li
 
-    wl = workload(args.workload)
     dev = f"cuda:{local}"
-    inp = generate(wl, seed=wl.seed + 1000 * rank)
-    hnew, Wd, Wk = construction_inputs(wl, seed=wl.seed + 1000 * rank)
     ctx = li.Context(local)
-    dt_code = {"f32": li.LI_F32, "bf16": li.LI_BF16, "e4m3": li.LI_E4M3}[wl.cache_dtype]
-    g = li.GroupIndexer(ctx, batch=wl.batch, capacity=wl.capacity, d_c=wl.d_c, H=wl.heads, d_k=wl.d_k,
-                        G=wl.group, dtype=dt_code, k=wl.k, B=wl.B, T=wl.queries, dsa=True, device=dev)
-    g.load(inp.lengths, inp.W_K, inp.q, inp.w, latent=inp.latent, hidden=inp.hidden, W_down=inp.W_down,
-           q_pos=inp.q_pos)
-    lengths = torch.from_numpy(inp.lengths).to(dev)
-    len_before = (lengths - 1).to(torch.int32)
-    bf = torch.bfloat16
-    h_anchor = torch.from_numpy(hnew).to(dev, bf)
-    h_layers = [torch.from_numpy(hnew).to(dev, bf) for _ in range(wl.group)]
-    W_down = torch.from_numpy(Wd).to(dev, bf)
-    W_k = [torch.from_numpy(x).to(dev, bf) for x in Wk]
-    W_K = [torch.from_numpy(x).to(dev, bf) for x in inp.W_K]
-    q = [torch.from_numpy(x).to(dev, bf) for x in inp.q]
-    w = [torch.from_numpy(x).to(dev) for x in inp.w]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    hs_keys, dsa_keys = keys_per_step(wl, inp.lengths)
-
-    def reset():
-        g.latent.lengths.copy_(len_before)
-        for kc in g.keys:
-            kc.lengths.copy_(len_before)
-
-    def hs_path():
-        g.append(h_anchor, W_down)
-        for l in range(wl.group):
-            g.w[l].copy_(w[l])
-            li.li_absorb_query(ctx, q[l], W_K[l], wl.d_c, g.dtype, g.q_abs[l], g.q_abs_scale[l])
-        g.hs_anchor(0)
-        for l in range(1, wl.group):
-            g.hs_follower(l)
-
-    def dsa_path():
-        for l in range(wl.group):
-            g.append_keys(l, h_layers[l], W_k[l])
-            li.li_absorb_query(ctx, q[l], None, wl.d_k, g.dtype, g.q_raw[l], g.q_raw_scale[l])
-            g.dsa_score_topk(l)
-
+    wl = workload(args.workload)
+    step = Step(li, ctx, wl, rank, dev)
     for _ in range(args.warmup):
-        reset()
-        hs_path()
-        dsa_path()
+        step.reset()
+        step.hs_path()
+        step.dsa_path()
     torch.cuda.synchronize()
-    st = li.li_device_status(ctx, g.ws)
-    if st != "LI_OK":
-        raise RuntimeError(f"device status after warm-up: {st}")
+    step.status("after warm-up")
+    step.capture()
+    for _ in range(args.warmup):
+        step.reset()
+        step.graphs[0].replay()
+        step.graphs[1].replay()
+    torch.cuda.synchronize()
+    step.status("after graph warm-up")
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    li.li_profile_reset(ctx)
+    # ---- timed region: the captured step graphs, replayed
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         t_wall = time.perf_counter()
         torch.cuda.nvtx.range_push("timed")
-        li.li_profile_enable(ctx, True)
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            reset()
-            ev[i][0].record(stream)
-            hs_path()
-            ev[i][1].record(stream)
-            dsa_path()
-            ev[i][2].record(stream)
-        li.li_profile_enable(ctx, False)
+        hs_ms, dsa_ms = timed_steps(step, args.steps, flush, stream, step.graphs)
         torch.cuda.nvtx.range_pop()
-        torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    hs_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    dsa_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(hs_ms) + sum(dsa_ms)
-    recs = li.li_profile_read(ctx)
-    li.li_profile_reset(ctx)
-    st = li.li_device_status(ctx, g.ws)
-    if st != "LI_OK":
-        raise RuntimeError(f"device status after the timed steps: {st}")
-
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    keys = hs_keys + dsa_keys
+    step.status("after the timed steps")
+    max_ms = max_over_ranks(sum(hs_ms) + sum(dsa_ms), dist, dev)
+    keys = step.hs_keys + step.dsa_keys
     value = world * keys * args.steps / (max_ms / 1e3)
 
-    # ---- roofline of the dominant kernel (the scan), from the live launch profile
+    # ---- second timed pass, eager, with a CUDA event pair around every launch:
+    #      per-kernel durations for the roofline and the launch count
+    with ClockSampler(local) as clk2:
+        recs, p_hs, p_dsa = profiled_steps(step, args.steps, flush, stream)
+    step.status("after the profiled steps")
+
+    inp = step.inp
     kernels = [r for r in recs if r["kernel"] != "memset"]
     scans = [r for r in recs if r["kernel"] == "scan"]
     per_step = len(scans) // args.steps
-    row_latent = wl.d_c * (1 if wl.cache_dtype == "e4m3" else 2 if wl.cache_dtype == "bf16" else 4) + \
-        (4 if wl.cache_dtype == "e4m3" else 0)
-    row_key = wl.d_k * (1 if wl.cache_dtype == "e4m3" else 2 if wl.cache_dtype == "bf16" else 4) + \
-        (4 if wl.cache_dtype == "e4m3" else 0)
+    row_latent, row_key = row_bytes(wl, wl.d_c), row_bytes(wl, wl.d_k)
     ntok = int(inp.lengths.sum())
     scan_bytes = [ntok * row_latent] + [ntok * row_key] * wl.group      # anchor scan, then 4 DSA scans
     alg_bytes = sum(scan_bytes[j % len(scan_bytes)] for j in range(len(scans)))
@@ -352,6 +497,7 @@ def main():
     for d in by_kernel.values():
         d["ms_per_step"] = d["ms"] / args.steps
         d["ms"] = round(d["ms"], 4)
+    hs_mean, dsa_mean = statistics.mean(hs_ms), statistics.mean(dsa_ms)
 
     out = {"metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
@@ -362,66 +508,99 @@ def main():
                         "kernel": "scan (tcgen05 latent / key scan, fused ReLU-weighted head reduction)",
                         "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                         "alg_bytes_per_key": {"latent": row_latent, "dsa_key": row_key},
-                        "launches_per_step": per_step, "scan_ms_per_step": scan_ms / args.steps},
-           "paths": {"hs_ms": statistics.mean(hs_ms), "dsa_ms": statistics.mean(dsa_ms),
-                     "hs_keys_per_step": hs_keys, "dsa_keys_per_step": dsa_keys,
-                     "hs_keys_per_s": hs_keys / (statistics.mean(hs_ms) / 1e3),
-                     "dsa_keys_per_s": dsa_keys / (statistics.mean(dsa_ms) / 1e3),
-                     "hs_speedup_over_dsa": statistics.mean(dsa_ms) / statistics.mean(hs_ms)},
+                        "launches_per_step": per_step, "scan_ms_per_step": scan_ms / args.steps,
+                        "timing": "CUDA event pair around every launch on the launching stream, in a "
+                                  "second timed pass of the same steps (eager, the GPU kept ahead of the host)"},
+           "paths": {"hs_ms": hs_mean, "dsa_ms": dsa_mean,
+                     "hs_ms_median": statistics.median(hs_ms), "dsa_ms_median": statistics.median(dsa_ms),
+                     "hs_keys_per_step": step.hs_keys, "dsa_keys_per_step": step.dsa_keys,
+                     "hs_keys_per_s": step.hs_keys / (hs_mean / 1e3),
+                     "dsa_keys_per_s": step.dsa_keys / (dsa_mean / 1e3),
+                     "hs_speedup_over_dsa": dsa_mean / hs_mean,
+                     "profiled_hs_ms": statistics.mean(p_hs), "profiled_dsa_ms": statistics.mean(p_dsa)},
            "kernels": by_kernel,
-           "gpu_launches": len(kernels),
+           "gpu_launches": len(kernels) // args.steps * args.steps,
+           "launch_mode": "each path captured once as a CUDA graph and replayed per step",
            "wall_s_timed_loop": t_wall}
     out["clocks"] = clk.summary()
+    out["clocks_profiled_pass"] = clk2.summary()
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers (eager calls)
     if not args.no_e2e:
+        bf = torch.bfloat16
         pin = lambda x: torch.from_numpy(np.ascontiguousarray(x)).pin_memory()  # noqa: E731
-        host_in = {"h_anchor": pin(hnew.astype(np.float32)).to(bf).pin_memory(),
-                   "h_layers": [pin(hnew.astype(np.float32)).to(bf).pin_memory() for _ in range(wl.group)],
+        host_in = {"h_anchor": pin(step.hnew.astype(np.float32)).to(bf).pin_memory(),
+                   "h_layers": [pin(step.hnew.astype(np.float32)).to(bf).pin_memory() for _ in range(wl.group)],
                    "q": [pin(x).to(bf).pin_memory() for x in inp.q], "w": [pin(x) for x in inp.w]}
         host_out = [torch.empty(wl.batch, 1, wl.k, dtype=torch.int32).pin_memory() for _ in range(2 * wl.group)]
         h2d = host_in["h_anchor"].numel() * 2 + sum(x.numel() * 2 for x in host_in["h_layers"]) + \
             sum(x.numel() * 2 for x in host_in["q"]) + sum(x.numel() * 4 for x in host_in["w"])
         d2h = sum(x.numel() * 4 for x in host_out)
+        g = step.g
 
         def e2e_step():
-            h_anchor.copy_(host_in["h_anchor"], non_blocking=True)
+            step.h_anchor.copy_(host_in["h_anchor"], non_blocking=True)
             for l in range(wl.group):
-                h_layers[l].copy_(host_in["h_layers"][l], non_blocking=True)
-                q[l].copy_(host_in["q"][l], non_blocking=True)
-                w[l].copy_(host_in["w"][l], non_blocking=True)
-            hs_path()
+                step.h_layers[l].copy_(host_in["h_layers"][l], non_blocking=True)
+                step.q[l].copy_(host_in["q"][l], non_blocking=True)
+                step.w[l].copy_(host_in["w"][l], non_blocking=True)
+            step.hs_path()
             hs_idx = [x.clone() for x in g.idx]
-            dsa_path()
+            step.dsa_path()
             for l in range(wl.group):
                 host_out[l].copy_(hs_idx[l], non_blocking=True)
                 host_out[wl.group + l].copy_(g.idx[l], non_blocking=True)
 
         for _ in range(2):
-            reset()
+            step.reset()
             e2e_step()
         torch.cuda.synchronize()
         e2e_ms = []
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
-            reset()
+            step.reset()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             e2e_step()
             e1.record(stream)
             e1.synchronize()
             e2e_ms.append(e0.elapsed_time(e1))
-        te = torch.tensor([sum(e2e_ms)], device=dev, dtype=torch.float64)
-        if dist:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        out["e2e"] = {"value": world * keys * args.steps / (float(te.item()) / 1e3), "unit": "keys/s",
+        te = max_over_ranks(sum(e2e_ms), dist, dev)
+        out["e2e"] = {"value": world * keys * args.steps / (te / 1e3), "unit": "keys/s",
                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                      "ms_per_step": float(te.item()) / args.steps}
+                      "ms_per_step": te / args.steps,
+                      "mode": "eager library calls per step, pinned host inputs in, selected indices out"}
+
+    # ---- HS against DSA-style at the shorter contexts (same library, same protocol)
+    if not args.no_other_contexts:
+        other = {}
+        for idx in (1, 2):
+            if idx == args.workload:
+                continue
+            s2 = Step(li, ctx, workload(idx), rank, dev)
+            for _ in range(args.warmup):
+                s2.reset()
+                s2.hs_path()
+                s2.dsa_path()
+            torch.cuda.synchronize()
+            s2.capture()
+            h2, d2 = timed_steps(s2, args.steps, flush, stream, s2.graphs)
+            s2.status(f"after timing {s2.wl.name}")
+            hm = max_over_ranks(statistics.mean(h2), dist, dev)
+            dm = max_over_ranks(statistics.mean(d2), dist, dev)
+            other[s2.wl.name] = {"hs_ms": hm, "dsa_ms": dm, "hs_speedup_over_dsa": dm / hm,
+                                 "hs_keys_per_s": world * s2.hs_keys / (hm / 1e3),
+                                 "dsa_keys_per_s": world * s2.dsa_keys / (dm / 1e3)}
+            s2.graphs = None
+            del s2
+            torch.cuda.empty_cache()
+        out["paths"]["other_contexts"] = other
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(inp, hnew, Wd, Wk)
+        out["cpu_baseline"] = cpu_baseline(inp, step.hnew, step.Wd, step.Wk)
     if rank == 0:
         print(json.dumps(out))
+    step.graphs = None
     ctx.close()
     if dist:
         dist.barrier()

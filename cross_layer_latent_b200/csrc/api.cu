@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -16,6 +17,38 @@
 #include "sm100.cuh"
 
 using namespace li;
+
+namespace li {
+
+cudaError_t raise_smem_limit(const void* fn, int bytes) {
+  struct Entry {
+    const void* fn;
+    int device;
+    int bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& x : done)
+    if (x.fn == fn && x.device == device && x.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return e;
+  }
+  for (Entry& x : done)
+    if (x.fn == fn && x.device == device) {
+      x.bytes = bytes;
+      return cudaSuccess;
+    }
+  done.push_back({fn, device, bytes});
+  return cudaSuccess;
+}
+
+}  // namespace li
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -569,6 +602,18 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
   float* tmp = at<float>(ws, L.tmp);
   const int eb = elt_bytes(h_dtype);
   const int tchunk = std::max(1, std::min(T, kAppendChunkTok / cache->batch));
+  {
+    const int n_tok = cache->batch * T;
+    const int splits = gemv_splits(d_model, n_tok);
+    if (append_fusable(n_tok, dim, splits)) {
+      Launch Lg(c, st, "append", 0, 256, 0);
+      const cudaError_t e = launch_append_fused(h, h_dtype, W_down, d_model, dim, cache->batch, T, splits, tmp,
+                                                cache->data, cache->scale, cache->lengths, cache->capacity,
+                                                cache->dtype, done, status, st);
+      Lg.done();
+      return e == cudaSuccess ? LI_OK : cuda_fail(c, e, "append launch");
+    }
+  }
   for (int t0 = 0; t0 < T; t0 += tchunk) {
     const int tn = std::min(tchunk, T - t0);
     int splits = 1;

@@ -91,6 +91,129 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const T* __restri
       out[(static_cast<int64_t>(sp) * n_tok + m0 + t) * dim + j] = acc[t];
 }
 
+// Write one fp32 row (lane holds elements lane + 32 e) into the cache at
+// `row` in the cache dtype; e4m3 rows also get their scale amax / 448.
+__device__ __forceinline__ void write_row(const float (&v)[8], float amax, int lane, int64_t row, int dim, int dtype,
+                                          void* data, float* scale) {
+  if (dtype == LI_F32) {
+    float* dst = reinterpret_cast<float*>(data) + row * dim;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (lane + 32 * e < dim) dst[lane + 32 * e] = v[e];
+  } else if (dtype == LI_BF16) {
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(data) + row * dim;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (lane + 32 * e < dim) dst[lane + 32 * e] = __float2bfloat16_rn(v[e]);
+  } else {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    uint8_t* dst = reinterpret_cast<uint8_t*>(data) + row * dim;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (lane + 32 * e < dim) dst[lane + 32 * e] = to_e4m3(__fdiv_rn(v[e], sc));
+    if (lane == 0) scale[row] = sc;
+  }
+}
+
+// Decode append in one launch: the split-K GEMV above, after which the last
+// block to finish (a counter in the workspace) adds every token's splits in
+// split order, quantises the rows, writes them at lengths[b] + t, advances
+// lengths[b] by T and resets the counter. Used when all tokens' fp32 rows fit
+// in the block's shared memory.
+constexpr int kFuseMaxFloats = 8192;
+
+template <typename T>
+__global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* __restrict__ h,
+                                                                      const T* __restrict__ W, int d_model,
+                                                                      int dim, int n_tok, int splits,
+                                                                      float* __restrict__ part, int batch, int T_tok,
+                                                                      void* data, float* scale, int32_t* lengths,
+                                                                      int capacity, int dtype,
+                                                                      unsigned int* done, int* status) {
+  __shared__ float cs[kFuseMaxFloats];
+  __shared__ unsigned last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int task = blockIdx.x * kGemvWarps + warp;
+  if (task < dim * splits) {
+    const int j = task / splits, sp = task % splits;
+    const int len = d_model / splits;
+    const int i0 = sp * len, i1 = i0 + len;
+    float acc[kGemvTok];
+#pragma unroll
+    for (int t = 0; t < kGemvTok; ++t) acc[t] = 0.f;
+    const T* wrow = W + static_cast<int64_t>(j) * d_model;
+    for (int i = i0 + lane * 8; i < i1; i += 256) {
+      float wv[8];
+      load8<T>(wrow + i, wv);
+#pragma unroll
+      for (int t = 0; t < kGemvTok; ++t) {
+        if (t < n_tok) {
+          float hv[8];
+          load8<T>(h + static_cast<int64_t>(t) * d_model + i, hv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[t] = fmaf(wv[e], hv[e], acc[t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kGemvTok; ++t) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+    }
+    if (lane == 0)
+      for (int t = 0; t < n_tok; ++t) part[(static_cast<int64_t>(sp) * n_tok + t) * dim + j] = acc[t];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(done, 1u) == gridDim.x - 1 ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int x = threadIdx.x; x < n_tok * dim; x += blockDim.x) {
+    // every split's partial in flight at once, then added in split order
+    float pv[kMaxSplits];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+      pv[sp] = sp < splits ? __ldcg(part + static_cast<int64_t>(sp) * n_tok * dim + x) : 0.f;
+    float sum = pv[0];
+#pragma unroll
+    for (int sp = 1; sp < kMaxSplits; ++sp)
+      if (sp < splits) sum += pv[sp];
+    cs[x] = sum;
+  }
+  __syncthreads();
+  for (int m = warp; m < n_tok; m += kGemvWarps) {
+    const int b = m / T_tok, t = m % T_tok;
+    const int len = lengths[b];
+    if (len < 0 || len + T_tok > capacity) {
+      if (lane == 0) record_status(status, kStatusCapacity);
+      continue;
+    }
+    float v[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = lane + 32 * e;
+      v[e] = i < dim ? cs[m * dim + i] : 0.f;
+      amax = fmaxf(amax, fabsf(v[e]));
+    }
+    write_row(v, amax, lane, static_cast<int64_t>(b) * capacity + len + t, dim, dtype, data, scale);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < batch; ++b) {
+      const int len = lengths[b];
+      if (len >= 0 && len + T_tok <= capacity) lengths[b] = len + T_tok;
+    }
+    *done = 0;
+    __threadfence();
+  }
+}
+
 // One warp per new token: write c (fp32 rows) into the cache at row
 // lengths[b] + t0 + t in the cache dtype.  The last block to finish advances
 // lengths[b] by T_total when `bump` is set (all blocks read lengths first).
@@ -129,26 +252,7 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
         v[e] = x;
         amax = fmaxf(amax, fabsf(v[e]));
       }
-      if (dtype == LI_F32) {
-        float* dst = reinterpret_cast<float*>(data) + row * dim;
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (lane + 32 * e < dim) dst[lane + 32 * e] = v[e];
-      } else if (dtype == LI_BF16) {
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(data) + row * dim;
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (lane + 32 * e < dim) dst[lane + 32 * e] = __float2bfloat16_rn(v[e]);
-      } else {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-        uint8_t* dst = reinterpret_cast<uint8_t*>(data) + row * dim;
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (lane + 32 * e < dim) dst[lane + 32 * e] = to_e4m3(__fdiv_rn(v[e], sc));
-        if (lane == 0) scale[row] = sc;
-      }
+      write_row(v, amax, lane, row, dim, dtype, data, scale);
     }
   }
   if (!bump) return;
@@ -269,6 +373,93 @@ __global__ void __launch_bounds__(256) absorb_kernel(const T* __restrict__ q, in
   }
 }
 
+__device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+
+// Shared decoder (one W_K for every head): rows (token, head) are taken R at a
+// time per block. The decoder is staged once in shared memory with 16-byte
+// loads, the R query rows as fp32; each thread then owns column pairs of a row
+// and accumulates j = 0..d_k-1 in order with fp32 fma (the same order as the
+// per-head kernel above, so both give identical results). A warp per row
+// finally converts the fp32 row to the output dtype.
+template <typename T>
+__global__ void __launch_bounds__(256) absorb_shared_kernel(const T* __restrict__ q, int M, int d_k,
+                                                            const T* __restrict__ W,
+                                                            const float* __restrict__ bK, int d_c, int R,
+                                                            int out_dtype, void* q_abs, float* q_abs_scale,
+                                                            float* beta) {
+  extern __shared__ __align__(16) unsigned char absorb_smem[];
+  T* Ws = reinterpret_cast<T*>(absorb_smem);                                   // [d_k][d_c]
+  float* qs = reinterpret_cast<float*>(absorb_smem + (static_cast<size_t>(d_k) * d_c * sizeof(T) + 15) / 16 * 16);
+  float* os = qs + R * d_k;                                                    // [R][d_c]
+  const int r0 = blockIdx.x * R;
+  const int nr = min(R, M - r0);
+  {
+    // every 16-byte piece of the decoder in flight at once (cp.async), the
+    // query rows meanwhile through registers
+    const int n16 = static_cast<int>(static_cast<size_t>(d_k) * d_c * sizeof(T) / 16);
+    const uint4* src = reinterpret_cast<const uint4*>(W);
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(Ws));
+    for (int x = threadIdx.x; x < n16; x += blockDim.x) cp_async_16(dst + 16u * x, src + x);
+    cp_async_commit();
+    const int nq = nr * d_k;
+    for (int x = threadIdx.x; x < R * d_k; x += blockDim.x)
+      qs[x] = x < nq ? to_f(q[static_cast<int64_t>(r0) * d_k + x]) : 0.f;
+    cp_async_wait_all();
+  }
+  __syncthreads();
+  const int npairs = d_c >> 1;
+  for (int u = threadIdx.x; u < nr * npairs; u += blockDim.x) {
+    const int rr = u / npairs, p = u - rr * npairs;
+    const float* qr = qs + rr * d_k;
+    const T* wc = Ws + 2 * p;
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < d_k; ++j) {
+      const float qv = qr[j];
+      const float2 w2 = load2(wc + static_cast<size_t>(j) * d_c);
+      a0 = fmaf(w2.x, qv, a0);
+      a1 = fmaf(w2.y, qv, a1);
+    }
+    os[rr * d_c + 2 * p] = a0;
+    os[rr * d_c + 2 * p + 1] = a1;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int rr = warp; rr < nr; rr += blockDim.x >> 5) {
+    const int64_t row = r0 + rr;
+    const float* orow = os + rr * d_c;
+    if (beta) {
+      float bsum = 0.f;
+      for (int j = lane; j < d_k; j += 32) bsum = fmaf(qs[rr * d_k + j], bK[j], bsum);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bsum += __shfl_xor_sync(0xffffffffu, bsum, o);
+      if (lane == 0) beta[row] = bsum;
+    }
+    if (out_dtype == LI_F32) {
+      for (int i = lane; i < d_c; i += 32) reinterpret_cast<float*>(q_abs)[row * d_c + i] = orow[i];
+    } else if (out_dtype == LI_BF16) {
+      for (int i = lane; i < d_c; i += 32)
+        reinterpret_cast<__nv_bfloat16*>(q_abs)[row * d_c + i] = __float2bfloat16_rn(orow[i]);
+    } else {
+      float m = 0.f;
+      for (int i = lane; i < d_c; i += 32) m = fmaxf(m, fabsf(orow[i]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const float sc = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+      for (int i = lane; i < d_c; i += 32)
+        reinterpret_cast<uint8_t*>(q_abs)[row * d_c + i] = to_e4m3(__fdiv_rn(orow[i], sc));
+      if (lane == 0) q_abs_scale[row] = sc;
+    }
+  }
+}
+
+size_t absorb_shared_smem(int d_k, int d_c, int R, size_t elt) {
+  return (static_cast<size_t>(d_k) * d_c * elt + 15) / 16 * 16 + static_cast<size_t>(R) * (d_k + d_c) * 4;
+}
+
 }  // namespace
 
 int gemv_splits(int d_model, int n_tok) {
@@ -295,6 +486,27 @@ cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_
   return cudaGetLastError();
 }
 
+bool append_fusable(int n_tok, int dim, int splits) {
+  return n_tok <= kGemvTok && n_tok * dim <= kFuseMaxFloats && dim <= 256;
+  (void)splits;
+}
+
+cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
+                                int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
+                                int dtype, unsigned int* done, int* status, cudaStream_t st) {
+  const int n_tok = batch * T;
+  const int grid = (dim * splits + kGemvWarps - 1) / kGemvWarps;
+  if (h_dtype == LI_BF16)
+    gemv_append_kernel<__nv_bfloat16><<<grid, kGemvWarps * 32, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim, n_tok,
+        splits, part, batch, T, data, scale, lengths, capacity, dtype, done, status);
+  else
+    gemv_append_kernel<float><<<grid, kGemvWarps * 32, 0, st>>>(
+        reinterpret_cast<const float*>(h), reinterpret_cast<const float*>(W), d_model, dim, n_tok, splits, part,
+        batch, T, data, scale, lengths, capacity, dtype, done, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits, int batch,
                                 int T_chunk, int t0, int T_total, bool bump, void* data, float* scale,
                                 int32_t* lengths, int capacity, int dim, int dtype, unsigned int* done_counter,
@@ -309,6 +521,33 @@ cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t sp
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
                           int out_dtype, void* q_abs, float* q_abs_scale, float* beta, cudaStream_t st) {
+  const size_t elt = q_dtype == LI_BF16 ? 2 : 4;
+  const int M = n_tok * H;
+  // shared decoder: rows of R (token, head) pairs; few rows per block at decode
+  // sizes so that the grid covers the GPU, more when there are many queries
+  const int R = M <= 4096 ? 4 : 32;
+  const size_t smem = absorb_shared_smem(d_k, d_c, R, elt);
+  const bool aligned = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (static_cast<size_t>(d_k) * d_c * elt) % 16 == 0;
+  if (W != nullptr && W_head_stride == 0 && b_head_stride == 0 && (d_c & 1) == 0 && aligned &&
+      smem <= 200 * 1024) {
+    const int grid = (M + R - 1) / R;
+    cudaError_t e;
+    if (q_dtype == LI_BF16) {
+      auto k = absorb_shared_kernel<__nv_bfloat16>;
+      e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      k<<<grid, 256, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), M, d_k,
+                                 reinterpret_cast<const __nv_bfloat16*>(W), b, d_c, R, out_dtype, q_abs,
+                                 q_abs_scale, beta);
+    } else {
+      auto k = absorb_shared_kernel<float>;
+      e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      k<<<grid, 256, smem, st>>>(reinterpret_cast<const float*>(q), M, d_k, reinterpret_cast<const float*>(W), b,
+                                 d_c, R, out_dtype, q_abs, q_abs_scale, beta);
+    }
+    return cudaGetLastError();
+  }
   const dim3 grid((H + kAbsorbHeads - 1) / kAbsorbHeads, n_tok);
   if (q_dtype == LI_BF16)
     absorb_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), H, d_k,

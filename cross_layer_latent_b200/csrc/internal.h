@@ -60,6 +60,12 @@ constexpr int kTraceCtas = 8, kTraceTiles = 64, kTraceEvents = 8;
 enum KernelKind { kKScan = 0, kKGather, kKTopkHist, kKTopkFilter, kKTopkSelect, kKTopkEmit,
                   kKAppendGemv, kKAppendStore, kKAbsorb, kKMemset };
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device. The attribute is set once per (kernel, device) and
+// remembered, so later calls make no runtime call at all (and so are safe
+// while a stream is being captured into a graph).
+cudaError_t raise_smem_limit(const void* fn, int bytes);
+
 cudaError_t launch_scan_kernel(int kind, bool gather, const ScanArgs& a, int grid, cudaStream_t st);
 
 // ---- top-k
@@ -118,6 +124,13 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st);
 int gemv_splits(int d_model, int n_tok);
 cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_model, int dim,
                                int n_tok, int splits, float* out, cudaStream_t st);
+// Decode-sized appends (at most 8 tokens, rows fitting one block's shared
+// memory) run as one launch: split-K GEMV, then the last block reduces the
+// splits in order and stores the rows.
+bool append_fusable(int n_tok, int dim, int splits);
+cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
+                                int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
+                                int dtype, unsigned int* done, int* status, cudaStream_t st);
 cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits,
                                 int batch, int T_chunk, int t0, int T_total, bool bump, void* data,
                                 float* scale, int32_t* lengths, int capacity, int dim, int dtype,

@@ -671,11 +671,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
 template <int KIND, bool GATHER>
 cudaError_t launch_one(const ScanArgs& a, int grid, cudaStream_t st) {
   auto k = scan_kernel<KIND, GATHER>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, a.smem_bytes);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return e;
-  }
+  const cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(k), a.smem_bytes);
+  if (e != cudaSuccess) return e;
   k<<<grid, kScanThreads, a.smem_bytes, st>>>(a);
   return cudaGetLastError();
 }

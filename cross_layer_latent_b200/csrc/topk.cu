@@ -352,23 +352,26 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
 }  // namespace li
 
 // ============================================================================
-// Single-launch cluster selection.
+// Single-launch selection for rows of up to 131072 positions.
 //
-// One thread-block cluster (CS <= 8 CTAs of 512 threads) per row; CTA c owns
-// positions [c*E, (c+1)*E), E = 512 * PT, as register-resident keys (warp w
-// holds a contiguous run of 32*PT positions, lane l position j*32 + l).  Four
-// cluster barriers:
-//   1. first-digit (top 11 bits) histograms are complete; every CTA sums the
-//      cluster's histograms through distributed shared memory and finds the
-//      boundary bucket b1 of each budget;
-//   2. each CTA has compacted the keys of its elements in the boundary
-//      bucket(s) to its own region of the workspace; every CTA then resolves
-//      the two remaining digits (11 + 10 bits) over all of them, redundantly,
-//      giving the exact k-th key T and how many elements equal to T are taken;
-//   3. per-CTA counts of (key > T, key == T) are published; an element's
-//      output rank is #greater before it + min(#equal before it, taken);
-//   4. no CTA leaves while another may still read its counts.
-// Up to two budgets (k and k2 <= k) are selected from the same keys.
+// A row is taken by CS <= 8 CTAs of 512 threads (a thread-block cluster when
+// CS > 1).  Warp w of CTA c owns the contiguous run of 32 * PT positions
+// starting at (c * 16 + w) * 32 * PT; in slab j of the run, lane l holds the
+// four positions j * 128 + 4 l + {0..3} (one coalesced 16-byte load per lane
+// and slab) as order-preserving uint32 keys in registers for the whole
+// kernel.  The exact k-th key T is found digit by digit (11 + 11 + 10 bits):
+// each pass histograms, in its own shared-memory array, the keys matching the
+// digits found so far, and reduces it to group counts (32 bins a group); the
+// CTAs meet at one barrier; then one warp per CTA sums the group counts of
+// every CTA through distributed shared memory, finds the boundary group, sums
+// that group's 32 bins the same way and finds the boundary bin.  Arrays are
+// never reused, so a pass needs one barrier, and only ~100 counters per CTA
+// cross the cluster per pass.  Up to two budgets (k and k2 <= k) share the
+// passes.  The output rank of a selected element is #greater before it +
+// min(#equal before it, #equal taken), from warp scans within slabs, warp
+// totals within the CTA and per-CTA totals pushed into the shared memory of
+// the later CTAs before a last barrier; after it no CTA touches another's
+// shared memory, so none has to wait for the others to exit.
 // ============================================================================
 #include <cooperative_groups.h>
 
@@ -377,250 +380,316 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-struct SelState {
-  int keff;          // min(k, n)
-  unsigned b1;       // boundary bucket of the first digit
-  int above1;        // elements in higher first-digit buckets
-  unsigned T;        // exact key of the keff-th element
-  int n_gt;          // elements with key > T
-  int need_eq;       // elements equal to T that are taken (lowest positions first)
-};
-
-constexpr int kCandCap = 16384;   // boundary-bucket keys a CTA stages in shared memory
-
-// Find the boundary bucket of `need` counting from the top in a 2048-bin
-// histogram whose per-thread bins are held in loc[0..3] (bins hi-1..hi-4).
-__device__ __forceinline__ void find_from_loc(const unsigned (&loc)[4], int hi, int need, int* scratch,
-                                              int* out) {
-  const int sum = static_cast<int>(loc[0] + loc[1] + loc[2] + loc[3]);
-  if (threadIdx.x == 0) { out[0] = 0; out[1] = 0; }
-  const int before = block_excl_scan(sum, scratch, nullptr);
-  if (before < need && need <= before + sum) {
-    int cum = before;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (cum + static_cast<int>(loc[i]) >= need) { out[0] = hi - 1 - i; out[1] = cum; break; }
-      cum += static_cast<int>(loc[i]);
-    }
-  }
-  __syncthreads();
+template <bool CL>
+__device__ __forceinline__ void sync_row(cg::cluster_group& cluster) {
+  if (CL) cluster.sync();
+  else __syncthreads();
 }
 
-// Remaining two digits over `m` candidate keys (shared memory).
-__device__ __forceinline__ void resolve_low_digits(SelState& st, const unsigned* cand, int m, unsigned* hist,
-                                                   int* scratch, int* res) {
-  int need = st.keff - st.above1;
-  unsigned prefix2 = 0;
-#pragma unroll
-  for (int d = 0; d < 2; ++d) {
-    const int nb = d == 0 ? 2048 : 1024;
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < m; i += blockDim.x) {
-      const unsigned key = cand[i];
-      if (d == 0) atomicAdd(&hist[(key >> 10) & 2047u], 1u);
-      else if (((key >> 10) & 2047u) == prefix2) atomicAdd(&hist[key & 1023u], 1u);
-    }
-    __syncthreads();
-    find_bucket_desc(hist, nb, need, scratch, res);
-    const unsigned bin = static_cast<unsigned>(res[0]);
-    const int above = res[1];
-    __syncthreads();
-    need -= above;
-    st.n_gt += above;
-    if (d == 0) prefix2 = bin;
-    else st.T = (st.b1 << 21) | (prefix2 << 10) | bin;
-  }
-  st.need_eq = need;
+template <bool CL, typename T>
+__device__ __forceinline__ T* rank_ptr(cg::cluster_group& cluster, T* p, int rk) {
+  if (CL) return cluster.map_shared_rank(p, rk);
+  return p;
 }
 
-// Thread t of CTA c owns positions [c*E + t*PT, +PT), E = 512 * PT, as
-// register keys; NSEL budgets (k, and k2 <= k) are selected from them.
-template <int PT, int NSEL>
-__global__ void __launch_bounds__(kClusterThreads, 1) topk_cluster_kernel(const TopkArgs a, const TopkOut2 o2) {
-  extern __shared__ __align__(16) unsigned cand_smem[];   // kCandCap keys
-  __shared__ __align__(16) unsigned hist[kHistBins];
-  __shared__ int scratch[32];
-  __shared__ int res[2];
-  __shared__ int cnt_local[2];                  // candidates of this CTA per bucket
-  __shared__ int ctot[2 * NSEL];                // (gt, eq) per budget of this CTA
+// After this CTA's histogram hist[NG * 32] is complete (and the block has
+// synchronised): the group counts (sum of bins [32 g, 32 g + 32)) are written
+// into slot c of ga[CS][NG] in the shared memory of every CTA of the row.
+template <int NG, bool CL>
+__device__ __forceinline__ void push_group_counts(cg::cluster_group& cluster, int CS, int c, const unsigned* hist,
+                                                  unsigned* ga) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int g = warp; g < NG; g += kClusterThreads / 32) {
+    const unsigned v = __reduce_add_sync(0xffffffffu, hist[g * 32 + lane]);
+    if (lane < CS) rank_ptr<CL>(cluster, ga, lane)[c * NG + g] = v;
+  }
+}
+
+// Warp 0: find, for each of nn counts need[i] (1 <= need[i] <= total), the bin
+// (counting from the top) that holds the need[i]-th element of the row's
+// histogram summed over the CS CTAs, and how many elements lie in higher
+// bins: res[i] = {bin, above}.  The boundary group comes from the gathered
+// group counts ga[CS][NG] (local), its 32 bins from every CTA's histogram
+// (distributed shared memory).  The block synchronises afterwards.
+template <int NG, bool CL>
+__device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, unsigned* hist, const unsigned* ga,
+                                          int nn, const int* need, int (*res)[2]) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  // lane l owns groups (descending) NG-1-(NG/32)l ... : 2 groups when NG = 64, 1 when 32
+  constexpr int GPL = NG / 32;
+  unsigned gc[GPL];
+#pragma unroll
+  for (int e = 0; e < GPL; ++e) gc[e] = 0;
+  {
+    const int g_lo = NG - GPL * (lane + 1);          // lowest group of this lane
+    unsigned v[kClusterMaxSize][GPL];
+#pragma unroll
+    for (int rk = 0; rk < kClusterMaxSize; ++rk) {
+      if (rk < CS) {
+        const unsigned* src = ga + rk * NG + g_lo;
+        if (GPL == 2) {
+          const uint2 u = *reinterpret_cast<const uint2*>(src);
+          v[rk][0] = u.y;                              // higher group first
+          v[rk][GPL - 1] = u.x;
+        } else {
+          v[rk][0] = src[0];
+        }
+      }
+    }
+#pragma unroll
+    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+      if (rk < CS) {
+#pragma unroll
+        for (int e = 0; e < GPL; ++e) gc[e] += v[rk][e];
+      }
+  }
+  unsigned tot = 0;
+#pragma unroll
+  for (int e = 0; e < GPL; ++e) tot += gc[e];
+  unsigned incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  const unsigned excl = incl - tot;
+  for (int i = 0; i < nn; ++i) {
+    const unsigned nd = static_cast<unsigned>(need[i]);
+    // boundary group and elements above it
+    const unsigned hit = __ballot_sync(0xffffffffu, excl < nd && nd <= incl);
+    const int src_lane = __ffs(hit) - 1;
+    int grp_sel = 0;
+    unsigned above = 0;
+    if (lane == src_lane) {
+      unsigned cum = excl;
+      grp_sel = NG - 1 - GPL * lane;
+#pragma unroll
+      for (int e = 0; e < GPL; ++e) {
+        if (cum + gc[e] >= nd) { grp_sel = NG - 1 - GPL * lane - e; break; }
+        cum += gc[e];
+      }
+      above = cum;
+    }
+    grp_sel = __shfl_sync(0xffffffffu, grp_sel, src_lane);
+    above = __shfl_sync(0xffffffffu, above, src_lane);
+    // the group's 32 bins, descending: lane l takes bin 32 g + 31 - l
+    const int bin = grp_sel * 32 + 31 - lane;
+    unsigned bv[kClusterMaxSize];
+#pragma unroll
+    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+      if (rk < CS) bv[rk] = rank_ptr<CL>(cluster, hist, rk)[bin];
+    unsigned bc = 0;
+#pragma unroll
+    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+      if (rk < CS) bc += bv[rk];
+    unsigned bincl = bc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned u = __shfl_up_sync(0xffffffffu, bincl, o);
+      if (lane >= o) bincl += u;
+    }
+    const unsigned nd2 = nd - above;
+    const unsigned bexcl = bincl - bc;
+    if (bexcl < nd2 && nd2 <= bincl) {
+      res[i][0] = bin;
+      res[i][1] = static_cast<int>(above + bexcl);
+    }
+  }
+}
+
+template <int PT, int NSEL, bool CL>
+__global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const TopkArgs a, const TopkOut2 o2) {
+  constexpr int NW = kClusterThreads / 32;
+  constexpr int NSLAB = PT / 4;
+  __shared__ __align__(16) unsigned H1[2048];          // top 11 bits
+  __shared__ __align__(16) unsigned H2[NSEL][2048];    // next 11 bits, per distinct first-digit bin
+  __shared__ __align__(16) unsigned H3[NSEL][1024];    // last 10 bits, per distinct 22-bit prefix
+  __shared__ __align__(16) unsigned G1[kClusterMaxSize * 64];          // group counts of every CTA
+  __shared__ __align__(16) unsigned G2[NSEL][kClusterMaxSize * 64];
+  __shared__ __align__(16) unsigned G3[NSEL][kClusterMaxSize * 32];
+  __shared__ int res[NSEL][2];
+  __shared__ int wtot[NSEL][NW];                        // packed (gt, eq) per warp
+  __shared__ int cin[kClusterMaxSize][2 * NSEL];        // (gt, eq) totals pushed by earlier CTAs
   cg::cluster_group cluster = cg::this_cluster();
-  const int CS = static_cast<int>(cluster.num_blocks());
-  const int c = static_cast<int>(cluster.block_rank());
+  const int CS = CL ? static_cast<int>(cluster.num_blocks()) : 1;
+  const int c = CL ? static_cast<int>(cluster.block_rank()) : 0;
   const int r = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = row_len(a, r);
-  SelState sel[NSEL];
-  sel[0].keff = min(a.k, n);
-  if (NSEL == 2) sel[NSEL - 1].keff = min(o2.k2, n);
+  int keff[NSEL];
+  keff[0] = min(a.k, n);
+  if (NSEL == 2) keff[NSEL - 1] = min(o2.k2, n);
   if (c == 0) {
 #pragma unroll
     for (int si = 0; si < NSEL; ++si) {
       const int kk = si == 0 ? a.k : o2.k2;
       int32_t* oi = (si == 0 ? a.out_idx : o2.out_idx2) + static_cast<int64_t>(r) * kk;
       float* osv = si == 0 ? a.out_score : o2.out_score2;
-      for (int j = max(sel[si].keff, 0) + threadIdx.x; j < kk; j += blockDim.x) {
+      for (int j = max(keff[si], 0) + threadIdx.x; j < kk; j += blockDim.x) {
         oi[j] = -1;
         if (osv) osv[static_cast<int64_t>(r) * kk + j] = -INFINITY;
       }
     }
-    if (a.out_count && threadIdx.x == 0) a.out_count[r] = max(sel[0].keff, 0);
+    if (a.out_count && threadIdx.x == 0) a.out_count[r] = max(keff[0], 0);
   }
-  if (sel[0].keff <= 0) return;   // uniform over the cluster (depends on the row only)
+  if (keff[0] <= 0) return;   // the same for every CTA of the row
 
-  const int64_t E = static_cast<int64_t>(kClusterThreads) * PT;
-  const int64_t p0 = static_cast<int64_t>(c) * E + static_cast<int64_t>(threadIdx.x) * PT;
+  {
+    uint4* z = reinterpret_cast<uint4*>(H1);
+    for (int i = threadIdx.x; i < 512; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    z = reinterpret_cast<uint4*>(&H2[0][0]);
+    for (int i = threadIdx.x; i < NSEL * 512; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    z = reinterpret_cast<uint4*>(&H3[0][0]);
+    for (int i = threadIdx.x; i < NSEL * 256; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+  }
+
+  const int64_t run = (static_cast<int64_t>(c) * NW + warp) * 32 * PT;   // first position of this warp
   const float* row = a.scores + static_cast<int64_t>(r) * a.row_stride;
   unsigned key[PT];
   unsigned vmask = 0;
-  if ((a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0 && p0 + PT <= n) {
+  if ((a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0 && run + 32 * PT <= n) {
 #pragma unroll
-    for (int j = 0; j < PT; j += 4) {
-      const float4 f = *reinterpret_cast<const float4*>(row + p0 + j);
-      key[j] = radix_key(f.x);
-      key[j + 1] = radix_key(f.y);
-      key[j + 2] = radix_key(f.z);
-      key[j + 3] = radix_key(f.w);
+    for (int j = 0; j < NSLAB; ++j) {
+      const float4 f = *reinterpret_cast<const float4*>(row + run + j * 128 + 4 * lane);
+      key[4 * j] = radix_key(f.x);
+      key[4 * j + 1] = radix_key(f.y);
+      key[4 * j + 2] = radix_key(f.z);
+      key[4 * j + 3] = radix_key(f.w);
     }
     vmask = PT == 32 ? 0xffffffffu : ((1u << PT) - 1u);
   } else {
 #pragma unroll
-    for (int j = 0; j < PT; ++j) {
-      key[j] = 0;
-      if (p0 + j < n) {
-        key[j] = radix_key(row[p0 + j]);
-        vmask |= 1u << j;
+    for (int j = 0; j < NSLAB; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t pos = run + j * 128 + 4 * lane + e;
+        key[4 * j + e] = 0;
+        if (pos < n) {
+          key[4 * j + e] = radix_key(row[pos]);
+          vmask |= 1u << (4 * j + e);
+        }
       }
     }
   }
+  __syncthreads();   // histograms cleared
 
-  // ---- 1. first digit: histograms summed over the cluster
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
+  // ---- pass 1: top 11 bits
 #pragma unroll
   for (int j = 0; j < PT; ++j)
-    if ((vmask >> j) & 1u) atomicAdd(&hist[key[j] >> 21], 1u);
-  cluster.sync();
-  const int hi = kHistBins - static_cast<int>(threadIdx.x) * 4;
-  unsigned loc[4] = {0, 0, 0, 0};
-  {
-    uint4 parts[kClusterMaxSize];
-#pragma unroll
-    for (int rk = 0; rk < kClusterMaxSize; ++rk)
-      if (rk < CS) parts[rk] = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, rk) + hi - 4);
-#pragma unroll
-    for (int rk = 0; rk < kClusterMaxSize; ++rk)
-      if (rk < CS) { loc[3] += parts[rk].x; loc[2] += parts[rk].y; loc[1] += parts[rk].z; loc[0] += parts[rk].w; }
-  }
+    if ((vmask >> j) & 1u) atomicAdd(&H1[key[j] >> 21], 1u);
+  __syncthreads();
+  push_group_counts<64, CL>(cluster, CS, c, H1, G1);
+  sync_row<CL>(cluster);
+  find_bins<64, CL>(cluster, CS, H1, G1, NSEL, keff, res);
+  __syncthreads();
+  int need[NSEL], above[NSEL];
+  unsigned pre[NSEL];
 #pragma unroll
   for (int si = 0; si < NSEL; ++si) {
-    find_from_loc(loc, hi, sel[si].keff, scratch, res);
-    sel[si].b1 = static_cast<unsigned>(res[0]);
-    sel[si].above1 = res[1];
-    sel[si].n_gt = res[1];
-    __syncthreads();
+    pre[si] = static_cast<unsigned>(res[si][0]);
+    above[si] = res[si][1];
+    need[si] = keff[si] - res[si][1];
+  }
+  // budget 1 shares budget 0's arrays when their prefixes agree
+  bool share = NSEL == 2 && pre[NSEL - 1] == pre[0];
+
+  // ---- pass 2: bits 20..10 of the keys in the boundary bin(s)
+#pragma unroll
+  for (int j = 0; j < PT; ++j) {
+    if (!((vmask >> j) & 1u)) continue;
+    const unsigned d1 = key[j] >> 21, d2 = (key[j] >> 10) & 2047u;
+    if (d1 == pre[0]) atomicAdd(&H2[0][d2], 1u);
+    else if (NSEL == 2 && !share && d1 == pre[NSEL - 1]) atomicAdd(&H2[NSEL - 1][d2], 1u);
+  }
+  __syncthreads();
+  push_group_counts<64, CL>(cluster, CS, c, H2[0], G2[0]);
+  if (NSEL == 2 && !share) push_group_counts<64, CL>(cluster, CS, c, H2[NSEL - 1], G2[NSEL - 1]);
+  sync_row<CL>(cluster);
+  if (NSEL == 1 || share) {
+    find_bins<64, CL>(cluster, CS, H2[0], G2[0], NSEL, need, res);
+  } else {
+    find_bins<64, CL>(cluster, CS, H2[0], G2[0], 1, need, res);
+    find_bins<64, CL>(cluster, CS, H2[NSEL - 1], G2[NSEL - 1], 1, need + (NSEL - 1), res + (NSEL - 1));
+  }
+  __syncthreads();
+#pragma unroll
+  for (int si = 0; si < NSEL; ++si) {
+    pre[si] = (pre[si] << 11) | static_cast<unsigned>(res[si][0]);
+    above[si] += res[si][1];
+    need[si] -= res[si][1];
+  }
+  share = NSEL == 2 && pre[NSEL - 1] == pre[0];
+
+  // ---- pass 3: bits 9..0 of the keys matching the 22-bit prefix(es)
+#pragma unroll
+  for (int j = 0; j < PT; ++j) {
+    if (!((vmask >> j) & 1u)) continue;
+    const unsigned p22 = key[j] >> 10, d3 = key[j] & 1023u;
+    if (p22 == pre[0]) atomicAdd(&H3[0][d3], 1u);
+    else if (NSEL == 2 && !share && p22 == pre[NSEL - 1]) atomicAdd(&H3[NSEL - 1][d3], 1u);
+  }
+  __syncthreads();
+  push_group_counts<32, CL>(cluster, CS, c, H3[0], G3[0]);
+  if (NSEL == 2 && !share) push_group_counts<32, CL>(cluster, CS, c, H3[NSEL - 1], G3[NSEL - 1]);
+  sync_row<CL>(cluster);
+  if (NSEL == 1 || share) {
+    find_bins<32, CL>(cluster, CS, H3[0], G3[0], NSEL, need, res);
+  } else {
+    find_bins<32, CL>(cluster, CS, H3[0], G3[0], 1, need, res);
+    find_bins<32, CL>(cluster, CS, H3[NSEL - 1], G3[NSEL - 1], 1, need + (NSEL - 1), res + (NSEL - 1));
+  }
+  __syncthreads();
+  unsigned T[NSEL];
+  int need_eq[NSEL];
+#pragma unroll
+  for (int si = 0; si < NSEL; ++si) {
+    T[si] = (pre[si] << 10) | static_cast<unsigned>(res[si][0]);
+    above[si] += res[si][1];
+    need_eq[si] = keff[si] - above[si];
   }
 
-  // ---- 2. this CTA's boundary-bucket keys -> its workspace region
-  //         (bucket of budget 0, then budget 1's if it differs)
-  const bool two = NSEL == 2 && sel[NSEL - 1].b1 != sel[0].b1;
-  unsigned* rowcand = reinterpret_cast<unsigned*>(a.cand) + static_cast<int64_t>(r) * a.n;
-  {
-    int m0 = 0, m1 = 0;
-#pragma unroll
-    for (int j = 0; j < PT; ++j) {
-      const bool v = (vmask >> j) & 1u;
-      const unsigned d = key[j] >> 21;
-      m0 += (v && d == sel[0].b1) ? 1 : 0;
-      m1 += (v && two && d == sel[NSEL - 1].b1) ? 1 : 0;
-    }
-    int tot = 0;
-    const int off = block_excl_scan(m0 | (m1 << 16), scratch, &tot);   // both counts < 2^15
-    int o0 = off & 0xFFFF, o1 = (off >> 16) + (tot & 0xFFFF);
-    unsigned* region = rowcand + static_cast<int64_t>(c) * E;
-#pragma unroll
-    for (int j = 0; j < PT; ++j) {
-      const bool v = (vmask >> j) & 1u;
-      const unsigned d = key[j] >> 21;
-      if (v && d == sel[0].b1) region[o0++] = key[j];
-      else if (v && two && d == sel[NSEL - 1].b1) region[o1++] = key[j];
-    }
-    if (threadIdx.x == 0) { cnt_local[0] = tot & 0xFFFF; cnt_local[1] = tot >> 16; }
-  }
-  cluster.sync();
-  // stage every CTA's keys of one bucket in shared memory, resolve the two
-  // remaining digits there (each CTA redundantly: no broadcast needed)
+  // ---- ordered output: warp totals, CTA totals, then per-slab warp scans
+  int base_gt[NSEL], base_eq[NSEL];
 #pragma unroll
   for (int si = 0; si < NSEL; ++si) {
-    const int bk = (si == 1 && two) ? 1 : 0;
-    int m = 0;
-    for (int rk = 0; rk < CS; ++rk) {
-      const int* rc = cluster.map_shared_rank(cnt_local, rk);
-      const int cnt = rc[bk];
-      const unsigned* src = rowcand + static_cast<int64_t>(rk) * E + (bk ? rc[0] : 0);
-      for (int i = threadIdx.x; i < cnt; i += blockDim.x)
-        if (m + i < kCandCap) cand_smem[m + i] = src[i];
-      m += cnt;
+    int x = 0;
+#pragma unroll
+    for (int j = 0; j < PT; ++j) {
+      const bool v = (vmask >> j) & 1u;
+      x += (v && key[j] > T[si]) ? 1 : 0;
+      x += (v && key[j] == T[si]) ? 0x10000 : 0;
     }
-    __syncthreads();
-    if (m <= kCandCap) {
-      resolve_low_digits(sel[si], cand_smem, m, hist, scratch, res);
-    } else {
-      // more boundary keys than shared memory holds (heavy ties): resolve from
-      // the workspace copies, one CTA region after the other
-      int need = sel[si].keff - sel[si].above1;
-      unsigned prefix2 = 0;
-#pragma unroll 1
-      for (int d = 0; d < 2; ++d) {
-        const int nb = d == 0 ? 2048 : 1024;
-        for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        for (int rk = 0; rk < CS; ++rk) {
-          const int* rc = cluster.map_shared_rank(cnt_local, rk);
-          const int cnt = rc[bk];
-          const unsigned* src = rowcand + static_cast<int64_t>(rk) * E + (bk ? rc[0] : 0);
-          for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-            const unsigned kq = src[i];
-            if (d == 0) atomicAdd(&hist[(kq >> 10) & 2047u], 1u);
-            else if (((kq >> 10) & 2047u) == prefix2) atomicAdd(&hist[kq & 1023u], 1u);
-          }
-        }
-        __syncthreads();
-        find_bucket_desc(hist, nb, need, scratch, res);
-        const unsigned bin = static_cast<unsigned>(res[0]);
-        const int above = res[1];
-        __syncthreads();
-        need -= above;
-        sel[si].n_gt += above;
-        if (d == 0) prefix2 = bin;
-        else sel[si].T = (sel[si].b1 << 21) | (prefix2 << 10) | bin;
+    x = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(x)));   // <= 32 * PT each field
+    if (lane == 0) wtot[si][warp] = x;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int si = 0; si < NSEL; ++si) {
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const int v = wtot[si][w];
+      before += w < warp ? v : 0;
+      total += v;
+    }
+    base_gt[si] = before & 0xFFFF;
+    base_eq[si] = before >> 16;
+    if (CL && threadIdx.x < CS && static_cast<int>(threadIdx.x) > c) {
+      int* dst = cluster.map_shared_rank(&cin[0][0], static_cast<int>(threadIdx.x));
+      dst[c * 2 * NSEL + 2 * si] = total & 0xFFFF;      // per-CTA totals <= 16384
+      dst[c * 2 * NSEL + 2 * si + 1] = total >> 16;
+    }
+  }
+  if (CL) {
+    cluster.sync();
+    for (int rk = 0; rk < c; ++rk) {
+#pragma unroll
+      for (int si = 0; si < NSEL; ++si) {
+        base_gt[si] += cin[rk][2 * si];
+        base_eq[si] += cin[rk][2 * si + 1];
       }
-      sel[si].need_eq = need;
     }
-    __syncthreads();
-  }
-
-  // ---- 3. ordered output: rank = #greater before + min(#equal before, need_eq)
-  int off_gt[NSEL], off_eq[NSEL];
-#pragma unroll
-  for (int si = 0; si < NSEL; ++si) {
-    int g = 0, e = 0;
-#pragma unroll
-    for (int j = 0; j < PT; ++j) {
-      const bool v = (vmask >> j) & 1u;
-      g += (v && key[j] > sel[si].T) ? 1 : 0;
-      e += (v && key[j] == sel[si].T) ? 1 : 0;
-    }
-    int tot = 0;
-    const int off = block_excl_scan(g | (e << 16), scratch, &tot);
-    off_gt[si] = off & 0xFFFF;
-    off_eq[si] = off >> 16;
-    if (threadIdx.x == 0) { ctot[2 * si] = tot & 0xFFFF; ctot[2 * si + 1] = tot >> 16; }
-  }
-  cluster.sync();
-  for (int rk = 0; rk < c; ++rk) {
-    const int* rt = cluster.map_shared_rank(ctot, rk);
-#pragma unroll
-    for (int si = 0; si < NSEL; ++si) { off_gt[si] += rt[2 * si]; off_eq[si] += rt[2 * si + 1]; }
   }
   const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
 #pragma unroll
@@ -629,42 +698,58 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_cluster_kernel(const 
     int32_t* oi = (si == 0 ? a.out_idx : o2.out_idx2) + static_cast<int64_t>(r) * kk;
     float* osv = si == 0 ? a.out_score : o2.out_score2;
     if (osv) osv += static_cast<int64_t>(r) * kk;
-    int gb = off_gt[si], eb = off_eq[si];
-    const unsigned T = sel[si].T;
-    const int need_eq = sel[si].need_eq;
+    int gb = base_gt[si], eb = base_eq[si];           // counts before this slab in this warp's run
+    const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-    for (int j = 0; j < PT; ++j) {
-      const bool v = (vmask >> j) & 1u;
-      const bool gt = v && key[j] > T;
-      const bool eq = v && key[j] == T;
-      if (gt || (eq && eb < need_eq)) {
-        const int rank = gb + min(eb, need_eq);
-        if (rank < kk) {
-          const int64_t pos = p0 + j;
-          oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
-          if (osv) osv[rank] = row[pos];
-        }
+    for (int j = 0; j < NSLAB; ++j) {
+      unsigned bg[4], be[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool v = (vmask >> (4 * j + e)) & 1u;
+        bg[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] > T[si]);
+        be[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] == T[si]);
       }
-      gb += gt ? 1 : 0;
-      eb += eq ? 1 : 0;
+      // elements of lower lanes in this slab come first
+      int g = gb, q = eb;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        g += __popc(bg[e] & lt);
+        q += __popc(be[e] & lt);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool gt = (bg[e] >> lane) & 1u;
+        const bool eq = (be[e] >> lane) & 1u;
+        if (gt || (eq && q < need_eq[si])) {
+          const int rank = g + min(q, need_eq[si]);
+          if (rank < kk) {
+            const int64_t pos = run + j * 128 + 4 * lane + e;
+            oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
+            if (osv) osv[rank] = row[pos];
+          }
+        }
+        g += gt ? 1 : 0;
+        q += eq ? 1 : 0;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        gb += __popc(bg[e]);
+        eb += __popc(be[e]);
+      }
     }
   }
-  cluster.sync();   // the counts of this CTA may be read until everyone is past here
 }
 
 template <int PT, int NSEL>
-cudaError_t launch_cluster_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
-  auto k = topk_cluster_kernel<PT, NSEL>;
-  const int dyn = kCandCap * 4;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return e;
+cudaError_t launch_radix_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
+  if (cs == 1) {
+    topk_radix_kernel<PT, NSEL, false><<<dim3(1, a.rows, 1), kClusterThreads, 0, st>>>(a, o2);
+    return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, a.rows, 1);
   cfg.blockDim = dim3(kClusterThreads, 1, 1);
-  cfg.dynamicSmemBytes = dyn;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -673,12 +758,12 @@ cudaError_t launch_cluster_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cud
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, a, o2);
+  return cudaLaunchKernelEx(&cfg, topk_radix_kernel<PT, NSEL, true>, a, o2);
 }
 
 template <int PT>
 cudaError_t launch_cluster_sel(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
-  return o2.k2 > 0 ? launch_cluster_pt<PT, 2>(a, o2, cs, st) : launch_cluster_pt<PT, 1>(a, o2, cs, st);
+  return o2.k2 > 0 ? launch_radix_pt<PT, 2>(a, o2, cs, st) : launch_radix_pt<PT, 1>(a, o2, cs, st);
 }
 
 }  // namespace

@@ -259,9 +259,10 @@ LI_API li_status li_topk(li_ctx* ctx, const float* scores, int rows, int n, int6
  * li_profile_read synchronises the recorded events and copies up to `max`
  * records into the host array `out` (in launch order), returning the number
  * of records in *count; li_profile_reset clears them.  Profiling adds two
- * event records per launch and is off by default. */
+ * event records per launch and is off by default; leave it off while a
+ * stream is being captured into a CUDA graph. */
 typedef struct {
-  char kernel[48];       /* "scan", "gather", "topk_filter", "append_gemv", ...  */
+  char kernel[48];       /* "scan", "gather", "topk_cluster", "append", ...    */
   float ms;              /* event-timed duration of the launch                   */
   int32_t grid;          /* CTAs launched (0 when not tracked)                   */
   int32_t block;         /* threads per CTA                                      */

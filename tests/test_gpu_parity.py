@@ -63,9 +63,12 @@ def test_append_matches_codec_bit_exactly(ctx, dtype):
     assert not data[2].any()          # nothing written for the overflowing sequence
 
 
-def test_append_with_projection(ctx):
-    rng = np.random.default_rng(6)
-    b, cap, T, dm, d = 2, 64, 5, 7168, 192
+@pytest.mark.parametrize("b,T", [(2, 5), (4, 1), (8, 1), (1, 3)])
+def test_append_with_projection(ctx, b, T):
+    """Multi-token appends (GEMV, then a store launch) and decode-sized ones
+    (one launch: the last block reduces the splits and stores)."""
+    rng = np.random.default_rng(6 + 10 * b + T)
+    cap, dm, d = 64, 7168, 192
     h = (rng.standard_normal((b, T, dm)) / np.sqrt(dm)).astype(np.float32)
     W = (rng.standard_normal((d, dm)) / np.sqrt(dm)).astype(np.float32)
     g32 = li.GroupIndexer(ctx, batch=b, capacity=cap, d_c=d, H=16, d_k=32, dtype=li.LI_F32, k=8)
@@ -83,7 +86,7 @@ def test_append_with_projection(ctx):
     codes, scale = codecs.e4m3_quantize_rows(c_gpu)
     assert np.array_equal(_np(g8.latent.data)[:, :T], codes)
     assert np.array_equal(_np(g8.latent.scale)[:, :T], scale)
-    assert _np(g32.latent.lengths).tolist() == [T, T]
+    assert _np(g32.latent.lengths).tolist() == [T] * b
 
 
 # ------------------------------------------------------------------ a2: absorption
@@ -112,6 +115,12 @@ def test_absorb_matches_oracle_and_codecs(ctx):
     assert np.array_equal(_np(out16), codecs.bf16_encode(g32))
     codes, scale = codecs.e4m3_quantize_rows(g32)
     assert np.array_equal(_np(out8), codes) and np.array_equal(_np(sc8), scale)
+    # the per-head kernel, given the shared decoder once per head, gives identical bits
+    Wt = np.ascontiguousarray(np.broadcast_to(W, (H, dk, dc)))
+    outt = torch.empty(n, H, dc, device=DEV)
+    li.li_absorb_query(ctx, qd, torch.from_numpy(Wt).to(DEV), dc, li.LI_F32, outt, W_K_head_stride=dk * dc)
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(outt), g32)
     # per-head decoders through the head stride
     Wh = (rng.standard_normal((H, dk, dc)) / np.sqrt(dk)).astype(np.float32)
     outh = torch.empty(n, H, dc, device=DEV)
@@ -120,6 +129,22 @@ def test_absorb_matches_oracle_and_codecs(ctx):
     refh, _ = indexer.absorb(q, Wh)
     boundh = np.einsum("nhk,hkc->nhc", np.abs(q), np.abs(Wh).astype(np.float64))
     assert np.all(np.abs(_np(outh) - refh) <= 1e-5 * boundh + 1e-30)
+
+
+@pytest.mark.parametrize("n,H,dk,dc", [(4, 64, 128, 192), (1, 8, 32, 48), (40, 32, 128, 256)])
+def test_absorb_bf16_inputs(ctx, n, H, dk, dc):
+    """bf16 queries and decoder (the decode path's inputs) against the oracle
+    on the decoded bf16 values, for decode, tiny and prefill-like shapes."""
+    rng = np.random.default_rng(8 + n)
+    q = torch.from_numpy((rng.standard_normal((n, H, dk)) / np.sqrt(dk)).astype(np.float32)).to(torch.bfloat16)
+    W = torch.from_numpy((rng.standard_normal((dk, dc)) / np.sqrt(dk)).astype(np.float32)).to(torch.bfloat16)
+    out = torch.empty(n, H, dc, device=DEV)
+    li.li_absorb_query(ctx, q.to(DEV), W.to(DEV), dc, li.LI_F32, out)
+    torch.cuda.synchronize()
+    qf, Wf = q.float().numpy(), W.float().numpy()
+    ref, _ = indexer.absorb(qf, Wf)
+    bound = np.einsum("nhk,kc->nhc", np.abs(qf), np.abs(Wf).astype(np.float64))
+    assert np.all(np.abs(_np(out) - ref) <= 1e-5 * bound + 1e-30)
 
 
 # ------------------------------------------------------------------ a3 + a4, a5 + a6, a7 on workloads
