@@ -267,7 +267,8 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   // in-flight item fit tensor memory), stage of KS K-chunks: the largest
   // stage that still leaves a pipeline of several stages.
   const bool has_meta = gather || c->dtype == LI_E4M3;
-  const size_t fixed_misc = 1024 + 16 + (kMaxSegments + 1) * 4 + 16 + kEpiWarps * (3 * N + 16) * 4;
+  const size_t fixed_misc = 1024 + 16 + (kMaxSegments + 1) * 4 + 16 + kEpiWarps * (3 * N + 16) * 4 +
+                            (gather ? 2 * kMaxSegments * 4 : 0);
   const size_t budget = static_cast<size_t>(ctx->max_smem_optin) - 1024;
   const size_t kStageCap = 48 * 1024;
   bool planned = false;
@@ -392,10 +393,10 @@ li_status run_topk_chunked(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L
   return LI_OK;
 }
 
-// One selection (and optionally a second budget k2 <= k over the same rows):
-// the single-launch cluster kernel when the rows fit it, else the chunked
-// multi-kernel path (which needs its histogram and row state cleared).
-li_status run_topk(li_ctx* ctx, TopkArgs& t, const TopkOut2& o2, void* ws, const WsLayout& L, cudaStream_t st) {
+// One selection: the single-launch cluster kernel when the rows fit it, else
+// the chunked multi-kernel path (which needs its histogram and row state
+// cleared).
+li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaStream_t st) {
   // workspace regions used by either path (the cluster kernel compacts its
   // boundary-bucket keys into `cand`)
   t.hist = at<unsigned int>(ws, L.hist);
@@ -408,7 +409,7 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, const TopkOut2& o2, void* ws, const
   if (t.n <= kClusterMaxN && t.rows <= 65535) {
     int cs = 0;
     Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);
-    const cudaError_t e = launch_topk_cluster(t, o2, st, &cs);
+    const cudaError_t e = launch_topk_cluster(t, st, &cs);
     Lc.grid = cs * t.rows;
     Lc.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster");
@@ -417,17 +418,7 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, const TopkOut2& o2, void* ws, const
   li_status s = clear_select_state(ctx, ws, L, t.rows, st);
   if (s != LI_OK) return s;
   t.hist_ready = false;
-  if ((s = run_topk_chunked(ctx, t, ws, L, st)) != LI_OK) return s;
-  if (o2.k2 > 0) {
-    TopkArgs t2 = t;
-    t2.k = o2.k2;
-    t2.out_idx = o2.out_idx2;
-    t2.out_score = o2.out_score2;
-    t2.out_count = nullptr;
-    if ((s = clear_select_state(ctx, ws, L, t.rows, st)) != LI_OK) return s;
-    return run_topk_chunked(ctx, t2, ws, L, st);
-  }
-  return LI_OK;
+  return run_topk_chunked(ctx, t, ws, L, st);
 }
 
 TopkArgs topk_args(const float* scores, int64_t stride, int rows, int n, int k) {
@@ -468,7 +459,7 @@ li_status score_topk_impl(li_ctx* ctx, const li_cache* c, const li_query* q, int
   t.q_pos = q->q_pos;
   t.out_idx = out_idx;
   t.out_score = out_score;
-  return run_topk(ctx, t, TopkOut2{0, nullptr, nullptr}, ws, L, st);
+  return run_topk(ctx, t, ws, L, st);
 }
 
 }  // namespace
@@ -704,15 +695,27 @@ li_status li_hs_anchor_candidates(li_ctx* c, const li_cache* cache, const li_que
   P.a.score_stride = cache->capacity;
   P.a.status = at<int>(ws, L.status);
   if ((s = run_scan(c, P, false, st)) != LI_OK) return s;
-  // candidates = top-B of the full prefix, and in the same selection launch
-  // the anchor's own top-k (the top-k under the same order is a subset)
+  // candidates = top-B of the full prefix, with their scores
+  float* cand_scores = at<float>(ws, L.cand_scores);
   TopkArgs t = topk_args(scores, cache->capacity, static_cast<int>(rows), cache->capacity, B);
   t.lengths = cache->lengths;
   t.len_div = q->T;
   t.q_pos = q->q_pos;
   t.out_idx = cand;
+  t.out_score = cand_scores;
   t.out_count = cand_n;
-  return run_topk(c, t, TopkOut2{k, anchor_idx, anchor_score}, ws, L, st);
+  if ((s = run_topk(c, t, ws, L, st)) != LI_OK) return s;
+  // the anchor's own top-k: under the same order (score desc, position asc)
+  // the top-k of the prefix is the top-k of its top-B, whose positions are
+  // ascending, so it is selected from the candidates' scores alone
+  TopkArgs t2 = topk_args(cand_scores, B, static_cast<int>(rows), B, k);
+  t2.lengths = cand_n;
+  t2.len_div = 1;
+  t2.idx_map = cand;
+  t2.map_stride = B;
+  t2.out_idx = anchor_idx;
+  t2.out_score = anchor_score;
+  return run_topk(c, t2, ws, L, st);
 }
 
 li_status li_hs_follower_refine(li_ctx* c, const li_cache* cache, const li_query* q, const int32_t* cand,
@@ -745,7 +748,7 @@ li_status li_hs_follower_refine(li_ctx* c, const li_cache* cache, const li_query
   t.map_stride = B;
   t.out_idx = out_idx;
   t.out_score = out_score;
-  return run_topk(c, t, TopkOut2{0, nullptr, nullptr}, ws, L, st);
+  return run_topk(c, t, ws, L, st);
 }
 
 li_status li_topk(li_ctx* c, const float* scores, int rows, int n, int64_t row_stride, const int32_t* lengths,
@@ -763,7 +766,7 @@ li_status li_topk(li_ctx* c, const float* scores, int rows, int n, int64_t row_s
   t.lengths = lengths;
   t.out_idx = out_idx;
   t.out_score = out_score;
-  return run_topk(c, t, TopkOut2{0, nullptr, nullptr}, ws, L, st);
+  return run_topk(c, t, ws, L, st);
 }
 
 li_status li_set_trace(li_ctx* c, void* buf, size_t bytes) {

@@ -96,17 +96,11 @@ struct TopkArgs {
 
 // Single-launch selection for rows of up to kClusterMaxN positions: one
 // thread-block cluster per row, keys held in registers, digit histograms
-// summed across the cluster in distributed shared memory.  A second budget
-// k2 <= k (out_idx2 / out_score2) can be selected in the same launch.
+// summed across the cluster in distributed shared memory.
 constexpr int kClusterThreads = 512;
 constexpr int kClusterMaxSize = 8;
 constexpr int kClusterMaxN = kClusterThreads * 32 * kClusterMaxSize;   // 131072
-struct TopkOut2 {
-  int k2;                     // 0: no second selection
-  int32_t* out_idx2;
-  float* out_score2;
-};
-cudaError_t launch_topk_cluster(const TopkArgs& a, const TopkOut2& o2, cudaStream_t st, int* cluster_size);
+cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size);
 
 constexpr int kTopkChunk = 4096;
 constexpr int kTopkThreads = 256;

@@ -54,6 +54,8 @@ struct ScanSmem {
   int* abort_flag;
   int* prefix;          // [kMaxSegments + 1]
   float* ep;            // kEpiWarps x (3 * N + 16) floats
+  int* seg_n;           // gather: [kMaxSegments] candidates of each segment (clamped)
+  int* seg_len;         // gather: [kMaxSegments] valid length of the segment's sequence
 };
 
 __device__ __forceinline__ ScanSmem carve(uint8_t* base, const ScanArgs& a) {
@@ -76,6 +78,8 @@ __device__ __forceinline__ ScanSmem carve(uint8_t* base, const ScanArgs& a) {
   s.prefix = s.abort_flag + 2;
   // 16-byte aligned parameter arrays (read four at a time)
   s.ep = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s.prefix + kMaxSegments + 1) + 15) & ~uintptr_t(15));
+  s.seg_n = reinterpret_cast<int*>(s.ep + kEpiWarps * (3 * a.N + 16));
+  s.seg_len = s.seg_n + kMaxSegments;
   return s;
 }
 
@@ -257,7 +261,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     tmem_relinquish();
   }
   // Items per segment, then an exclusive prefix over segments.
-  for (int i = tid; i < a.n_segments; i += blockDim.x) s.prefix[i + 1] = segment_items<GATHER>(a, i);
+  for (int i = tid; i < a.n_segments; i += blockDim.x) {
+    s.prefix[i + 1] = segment_items<GATHER>(a, i);
+    if (GATHER) {
+      int n = a.cand_n[i];
+      s.seg_n[i] = n < 0 ? 0 : (n > a.cand_stride ? a.cand_stride : n);
+      int len = a.lengths[i / a.T];
+      s.seg_len[i] = len < 0 ? 0 : (len > a.capacity ? a.capacity : len);
+    }
+  }
   __syncthreads();
   if (warp == 0) {
     int carry = 0;
@@ -374,20 +386,39 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ loader (gather), 32 lanes
-    // Each lane copies R/32 candidate rows with 16-byte cp.async into the
-    // [chunk][row] swizzled layout the 3-D TMA box would produce, plus the
-    // rows' token ids and fp8 scales into the item's metadata slot.  A stage
-    // (and the metadata with an item's first stage) is signalled once every
-    // lane's copies for it have landed; kDepth stages stay in flight.  All
-    // waits are warp-uniform.
-    constexpr int kDepth = 4;
+    // Per item: the lanes read the item's candidate ids (prefetched one item
+    // ahead, coalesced), validate them against the segment's limits cached
+    // in the prologue and publish token ids and fp8 scales in the item's
+    // metadata slot; then every copy instruction moves `rpi` whole chunk-rows
+    // (lanes take consecutive 16-byte pieces of the same row) with cp.async
+    // into the [chunk][row] swizzled layout a 3-D TMA box would produce.  A
+    // stage (and the metadata with an item's first stage) is signalled once
+    // every lane's copies for it have landed, at most kDepth stages behind
+    // the newest.  All waits are warp-uniform.
+    constexpr int kDepth = 8;
+    constexpr int kIdsPerLane = kMaxItemRows / 32;
     uint32_t pend[kDepth];     // stage | (meta slot + 1) << 16
     uint32_t issued = 0, retired = 0, n_bs = 0;
-    const int chunks16 = k_swz >> 4;
+    const int pieces = k_swz >> 4;                 // 16-byte pieces of a chunk-row
+    const int rpi = 32 / pieces;                   // chunk-rows per copy instruction
+    const int prow = lane / pieces, piece = lane - prow * pieces;
     const int rows_per_lane = k_R >> 5;
     Ring st, bs, ms;
     SegWalk w{s.prefix, n_groups};
+    SegWalk wn{s.prefix, n_groups};                // one item ahead
     bool first = true;
+    int ids[kIdsPerLane];
+    auto fetch_ids = [&](int item, SegWalk& ww, int (&out)[kIdsPerLane]) {
+      ww.to(item);
+      const int sg = ww.seg, itn = item - s.prefix[sg];
+#pragma unroll
+      for (int i = 0; i < kIdsPerLane; ++i) {
+        out[i] = -1;
+        const int j = itn * k_R + lane + 32 * i;
+        if (i < rows_per_lane && j < k_cand_stride) out[i] = k_cand[static_cast<int64_t>(sg) * k_cand_stride + j];
+      }
+    };
+    if (begin < end) fetch_ids(begin, wn, ids);
     for (int item = begin; item < end; ++item) {
       if (*s.abort_flag) break;
       const bool moved = w.to(item) || first;
@@ -405,47 +436,42 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         bs.step(NB);
         ++n_bs;
       }
-      int len = k_lengths[w.b];
-      len = len < 0 ? 0 : (len > k_capacity ? k_capacity : len);
-      int cn = k_cand_n[seg];
-      cn = cn < 0 ? 0 : (cn > k_cand_stride ? k_cand_stride : cn);
+      int cur[kIdsPerLane];
+#pragma unroll
+      for (int i = 0; i < kIdsPerLane; ++i) cur[i] = ids[i];
+      if (item + 1 < end) fetch_ids(item + 1, wn, ids);   // in flight while this item is copied
+      const int len = s.seg_len[seg], cn = s.seg_n[seg];
       if (!bounded_wait(&s.mempty[ms.i], ms.ph ^ 1u, wc)) break;
       float* mscale = reinterpret_cast<float*>(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes);
       int* mtok = reinterpret_cast<int*>(mscale + k_R);
       const int64_t seq_row = static_cast<int64_t>(w.b) * k_capacity;
-      int tok[kMaxItemRows / 32];
 #pragma unroll
-      for (int i = 0; i < kMaxItemRows / 32; ++i) {
-        tok[i] = -1;
+      for (int i = 0; i < kIdsPerLane; ++i) {
         if (i < rows_per_lane) {
           const int r = lane + 32 * i;
           const int j = it * k_R + r;
-          int t = j < cn ? k_cand[static_cast<int64_t>(seg) * k_cand_stride + j] : -1;
+          int t = j < cn ? cur[i] : -1;
           if (j < cn && (t < 0 || t >= len)) t = -2;     // invalid candidate
-          tok[i] = t;
           mtok[r] = t;
           if (e4) cp_async_4_zfill(smem_addr(mscale + r), k_cache_scale + seq_row + (t >= 0 ? t : 0), t >= 0 ? 4 : 0);
         }
       }
+      __syncwarp();
       const uint32_t mslot = ms.i;
       ms.step(kMetaSlots);
       bool ok = true;
       for (int sp = 0; sp < k_spi; ++sp) {
         if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
         const uint32_t dst = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
-#pragma unroll
-        for (int i = 0; i < kMaxItemRows / 32; ++i) {
-          if (i >= rows_per_lane) break;
-          const int r = lane + 32 * i;
-          const int t = tok[i] >= 0 ? tok[i] : 0;
-          const int nbytes = tok[i] >= 0 ? 16 : 0;
+        for (int r = prow; r < k_R; r += rpi) {
+          const int t = mtok[r];
+          const int nbytes = t >= 0 ? 16 : 0;
+          const uint8_t* src = k_cache + (seq_row + (t >= 0 ? t : 0)) * k_row_bytes + piece * 16;
+          const uint32_t off = swizzle(static_cast<uint32_t>(r * k_swz + piece * 16), k_swz);
           for (int c = 0; c < k_KS; ++c) {
             const int kc = sp * k_KS + c;
-            const uint8_t* src = k_cache + (seq_row + t) * k_row_bytes + static_cast<int64_t>(kc) * k_swz;
-            const uint32_t rowdst = dst + static_cast<uint32_t>(c) * chunk_region;
-            for (int q = 0; q < chunks16; ++q)
-              cp_async_16_zfill(rowdst + swizzle(static_cast<uint32_t>(r * k_swz + q * 16), k_swz), src + q * 16,
-                                nbytes);
+            cp_async_16_zfill(dst + static_cast<uint32_t>(c) * chunk_region + off, src + static_cast<int64_t>(kc) * k_swz,
+                              nbytes);
           }
         }
         cp_async_commit();
@@ -455,6 +481,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (issued - retired == kDepth) {
           cp_async_wait_group<kDepth - 1>();
           fence_proxy_async_smem();
+          __syncwarp();
           const uint32_t p = pend[retired & (kDepth - 1)];
           mbar_arrive(&s.full[p & 0xFFFFu]);
           if (p >> 16) mbar_arrive(&s.mfull[(p >> 16) - 1]);
@@ -465,6 +492,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
+    __syncwarp();
     if (!*s.abort_flag) {
       while (retired < issued) {
         const uint32_t p = pend[retired & (kDepth - 1)];

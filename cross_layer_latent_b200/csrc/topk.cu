@@ -366,8 +366,8 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
 // every CTA through distributed shared memory, finds the boundary group, sums
 // that group's 32 bins the same way and finds the boundary bin.  Arrays are
 // never reused, so a pass needs one barrier, and only ~100 counters per CTA
-// cross the cluster per pass.  Up to two budgets (k and k2 <= k) share the
-// passes.  The output rank of a selected element is #greater before it +
+// cross the cluster per pass.  The output rank of a selected element is
+// #greater before it +
 // min(#equal before it, #equal taken), from warp scans within slabs, warp
 // totals within the CTA and per-CTA totals pushed into the shared memory of
 // the later CTAs before a last barrier; after it no CTA touches another's
@@ -498,50 +498,44 @@ __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, un
   }
 }
 
-template <int PT, int NSEL, bool CL>
-__global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const TopkArgs a, const TopkOut2 o2) {
+template <int PT, bool CL>
+__global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const TopkArgs a) {
   constexpr int NW = kClusterThreads / 32;
   constexpr int NSLAB = PT / 4;
-  __shared__ __align__(16) unsigned H1[2048];          // top 11 bits
-  __shared__ __align__(16) unsigned H2[NSEL][2048];    // next 11 bits, per distinct first-digit bin
-  __shared__ __align__(16) unsigned H3[NSEL][1024];    // last 10 bits, per distinct 22-bit prefix
-  __shared__ __align__(16) unsigned G1[kClusterMaxSize * 64];          // group counts of every CTA
-  __shared__ __align__(16) unsigned G2[NSEL][kClusterMaxSize * 64];
-  __shared__ __align__(16) unsigned G3[NSEL][kClusterMaxSize * 32];
-  __shared__ int res[NSEL][2];
-  __shared__ int wtot[NSEL][NW];                        // packed (gt, eq) per warp
-  __shared__ int cin[kClusterMaxSize][2 * NSEL];        // (gt, eq) totals pushed by earlier CTAs
+  __shared__ __align__(16) unsigned H1[2048];                       // top 11 bits
+  __shared__ __align__(16) unsigned H2[2048];                       // next 11 bits (boundary bin)
+  __shared__ __align__(16) unsigned H3[1024];                       // last 10 bits (boundary prefix)
+  __shared__ __align__(16) unsigned G1[kClusterMaxSize * 64];       // group counts of every CTA
+  __shared__ __align__(16) unsigned G2[kClusterMaxSize * 64];
+  __shared__ __align__(16) unsigned G3[kClusterMaxSize * 32];
+  __shared__ int res[1][2];
+  __shared__ int wtot[NW];                                          // packed (gt, eq) per warp
+  __shared__ int cin[kClusterMaxSize][2];                           // (gt, eq) totals of earlier CTAs
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = CL ? static_cast<int>(cluster.num_blocks()) : 1;
   const int c = CL ? static_cast<int>(cluster.block_rank()) : 0;
   const int r = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = row_len(a, r);
-  int keff[NSEL];
-  keff[0] = min(a.k, n);
-  if (NSEL == 2) keff[NSEL - 1] = min(o2.k2, n);
+  const int keff = min(a.k, n);
+  int32_t* oi = a.out_idx + static_cast<int64_t>(r) * a.k;
+  float* osv = a.out_score ? a.out_score + static_cast<int64_t>(r) * a.k : nullptr;
   if (c == 0) {
-#pragma unroll
-    for (int si = 0; si < NSEL; ++si) {
-      const int kk = si == 0 ? a.k : o2.k2;
-      int32_t* oi = (si == 0 ? a.out_idx : o2.out_idx2) + static_cast<int64_t>(r) * kk;
-      float* osv = si == 0 ? a.out_score : o2.out_score2;
-      for (int j = max(keff[si], 0) + threadIdx.x; j < kk; j += blockDim.x) {
-        oi[j] = -1;
-        if (osv) osv[static_cast<int64_t>(r) * kk + j] = -INFINITY;
-      }
+    for (int j = max(keff, 0) + threadIdx.x; j < a.k; j += blockDim.x) {
+      oi[j] = -1;
+      if (osv) osv[j] = -INFINITY;
     }
-    if (a.out_count && threadIdx.x == 0) a.out_count[r] = max(keff[0], 0);
+    if (a.out_count && threadIdx.x == 0) a.out_count[r] = max(keff, 0);
   }
-  if (keff[0] <= 0) return;   // the same for every CTA of the row
+  if (keff <= 0) return;   // the same for every CTA of the row
 
   {
     uint4* z = reinterpret_cast<uint4*>(H1);
     for (int i = threadIdx.x; i < 512; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
-    z = reinterpret_cast<uint4*>(&H2[0][0]);
-    for (int i = threadIdx.x; i < NSEL * 512; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
-    z = reinterpret_cast<uint4*>(&H3[0][0]);
-    for (int i = threadIdx.x; i < NSEL * 256; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    z = reinterpret_cast<uint4*>(H2);
+    for (int i = threadIdx.x; i < 512; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    z = reinterpret_cast<uint4*>(H3);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
   }
 
   const int64_t run = (static_cast<int64_t>(c) * NW + warp) * 32 * PT;   // first position of this warp
@@ -581,169 +575,120 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   __syncthreads();
   push_group_counts<64, CL>(cluster, CS, c, H1, G1);
   sync_row<CL>(cluster);
-  find_bins<64, CL>(cluster, CS, H1, G1, NSEL, keff, res);
+  find_bins<64, CL>(cluster, CS, H1, G1, 1, &keff, res);
   __syncthreads();
-  int need[NSEL], above[NSEL];
-  unsigned pre[NSEL];
-#pragma unroll
-  for (int si = 0; si < NSEL; ++si) {
-    pre[si] = static_cast<unsigned>(res[si][0]);
-    above[si] = res[si][1];
-    need[si] = keff[si] - res[si][1];
-  }
-  // budget 1 shares budget 0's arrays when their prefixes agree
-  bool share = NSEL == 2 && pre[NSEL - 1] == pre[0];
+  unsigned pre = static_cast<unsigned>(res[0][0]);
+  int above = res[0][1];
+  int need = keff - above;
 
-  // ---- pass 2: bits 20..10 of the keys in the boundary bin(s)
+  // ---- pass 2: bits 20..10 of the keys in the boundary bin
 #pragma unroll
-  for (int j = 0; j < PT; ++j) {
-    if (!((vmask >> j) & 1u)) continue;
-    const unsigned d1 = key[j] >> 21, d2 = (key[j] >> 10) & 2047u;
-    if (d1 == pre[0]) atomicAdd(&H2[0][d2], 1u);
-    else if (NSEL == 2 && !share && d1 == pre[NSEL - 1]) atomicAdd(&H2[NSEL - 1][d2], 1u);
-  }
+  for (int j = 0; j < PT; ++j)
+    if (((vmask >> j) & 1u) && (key[j] >> 21) == pre) atomicAdd(&H2[(key[j] >> 10) & 2047u], 1u);
   __syncthreads();
-  push_group_counts<64, CL>(cluster, CS, c, H2[0], G2[0]);
-  if (NSEL == 2 && !share) push_group_counts<64, CL>(cluster, CS, c, H2[NSEL - 1], G2[NSEL - 1]);
+  push_group_counts<64, CL>(cluster, CS, c, H2, G2);
   sync_row<CL>(cluster);
-  if (NSEL == 1 || share) {
-    find_bins<64, CL>(cluster, CS, H2[0], G2[0], NSEL, need, res);
-  } else {
-    find_bins<64, CL>(cluster, CS, H2[0], G2[0], 1, need, res);
-    find_bins<64, CL>(cluster, CS, H2[NSEL - 1], G2[NSEL - 1], 1, need + (NSEL - 1), res + (NSEL - 1));
-  }
+  find_bins<64, CL>(cluster, CS, H2, G2, 1, &need, res);
   __syncthreads();
-#pragma unroll
-  for (int si = 0; si < NSEL; ++si) {
-    pre[si] = (pre[si] << 11) | static_cast<unsigned>(res[si][0]);
-    above[si] += res[si][1];
-    need[si] -= res[si][1];
-  }
-  share = NSEL == 2 && pre[NSEL - 1] == pre[0];
+  pre = (pre << 11) | static_cast<unsigned>(res[0][0]);
+  above += res[0][1];
+  need -= res[0][1];
 
-  // ---- pass 3: bits 9..0 of the keys matching the 22-bit prefix(es)
+  // ---- pass 3: bits 9..0 of the keys matching the 22-bit prefix
 #pragma unroll
-  for (int j = 0; j < PT; ++j) {
-    if (!((vmask >> j) & 1u)) continue;
-    const unsigned p22 = key[j] >> 10, d3 = key[j] & 1023u;
-    if (p22 == pre[0]) atomicAdd(&H3[0][d3], 1u);
-    else if (NSEL == 2 && !share && p22 == pre[NSEL - 1]) atomicAdd(&H3[NSEL - 1][d3], 1u);
-  }
+  for (int j = 0; j < PT; ++j)
+    if (((vmask >> j) & 1u) && (key[j] >> 10) == pre) atomicAdd(&H3[key[j] & 1023u], 1u);
   __syncthreads();
-  push_group_counts<32, CL>(cluster, CS, c, H3[0], G3[0]);
-  if (NSEL == 2 && !share) push_group_counts<32, CL>(cluster, CS, c, H3[NSEL - 1], G3[NSEL - 1]);
+  push_group_counts<32, CL>(cluster, CS, c, H3, G3);
   sync_row<CL>(cluster);
-  if (NSEL == 1 || share) {
-    find_bins<32, CL>(cluster, CS, H3[0], G3[0], NSEL, need, res);
-  } else {
-    find_bins<32, CL>(cluster, CS, H3[0], G3[0], 1, need, res);
-    find_bins<32, CL>(cluster, CS, H3[NSEL - 1], G3[NSEL - 1], 1, need + (NSEL - 1), res + (NSEL - 1));
-  }
+  find_bins<32, CL>(cluster, CS, H3, G3, 1, &need, res);
   __syncthreads();
-  unsigned T[NSEL];
-  int need_eq[NSEL];
-#pragma unroll
-  for (int si = 0; si < NSEL; ++si) {
-    T[si] = (pre[si] << 10) | static_cast<unsigned>(res[si][0]);
-    above[si] += res[si][1];
-    need_eq[si] = keff[si] - above[si];
-  }
+  const unsigned T = (pre << 10) | static_cast<unsigned>(res[0][0]);
+  above += res[0][1];
+  const int need_eq = keff - above;     // elements equal to T that are taken
 
-  // ---- ordered output: warp totals, CTA totals, then per-slab warp scans
-  int base_gt[NSEL], base_eq[NSEL];
-#pragma unroll
-  for (int si = 0; si < NSEL; ++si) {
+  // ---- ordered output: warp totals, CTA totals, then per-slab ballots
+  {
     int x = 0;
 #pragma unroll
     for (int j = 0; j < PT; ++j) {
       const bool v = (vmask >> j) & 1u;
-      x += (v && key[j] > T[si]) ? 1 : 0;
-      x += (v && key[j] == T[si]) ? 0x10000 : 0;
+      x += (v && key[j] > T) ? 1 : 0;
+      x += (v && key[j] == T) ? 0x10000 : 0;
     }
     x = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(x)));   // <= 32 * PT each field
-    if (lane == 0) wtot[si][warp] = x;
+    if (lane == 0) wtot[warp] = x;
   }
   __syncthreads();
-#pragma unroll
-  for (int si = 0; si < NSEL; ++si) {
+  int gb = 0, eb = 0;                   // elements before this warp's run
+  {
     int before = 0, total = 0;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const int v = wtot[si][w];
+      const int v = wtot[w];
       before += w < warp ? v : 0;
       total += v;
     }
-    base_gt[si] = before & 0xFFFF;
-    base_eq[si] = before >> 16;
+    gb = before & 0xFFFF;
+    eb = before >> 16;
     if (CL && threadIdx.x < CS && static_cast<int>(threadIdx.x) > c) {
       int* dst = cluster.map_shared_rank(&cin[0][0], static_cast<int>(threadIdx.x));
-      dst[c * 2 * NSEL + 2 * si] = total & 0xFFFF;      // per-CTA totals <= 16384
-      dst[c * 2 * NSEL + 2 * si + 1] = total >> 16;
+      dst[2 * c] = total & 0xFFFF;        // per-CTA totals <= 16384
+      dst[2 * c + 1] = total >> 16;
     }
   }
   if (CL) {
     cluster.sync();
     for (int rk = 0; rk < c; ++rk) {
-#pragma unroll
-      for (int si = 0; si < NSEL; ++si) {
-        base_gt[si] += cin[rk][2 * si];
-        base_eq[si] += cin[rk][2 * si + 1];
-      }
+      gb += cin[rk][0];
+      eb += cin[rk][1];
     }
   }
   const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
+  const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int si = 0; si < NSEL; ++si) {
-    const int kk = si == 0 ? a.k : o2.k2;
-    int32_t* oi = (si == 0 ? a.out_idx : o2.out_idx2) + static_cast<int64_t>(r) * kk;
-    float* osv = si == 0 ? a.out_score : o2.out_score2;
-    if (osv) osv += static_cast<int64_t>(r) * kk;
-    int gb = base_gt[si], eb = base_eq[si];           // counts before this slab in this warp's run
-    const unsigned lt = (1u << lane) - 1u;
+  for (int j = 0; j < NSLAB; ++j) {
+    unsigned bg[4], be[4];
 #pragma unroll
-    for (int j = 0; j < NSLAB; ++j) {
-      unsigned bg[4], be[4];
+    for (int e = 0; e < 4; ++e) {
+      const bool v = (vmask >> (4 * j + e)) & 1u;
+      bg[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] > T);
+      be[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] == T);
+    }
+    // elements of lower lanes in this slab come first
+    int g = gb, q = eb;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool v = (vmask >> (4 * j + e)) & 1u;
-        bg[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] > T[si]);
-        be[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] == T[si]);
-      }
-      // elements of lower lanes in this slab come first
-      int g = gb, q = eb;
+    for (int e = 0; e < 4; ++e) {
+      g += __popc(bg[e] & lt);
+      q += __popc(be[e] & lt);
+    }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        g += __popc(bg[e] & lt);
-        q += __popc(be[e] & lt);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool gt = (bg[e] >> lane) & 1u;
-        const bool eq = (be[e] >> lane) & 1u;
-        if (gt || (eq && q < need_eq[si])) {
-          const int rank = g + min(q, need_eq[si]);
-          if (rank < kk) {
-            const int64_t pos = run + j * 128 + 4 * lane + e;
-            oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
-            if (osv) osv[rank] = row[pos];
-          }
+    for (int e = 0; e < 4; ++e) {
+      const bool gt = (bg[e] >> lane) & 1u;
+      const bool eq = (be[e] >> lane) & 1u;
+      if (gt || (eq && q < need_eq)) {
+        const int rank = g + min(q, need_eq);
+        if (rank < a.k) {
+          const int64_t pos = run + j * 128 + 4 * lane + e;
+          oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
+          if (osv) osv[rank] = row[pos];
         }
-        g += gt ? 1 : 0;
-        q += eq ? 1 : 0;
       }
+      g += gt ? 1 : 0;
+      q += eq ? 1 : 0;
+    }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        gb += __popc(bg[e]);
-        eb += __popc(be[e]);
-      }
+    for (int e = 0; e < 4; ++e) {
+      gb += __popc(bg[e]);
+      eb += __popc(be[e]);
     }
   }
 }
 
-template <int PT, int NSEL>
-cudaError_t launch_radix_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
+template <int PT>
+cudaError_t launch_radix_pt(const TopkArgs& a, int cs, cudaStream_t st) {
   if (cs == 1) {
-    topk_radix_kernel<PT, NSEL, false><<<dim3(1, a.rows, 1), kClusterThreads, 0, st>>>(a, o2);
+    topk_radix_kernel<PT, false><<<dim3(1, a.rows, 1), kClusterThreads, 0, st>>>(a);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -758,26 +703,21 @@ cudaError_t launch_radix_pt(const TopkArgs& a, const TopkOut2& o2, int cs, cudaS
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_radix_kernel<PT, NSEL, true>, a, o2);
-}
-
-template <int PT>
-cudaError_t launch_cluster_sel(const TopkArgs& a, const TopkOut2& o2, int cs, cudaStream_t st) {
-  return o2.k2 > 0 ? launch_radix_pt<PT, 2>(a, o2, cs, st) : launch_radix_pt<PT, 1>(a, o2, cs, st);
+  return cudaLaunchKernelEx(&cfg, topk_radix_kernel<PT, true>, a);
 }
 
 }  // namespace
 
-cudaError_t launch_topk_cluster(const TopkArgs& a, const TopkOut2& o2, cudaStream_t st, int* cluster_size) {
+cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size) {
   const int64_t n = a.n;
   int cs = static_cast<int>((n + kClusterThreads * 16 - 1) / (kClusterThreads * 16));
   cs = cs < 1 ? 1 : (cs > kClusterMaxSize ? kClusterMaxSize : cs);
   const int64_t per_thread = (n + static_cast<int64_t>(cs) * kClusterThreads - 1) / (static_cast<int64_t>(cs) * kClusterThreads);
   if (cluster_size) *cluster_size = cs;
-  if (per_thread <= 4) return launch_cluster_sel<4>(a, o2, cs, st);
-  if (per_thread <= 8) return launch_cluster_sel<8>(a, o2, cs, st);
-  if (per_thread <= 16) return launch_cluster_sel<16>(a, o2, cs, st);
-  if (per_thread <= 32) return launch_cluster_sel<32>(a, o2, cs, st);
+  if (per_thread <= 4) return launch_radix_pt<4>(a, cs, st);
+  if (per_thread <= 8) return launch_radix_pt<8>(a, cs, st);
+  if (per_thread <= 16) return launch_radix_pt<16>(a, cs, st);
+  if (per_thread <= 32) return launch_radix_pt<32>(a, cs, st);
   return cudaErrorInvalidValue;
 }
 
