@@ -282,7 +282,7 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
         const int64_t room = static_cast<int64_t>(budget) - static_cast<int64_t>(bslots) * a.b_slot_bytes -
                              static_cast<int64_t>(meta + fixed_misc);
         const int stages = room > 0 ? static_cast<int>(std::min<int64_t>(kMaxStages, room / stage)) : 0;
-        const int need = gather ? 6 : (KS < a.n_kchunks ? 4 : 3);
+        const int need = KS < a.n_kchunks ? 4 : 3;
         if (stages < need) continue;
         a.R = R;
         a.MB = R / 128;
@@ -309,7 +309,14 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
 
   // Tensor maps: cache rows as {chunk elements, rows, chunks} so that one
   // box carries all KS chunks of R rows in [chunk][row] order, and queries.
-  {
+  if (gather) {
+    // rows gathered four at a time: a 2-D map whose box is one row high
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c->dim), static_cast<cuuint64_t>(c->batch) * c->capacity};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(swz / eb), 1};
+    li_status s = encode_map(ctx, &a.map_a, c->dtype, 2, c->data, dims, strides, box, swz);
+    if (s != LI_OK) return s;
+  } else {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(swz / eb), static_cast<cuuint64_t>(c->batch) * c->capacity,
                                 static_cast<cuuint64_t>(a.n_kchunks)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(swz)};

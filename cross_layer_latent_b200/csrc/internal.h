@@ -21,7 +21,8 @@ constexpr int kHistBins = 2048;      // first radix digit: key bits 31..21
 // Arguments of the scoring kernel (scan of whole prefixes, or gather of
 // candidate rows).  Tensor maps first: they must stay 64-byte aligned.
 struct alignas(64) ScanArgs {
-  CUtensorMap map_a;          // cache rows: dims {swz/elt, batch*capacity, n_kchunks}, box {swz/elt, R, KS}
+  CUtensorMap map_a;          // cache rows: dims {swz/elt, batch*capacity, n_kchunks}, box {swz/elt, R, KS};
+                              // gather: dims {dim, batch*capacity}, box {swz/elt, 1}
   CUtensorMap map_b;          // queries: dims {dim, H, batch*T}, box {swz/elt, H_pad, Qg}
   const uint8_t* cache;       // cache data (gather loads)
   const float* cache_scale;   // [batch*capacity] or null

@@ -245,11 +245,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const bool has_meta = GATHER || e4;
 
   if (tid == 0) {
-    for (int i = 0; i < a.n_stages; ++i) { mbar_init(&s.full[i], GATHER ? 32 : 1); mbar_init(&s.empty[i], 1); }
+    for (int i = 0; i < a.n_stages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
     for (int i = 0; i < a.n_bslots; ++i) { mbar_init(&s.bfull[i], 1); mbar_init(&s.bempty[i], 1); }
     for (int i = 0; i < a.n_acc; ++i) { mbar_init(&s.accfull[i], 1); mbar_init(&s.accempty[i], 4 * a.MB); }
     for (int i = 0; i < kMetaSlots; ++i) {
-      mbar_init(&s.mfull[i], GATHER ? 32 : 1);
+      // gather: every loader lane arrives once after storing its token ids
+      // and once (asynchronously) when its scale copies have landed
+      mbar_init(&s.mfull[i], GATHER ? 64 : 1);
       mbar_init(&s.mempty[i], 4 * a.MB);
     }
     mbar_init(s.drain, 1);
@@ -388,21 +390,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     // ------------------------------------------------------------ loader (gather), 32 lanes
     // Per item: the lanes read the item's candidate ids (prefetched one item
     // ahead, coalesced), validate them against the segment's limits cached
-    // in the prologue and publish token ids and fp8 scales in the item's
-    // metadata slot; then every copy instruction moves `rpi` whole chunk-rows
-    // (lanes take consecutive 16-byte pieces of the same row) with cp.async
-    // into the [chunk][row] swizzled layout a 3-D TMA box would produce.  A
-    // stage (and the metadata with an item's first stage) is signalled once
-    // every lane's copies for it have landed, at most kDepth stages behind
-    // the newest.  All waits are warp-uniform.
-    constexpr int kDepth = 8;
+    // in the prologue and publish token ids (and, with fp8, the rows' scales
+    // by 4-byte cp.async) in the item's metadata slot.  The rows themselves
+    // move by TMA row gathers, four rows of one K-chunk per instruction,
+    // spread over the 32 lanes, into the [chunk][row] swizzled layout the
+    // tiled load produces; a stage completes by its transaction count.
+    // Invalid or padding candidates gather row 0 of the sequence; the
+    // epilogue masks them.  All waits are warp-uniform.
     constexpr int kIdsPerLane = kMaxItemRows / 32;
-    uint32_t pend[kDepth];     // stage | (meta slot + 1) << 16
-    uint32_t issued = 0, retired = 0, n_bs = 0;
-    const int pieces = k_swz >> 4;                 // 16-byte pieces of a chunk-row
-    const int rpi = 32 / pieces;                   // chunk-rows per copy instruction
-    const int prow = lane / pieces, piece = lane - prow * pieces;
+    uint32_t n_st = 0, n_bs = 0;
     const int rows_per_lane = k_R >> 5;
+    const int groups = k_R >> 2;                   // 4-row gathers per K-chunk
     Ring st, bs, ms;
     SegWalk w{s.prefix, n_groups};
     SegWalk wn{s.prefix, n_groups};                // one item ahead
@@ -439,12 +437,12 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       int cur[kIdsPerLane];
 #pragma unroll
       for (int i = 0; i < kIdsPerLane; ++i) cur[i] = ids[i];
-      if (item + 1 < end) fetch_ids(item + 1, wn, ids);   // in flight while this item is copied
+      if (item + 1 < end) fetch_ids(item + 1, wn, ids);   // in flight while this item is issued
       const int len = s.seg_len[seg], cn = s.seg_n[seg];
       if (!bounded_wait(&s.mempty[ms.i], ms.ph ^ 1u, wc)) break;
       float* mscale = reinterpret_cast<float*>(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes);
       int* mtok = reinterpret_cast<int*>(mscale + k_R);
-      const int64_t seq_row = static_cast<int64_t>(w.b) * k_capacity;
+      const int seq_row = w.b * k_capacity;
 #pragma unroll
       for (int i = 0; i < kIdsPerLane; ++i) {
         if (i < rows_per_lane) {
@@ -456,53 +454,35 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           if (e4) cp_async_4_zfill(smem_addr(mscale + r), k_cache_scale + seq_row + (t >= 0 ? t : 0), t >= 0 ? 4 : 0);
         }
       }
+      cp_async_arrive_noinc(&s.mfull[ms.i]);
+      mbar_arrive(&s.mfull[ms.i]);
       __syncwarp();
-      const uint32_t mslot = ms.i;
       ms.step(kMetaSlots);
       bool ok = true;
       for (int sp = 0; sp < k_spi; ++sp) {
         if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
-        const uint32_t dst = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
-        for (int r = prow; r < k_R; r += rpi) {
-          const int t = mtok[r];
-          const int nbytes = t >= 0 ? 16 : 0;
-          const uint8_t* src = k_cache + (seq_row + (t >= 0 ? t : 0)) * k_row_bytes + piece * 16;
-          const uint32_t off = swizzle(static_cast<uint32_t>(r * k_swz + piece * 16), k_swz);
-          for (int c = 0; c < k_KS; ++c) {
-            const int kc = sp * k_KS + c;
-            cp_async_16_zfill(dst + static_cast<uint32_t>(c) * chunk_region + off, src + static_cast<int64_t>(kc) * k_swz,
-                              nbytes);
-          }
+        if (lane == 0) mbar_arrive_expect_tx(&s.full[st.i], k_a_stage_bytes);
+        __syncwarp();
+        const uint32_t stage = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
+        for (int u = lane; u < groups * k_KS; u += 32) {
+          const int c = u / groups, r0 = 4 * (u - c * groups);
+          const int t0 = mtok[r0], t1 = mtok[r0 + 1], t2 = mtok[r0 + 2], t3 = mtok[r0 + 3];
+          tma_gather4(stage + static_cast<uint32_t>(c) * chunk_region + static_cast<uint32_t>(r0 * k_swz), &a.map_a,
+                      &s.full[st.i], (sp * k_KS + c) * elt_per_chunk, seq_row + (t0 >= 0 ? t0 : 0),
+                      seq_row + (t1 >= 0 ? t1 : 0), seq_row + (t2 >= 0 ? t2 : 0), seq_row + (t3 >= 0 ? t3 : 0));
         }
-        cp_async_commit();
-        pend[issued & (kDepth - 1)] = st.i | (sp == 0 ? (mslot + 1u) << 16 : 0u);
-        ++issued;
         st.step(S);
-        if (issued - retired == kDepth) {
-          cp_async_wait_group<kDepth - 1>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          const uint32_t p = pend[retired & (kDepth - 1)];
-          mbar_arrive(&s.full[p & 0xFFFFu]);
-          if (p >> 16) mbar_arrive(&s.mfull[(p >> 16) - 1]);
-          ++retired;
-        }
+        ++n_st;
       }
       if (!ok) break;
     }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (!*s.abort_flag) {
-      while (retired < issued) {
-        const uint32_t p = pend[retired & (kDepth - 1)];
-        mbar_arrive(&s.full[p & 0xFFFFu]);
-        if (p >> 16) mbar_arrive(&s.mfull[(p >> 16) - 1]);
-        ++retired;
+    if (*s.abort_flag) {
+      // let every copy already issued land before the CTA exits
+      cp_async_wait_all();
+      if (lane == 0) {
+        drain_ring(s.full, S, n_st);
+        drain_ring(s.bfull, NB, n_bs);
       }
-    } else if (lane == 0) {
-      // B slots were loaded by TMA: let them land (the cp.async rows are done)
-      drain_ring(s.bfull, NB, n_bs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer, one lane
