@@ -70,6 +70,8 @@ _sigs = {
     "li_absorb_query": (_I, [_P, _P, _I, _I, _I, _I, _P, _I64, _P, _I64, _I, _I, _P, _P, _P, _P]),
     "li_score_topk": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _I, _P, _P, _P, _P,
                            _SZ, _P]),
+    "li_score_topk_static": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _I, _P, _P, _P,
+                                  _P]),
     "li_hs_anchor_candidates": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _I, _I, _P,
                                      _P, _P, _P, _P, _P, _SZ, _P]),
     "li_hs_follower_refine": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _P, _P, _I, _I,
@@ -229,6 +231,15 @@ def li_score_topk(ctx: Context, cache: Cache, query: Query, k: int, out_idx: tor
     cc, qq = cache.c(), query.c()
     ctx.check(_lib.li_score_topk(ctx.handle, ctypes.byref(cc), ctypes.byref(qq), int(k), _ptr(out_idx),
                                  _ptr(out_score), _ptr(scores_dump), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def li_score_topk_static(ctx: Context, cache: Cache, query: Query, k: int, out_idx: torch.Tensor,
+                         out_score: Optional[torch.Tensor] = None, device_status: Optional[torch.Tensor] = None,
+                         stream=None):
+    """li_score_topk with the library's fixed internal scratch instead of a workspace."""
+    cc, qq = cache.c(), query.c()
+    ctx.check(_lib.li_score_topk_static(ctx.handle, ctypes.byref(cc), ctypes.byref(qq), int(k), _ptr(out_idx),
+                                        _ptr(out_score), _ptr(device_status), _stream(stream)))
 
 
 def li_dsa_score_topk(ctx: Context, key_cache: Cache, query: Query, k: int, out_idx: torch.Tensor,

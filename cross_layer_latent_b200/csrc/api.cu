@@ -602,7 +602,7 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
   const int tchunk = std::max(1, std::min(T, kAppendChunkTok / cache->batch));
   {
     const int n_tok = cache->batch * T;
-    const int splits = gemv_splits(d_model, n_tok);
+    const int splits = append_fused_splits(d_model, dim);
     if (append_fusable(n_tok, dim, splits)) {
       Launch Lg(c, st, "append", 0, 256, 0);
       const cudaError_t e = launch_append_fused(h, h_dtype, W_down, d_model, dim, cache->batch, T, splits, tmp,
@@ -821,3 +821,99 @@ li_status li_profile_reset(li_ctx* c) {
 }
 
 }  // extern "C"
+
+// ======================================================================== allocation-free selection
+
+namespace {
+
+// Scratch of li_score_topk_static, part of the library image (no allocation
+// at any time): a 256-byte header holding the device status word, then the
+// fp32 scores of every query row.  The module loader zero-fills it; the
+// entry point clears the status word itself before every call.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;   // 8 MiB
+constexpr size_t kStaticScoresOffset = 256;
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kStaticMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per
+// device (the lookup is the only setup this entry point needs).
+li_status static_scratch(li_ctx* c, void** out, const char* what) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(c, e, what);
+  if (dev != c->device)
+    return fail(c, LI_ERR_ARG, "%s: the context's device (%d) must be the current device (%d)", what, c->device,
+                dev);
+  if (dev < 0 || dev >= kStaticMaxDevices)
+    return fail(c, LI_ERR_UNSUPPORTED, "%s: device ordinal %d above %d", what, dev, kStaticMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return cuda_fail(c, e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress (static scratch)");
+    }
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return LI_OK;
+}
+
+}  // namespace
+
+extern "C" li_status li_score_topk_static(li_ctx* c, const li_cache* cache, const li_query* q, int k,
+                                          int32_t* out_idx, float* out_score, int32_t* device_status,
+                                          void* stream) {
+  const char* what = "li_score_topk_static";
+  if (!c) return LI_ERR_ARG;
+  li_status s = check_cache(c, cache, what);
+  if (s != LI_OK) return s;
+  if ((s = check_query(c, cache, q, what)) != LI_OK) return s;
+  if (!out_idx) return fail(c, LI_ERR_ARG, "%s: out_idx is NULL", what);
+  if (k < 1 || k > cache->capacity) return fail(c, LI_ERR_ARG, "%s: k = %d must be in [1, capacity]", what, k);
+  const int64_t rows = static_cast<int64_t>(cache->batch) * q->T;
+  if (cache->capacity > kClusterMaxN || rows > 65535)
+    return fail(c, LI_ERR_UNSUPPORTED, "%s: rows of at most %d positions and at most 65535 query rows (got %d, %lld)",
+                what, kClusterMaxN, cache->capacity, static_cast<long long>(rows));
+  const size_t need = kStaticScoresOffset + static_cast<size_t>(rows) * cache->capacity * sizeof(float);
+  if (need > kStaticScratchBytes)
+    return fail(c, LI_ERR_WORKSPACE, "%s: %lld query rows x %d positions need %zu bytes of scratch; the static "
+                "scratch holds %zu (use li_score_topk with a caller-owned workspace)", what,
+                static_cast<long long>(rows), cache->capacity, need, kStaticScratchBytes);
+  void* base = nullptr;
+  if ((s = static_scratch(c, &base, what)) != LI_OK) return s;
+  int* status = static_cast<int*>(base);
+  float* scores = reinterpret_cast<float*>(static_cast<uint8_t*>(base) + kStaticScoresOffset);
+  ScanPlan P;
+  if ((s = plan_scan(c, cache, q, false, 0, &P, what)) != LI_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(c, e, "static scratch status clear");
+  P.a.scores = scores;
+  P.a.score_stride = cache->capacity;
+  P.a.status = status;
+  if ((s = run_scan(c, P, false, st)) != LI_OK) return s;
+  TopkArgs t = topk_args(scores, cache->capacity, static_cast<int>(rows), cache->capacity, k);
+  t.lengths = cache->lengths;
+  t.len_div = q->T;
+  t.q_pos = q->q_pos;
+  t.out_idx = out_idx;
+  t.out_score = out_score;
+  {
+    int cs = 0;
+    Launch Lc(c, st, "topk_cluster", 0, kClusterThreads, 0);
+    e = launch_topk_cluster(t, st, &cs);
+    Lc.grid = cs * t.rows;
+    Lc.done();
+    if (e != cudaSuccess) return cuda_fail(c, e, "topk_cluster");
+  }
+  if (device_status) {
+    e = cudaMemcpyAsync(device_status, status, sizeof(int), cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "static scratch status copy");
+  }
+  return LI_OK;
+}

@@ -243,6 +243,41 @@ LI_API li_status li_dsa_score_topk(li_ctx* ctx, const li_cache* key_cache, const
                             int32_t* out_idx, float* out_score, float* scores_dump, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* ------------------------------------------- scan and select without workspace */
+
+/* li_score_topk for callers that cannot hand the library any device memory
+ * of their own.  This entry point has no counterpart in the LatentIndex
+ * summary; it exists for the library's users.  Typical such callers: a
+ * plugin or foreign-function boundary that receives only a stream and its
+ * input and output buffers and has no allocator to draw a workspace from,
+ * and latency-critical code that must not call an allocator (an allocation
+ * can synchronise the device or fail under memory pressure at the worst
+ * moment).
+ *
+ * Computes exactly what li_score_topk computes (same kernels, same results)
+ * with out_idx [batch][T][k] and out_score [batch][T][k] (or NULL) as there,
+ * but its scratch -- the device status word and the fp32 scores of every
+ * query row -- is a fixed 8 MiB array inside the library image, not a
+ * workspace: nothing is allocated, ever.
+ * Limits: batch * T * capacity * 4 + 256 <= 8 MiB (e.g. 4 x 131072, 16 x
+ *   32768), capacity <= 131072 and batch * T <= 65535; larger requests are
+ *   refused with LI_ERR_WORKSPACE / LI_ERR_UNSUPPORTED before anything is
+ *   enqueued (use li_score_topk with a workspace).
+ * Setup: the first call on a device looks up the scratch's device address
+ *   (once per device, with the context's device current; a failure returns
+ *   LI_ERR_CUDA).  Make that first call before any stream capture begins.
+ * Zeroing: the scratch starts zeroed when the library is loaded; the status
+ *   word is cleared by every call itself; the scores need no clearing.
+ * Status: device-detected errors (a bounded wait that ran out) are written to
+ *   device_status ([1] int32, device pointer) at the end of the call when it
+ *   is not NULL; li_device_status does not see them.
+ * Concurrency: every call on a device shares the one scratch array, so two
+ *   calls whose work overlaps on the GPU (different streams, or different
+ *   host threads without ordering) race and corrupt each other's results.
+ *   Order them on one stream. */
+LI_API li_status li_score_topk_static(li_ctx* ctx, const li_cache* cache, const li_query* q, int k,
+                               int32_t* out_idx, float* out_score, int32_t* device_status, void* stream);
+
 /* ----------------------------------------------------- a4: plain selection */
 
 /* Top-k of `rows` fp32 rows: row r is scores[r * row_stride + 0 .. n_r),
