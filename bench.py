@@ -406,10 +406,17 @@ def profiled_steps(step, steps, flush, stream, lead_ms=4.0):
 
 
 def max_over_ranks(x, dist, dev):
+    """The slowest rank's value (every rank gets it)."""
     t = torch.tensor([x], device=dev, dtype=torch.float64)
     if dist:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(world, units_per_rank_step, steps, max_ms):
+    """Weak scaling: every rank processes the same number of units per step;
+    the job's rate is all ranks' units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
 
 
 def row_bytes(wl, dim):
@@ -469,7 +476,7 @@ def main():
     step.status("after the timed steps")
     max_ms = max_over_ranks(sum(hs_ms) + sum(dsa_ms), dist, dev)
     keys = step.hs_keys + step.dsa_keys
-    value = world * keys * args.steps / (max_ms / 1e3)
+    value = whole_job_rate(world, keys, args.steps, max_ms)
 
     # ---- second timed pass, eager, with a CUDA event pair around every launch:
     #      per-kernel durations for the roofline and the launch count
@@ -566,7 +573,7 @@ def main():
             e1.synchronize()
             e2e_ms.append(e0.elapsed_time(e1))
         te = max_over_ranks(sum(e2e_ms), dist, dev)
-        out["e2e"] = {"value": world * keys * args.steps / (te / 1e3), "unit": "keys/s",
+        out["e2e"] = {"value": whole_job_rate(world, keys, args.steps, te), "unit": "keys/s",
                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                       "ms_per_step": te / args.steps,
                       "mode": "eager library calls per step, pinned host inputs in, selected indices out"}

@@ -66,6 +66,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // try_wait with a suspend-time hint: the thread may sleep up to `ns` waiting
 // for the phase (and is woken when it completes) instead of polling.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
@@ -90,7 +103,15 @@ struct WaitCtl {
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up
 // (returns false) when another role of the CTA has aborted, or after
 // limit_ns, in which case it records the timeout and raises the abort flag.
+__device__ __forceinline__ bool give_up(const WaitCtl& w) {
+  *w.abort_flag = 1;
+  record_status(w.status, kStatusTimeout);
+  return false;
+}
+
+// A limit of 0 gives up on any wait that is not satisfied when it starts.
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  if (w.limit_ns == 0) return mbar_test_wait(bar, parity) ? true : give_up(w);
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = cycles();
   for (uint32_t it = 1;; ++it) {
@@ -107,6 +128,7 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, con
 // bounded_wait for a waiter that is not on the critical issue path: it
 // sleeps between polls so that it does not crowd the barrier unit.
 __device__ __forceinline__ bool bounded_wait_sleep(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  if (w.limit_ns == 0) return mbar_test_wait(bar, parity) ? true : give_up(w);
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = cycles();
   for (;;) {

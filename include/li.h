@@ -148,7 +148,8 @@ LI_API li_status li_device_status(li_ctx* ctx, const void* ws, void* stream, li_
 /* Upper bound, in nanoseconds, of every wait inside the library's kernels
  * (default 2e9 = 2 s).  When a wait runs out the kernel records
  * LI_ERR_DEVICE_TIMEOUT, drains its own copies in flight, frees its tensor
- * memory and returns. */
+ * memory and returns.  0 makes every wait that is not already satisfied
+ * when it starts give up at once (a way to exercise that path). */
 LI_API li_status li_set_wait_limit(li_ctx* ctx, uint64_t ns);
 
 /* ------------------------------------------------------------- a1: append */
