@@ -339,7 +339,6 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
     // the loader copies each tile's 128 scales in 16-byte pieces
     return fail(ctx, LI_ERR_SHAPE, "%s: scanning an E4M3 cache needs capacity %% 4 == 0 (got %d)", what,
                 c->capacity);
-  a.cache = static_cast<const uint8_t*>(c->data);
   a.cache_scale = c->dtype == LI_E4M3 ? c->scale : nullptr;
   a.lengths = c->lengths;
   a.q_pos = q->q_pos;

@@ -9,6 +9,8 @@
 //
 // Both accumulate in fp32 in a fixed order, so a result is identical whichever
 // output dtype is requested.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -56,6 +58,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const T* __restri
                                                                const T* __restrict__ W, int d_model,
                                                                int dim, int n_tok, int splits,
                                                                float* __restrict__ out) {
+  pdl_begin();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int task = blockIdx.x * kGemvWarps + warp;
   if (task >= dim * splits) return;
@@ -120,9 +123,11 @@ __device__ __forceinline__ void write_row(const float (&v)[8], float amax, int l
 // Decode append in one launch: the split-K GEMV above, after which the last
 // block to finish (a counter in the workspace) adds every token's splits in
 // split order, quantises the rows, writes them at lengths[b] + t, advances
-// lengths[b] by T and resets the counter. Used when all tokens' fp32 rows fit
-// in the block's shared memory.
-constexpr int kFuseMaxFloats = 8192;
+// lengths[b] by T and resets the counter.  The last block first copies all
+// partial sums to shared memory with many loads in flight, then sums each
+// output over the splits in order.  Used when the partials fit in the
+// block's shared memory.
+constexpr int kFuseMaxPartials = 16384;   // floats of partial sums (64 KB)
 
 template <typename T>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* __restrict__ h,
@@ -132,7 +137,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* _
                                                                       void* data, float* scale, int32_t* lengths,
                                                                       int capacity, int dtype,
                                                                       unsigned int* done, int* status) {
-  __shared__ float cs[kFuseMaxFloats];
+  pdl_begin();
+  extern __shared__ __align__(16) float ps[];       // [splits][n_tok * dim], then cs [n_tok * dim]
   __shared__ unsigned last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int task = blockIdx.x * kGemvWarps + warp;
@@ -144,6 +150,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* _
 #pragma unroll
     for (int t = 0; t < kGemvTok; ++t) acc[t] = 0.f;
     const T* wrow = W + static_cast<int64_t>(j) * d_model;
+#pragma unroll 4
     for (int i = i0 + lane * 8; i < i1; i += 256) {
       float wv[8];
       load8<T>(wrow + i, wv);
@@ -173,16 +180,25 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* _
   __syncthreads();
   if (!last) return;
   __threadfence();
-  for (int x = threadIdx.x; x < n_tok * dim; x += blockDim.x) {
-    // every split's partial in flight at once, then added in split order
-    float pv[kMaxSplits];
+  const int nx = n_tok * dim, np = splits * nx;
+  for (int base = threadIdx.x; base < np; base += blockDim.x * 8) {
+    float v[8];
 #pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp)
-      pv[sp] = sp < splits ? __ldcg(part + static_cast<int64_t>(sp) * n_tok * dim + x) : 0.f;
-    float sum = pv[0];
+    for (int m = 0; m < 8; ++m) {
+      const int idx = base + m * static_cast<int>(blockDim.x);
+      v[m] = idx < np ? __ldcg(part + idx) : 0.f;
+    }
 #pragma unroll
-    for (int sp = 1; sp < kMaxSplits; ++sp)
-      if (sp < splits) sum += pv[sp];
+    for (int m = 0; m < 8; ++m) {
+      const int idx = base + m * static_cast<int>(blockDim.x);
+      if (idx < np) ps[idx] = v[m];
+    }
+  }
+  __syncthreads();
+  float* cs = ps + np;
+  for (int x = threadIdx.x; x < nx; x += blockDim.x) {
+    float sum = ps[x];
+    for (int sp = 1; sp < splits; ++sp) sum += ps[sp * nx + x];
     cs[x] = sum;
   }
   __syncthreads();
@@ -223,6 +239,7 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
                                                     void* data, float* scale, int32_t* lengths,
                                                     int capacity, int dim, int dtype,
                                                     unsigned int* done, int* status) {
+  pdl_begin();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok = blockIdx.x * 8 + warp;
   if (tok < batch * T_chunk) {
@@ -288,6 +305,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(const T* __restrict__ q, in
                                                      const float* __restrict__ bK, int64_t b_hs, int d_c,
                                                      int out_dtype, void* q_abs, float* q_abs_scale,
                                                      float* beta) {
+  pdl_begin();
   __shared__ float qs[kAbsorbHeads][256];
   __shared__ float red[8][kAbsorbHeads];
   const int t = blockIdx.y, h0 = blockIdx.x * kAbsorbHeads;
@@ -390,6 +408,7 @@ __global__ void __launch_bounds__(256) absorb_shared_kernel(const T* __restrict_
                                                             const float* __restrict__ bK, int d_c, int R,
                                                             int out_dtype, void* q_abs, float* q_abs_scale,
                                                             float* beta) {
+  pdl_begin();
   extern __shared__ __align__(16) unsigned char absorb_smem[];
   T* Ws = reinterpret_cast<T*>(absorb_smem);                                   // [d_k][d_c]
   float* qs = reinterpret_cast<float*>(absorb_smem + (static_cast<size_t>(d_k) * d_c * sizeof(T) + 15) / 16 * 16);
@@ -476,19 +495,27 @@ cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_
                                int splits, float* out, cudaStream_t st) {
   const dim3 grid((dim * splits + kGemvWarps - 1) / kGemvWarps, (n_tok + kGemvTok - 1) / kGemvTok);
   if (h_dtype == LI_BF16)
-    gemv_kernel<__nv_bfloat16><<<grid, kGemvWarps * 32, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim,
-        n_tok, splits, out);
-  else
-    gemv_kernel<float><<<grid, kGemvWarps * 32, 0, st>>>(reinterpret_cast<const float*>(h),
-                                                          reinterpret_cast<const float*>(W), d_model, dim,
-                                                          n_tok, splits, out);
-  return cudaGetLastError();
+    return launch_pdl(gemv_kernel<__nv_bfloat16>, grid, dim3(kGemvWarps * 32), 0, st, 1,
+                      reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(W), d_model,
+                      dim, n_tok, splits, out);
+  return launch_pdl(gemv_kernel<float>, grid, dim3(kGemvWarps * 32), 0, st, 1, reinterpret_cast<const float*>(h),
+                    reinterpret_cast<const float*>(W), d_model, dim, n_tok, splits, out);
+}
+
+int append_fused_splits(int d_model, int dim) {
+  // enough (output, split) warp tasks for a wave of 8 warps on every SM, with
+  // slices of whole 256-element steps
+  if (d_model % 256) return 0;
+  const int steps = d_model / 256;
+  for (int sp = 1; sp <= steps && sp <= kMaxSplits; ++sp)
+    if (steps % sp == 0 && dim * sp >= 148 * kGemvWarps) return sp;
+  for (int sp = std::min(steps, kMaxSplits); sp >= 1; --sp)
+    if (steps % sp == 0) return sp;
+  return 1;
 }
 
 bool append_fusable(int n_tok, int dim, int splits) {
-  return n_tok <= kGemvTok && n_tok * dim <= kFuseMaxFloats && dim <= 256;
-  (void)splits;
+  return splits >= 1 && n_tok <= kGemvTok && dim <= 256 && (splits + 1) * n_tok * dim <= kFuseMaxPartials;
 }
 
 cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
@@ -496,15 +523,21 @@ cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d
                                 int dtype, unsigned int* done, int* status, cudaStream_t st) {
   const int n_tok = batch * T;
   const int grid = (dim * splits + kGemvWarps - 1) / kGemvWarps;
-  if (h_dtype == LI_BF16)
-    gemv_append_kernel<__nv_bfloat16><<<grid, kGemvWarps * 32, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(h), reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim, n_tok,
-        splits, part, batch, T, data, scale, lengths, capacity, dtype, done, status);
-  else
-    gemv_append_kernel<float><<<grid, kGemvWarps * 32, 0, st>>>(
-        reinterpret_cast<const float*>(h), reinterpret_cast<const float*>(W), d_model, dim, n_tok, splits, part,
-        batch, T, data, scale, lengths, capacity, dtype, done, status);
-  return cudaGetLastError();
+  const size_t smem = static_cast<size_t>(splits + 1) * n_tok * dim * sizeof(float);
+  cudaError_t e;
+  if (h_dtype == LI_BF16) {
+    auto k = gemv_append_kernel<__nv_bfloat16>;
+    if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
+    return launch_pdl(k, dim3(grid), dim3(kGemvWarps * 32), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(h),
+                      reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim, n_tok, splits, part, batch, T, data,
+                      scale, lengths, capacity, dtype, done, status);
+  } else {
+    auto k = gemv_append_kernel<float>;
+    if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
+    return launch_pdl(k, dim3(grid), dim3(kGemvWarps * 32), smem, st, 1, reinterpret_cast<const float*>(h),
+                      reinterpret_cast<const float*>(W), d_model, dim, n_tok, splits, part, batch, T, data, scale,
+                      lengths, capacity, dtype, done, status);
+  }
 }
 
 cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits, int batch,
@@ -513,9 +546,8 @@ cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t sp
                                 int* status, cudaStream_t st) {
   const int n_tok = batch * T_chunk;
   const int grid = (n_tok + 7) / 8;
-  store_kernel<<<grid, 256, 0, st>>>(c, c_tok_stride, split_stride, splits, batch, T_chunk, t0, T_total,
-                                     bump ? 1 : 0, data, scale, lengths, capacity, dim, dtype, done_counter, status);
-  return cudaGetLastError();
+  return launch_pdl(store_kernel, dim3(grid), dim3(256), 0, st, 1, c, c_tok_stride, split_stride, splits, batch, T_chunk,
+                    t0, T_total, bump ? 1 : 0, data, scale, lengths, capacity, dim, dtype, done_counter, status);
 }
 
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
@@ -536,28 +568,24 @@ cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k,
       auto k = absorb_shared_kernel<__nv_bfloat16>;
       e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
       if (e != cudaSuccess) return e;
-      k<<<grid, 256, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), M, d_k,
-                                 reinterpret_cast<const __nv_bfloat16*>(W), b, d_c, R, out_dtype, q_abs,
-                                 q_abs_scale, beta);
+      return launch_pdl(k, dim3(grid), dim3(256), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(q), M, d_k,
+                        reinterpret_cast<const __nv_bfloat16*>(W), b, d_c, R, out_dtype, q_abs, q_abs_scale, beta);
     } else {
       auto k = absorb_shared_kernel<float>;
       e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
       if (e != cudaSuccess) return e;
-      k<<<grid, 256, smem, st>>>(reinterpret_cast<const float*>(q), M, d_k, reinterpret_cast<const float*>(W), b,
-                                 d_c, R, out_dtype, q_abs, q_abs_scale, beta);
+      return launch_pdl(k, dim3(grid), dim3(256), smem, st, 1, reinterpret_cast<const float*>(q), M, d_k,
+                        reinterpret_cast<const float*>(W), b, d_c, R, out_dtype, q_abs, q_abs_scale, beta);
     }
-    return cudaGetLastError();
   }
   const dim3 grid((H + kAbsorbHeads - 1) / kAbsorbHeads, n_tok);
   if (q_dtype == LI_BF16)
-    absorb_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), H, d_k,
-                                                       reinterpret_cast<const __nv_bfloat16*>(W), W_head_stride, b,
-                                                       b_head_stride, d_c, out_dtype, q_abs, q_abs_scale, beta);
-  else
-    absorb_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(q), H, d_k,
-                                               reinterpret_cast<const float*>(W), W_head_stride, b, b_head_stride,
-                                               d_c, out_dtype, q_abs, q_abs_scale, beta);
-  return cudaGetLastError();
+    return launch_pdl(absorb_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, 1,
+                      reinterpret_cast<const __nv_bfloat16*>(q), H, d_k, reinterpret_cast<const __nv_bfloat16*>(W),
+                      W_head_stride, b, b_head_stride, d_c, out_dtype, q_abs, q_abs_scale, beta);
+  return launch_pdl(absorb_kernel<float>, grid, dim3(256), 0, st, 1, reinterpret_cast<const float*>(q), H, d_k,
+                    reinterpret_cast<const float*>(W), W_head_stride, b, b_head_stride, d_c, out_dtype, q_abs,
+                    q_abs_scale, beta);
 }
 
 }  // namespace li

@@ -24,7 +24,6 @@ struct alignas(64) ScanArgs {
   CUtensorMap map_a;          // cache rows: dims {swz/elt, batch*capacity, n_kchunks}, box {swz/elt, R, KS};
                               // gather: dims {dim, batch*capacity}, box {swz/elt, 1}
   CUtensorMap map_b;          // queries: dims {dim, H, batch*T}, box {swz/elt, H_pad, Qg}
-  const uint8_t* cache;       // cache data (gather loads)
   const float* cache_scale;   // [batch*capacity] or null
   const int* lengths;         // [batch]
   const int* q_pos;           // [batch*T] or null
@@ -60,6 +59,35 @@ constexpr int kTraceCtas = 8, kTraceTiles = 64, kTraceEvents = 8;
 // Kernel families (for the launch profile).
 enum KernelKind { kKScan = 0, kKGather, kKTopkHist, kKTopkFilter, kKTopkSelect, kKTopkEmit,
                   kKAppendGemv, kKAppendStore, kKAbsorb, kKMemset };
+
+// Launch `kernel` with programmatic stream serialisation (it may begin while
+// the previous kernel on the stream finishes; the kernel itself waits for it
+// in pdl_begin() before touching global memory), as a cluster of cluster_x
+// CTAs along x when cluster_x > 1.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
 // current device. The attribute is set once per (kernel, device) and
@@ -119,9 +147,10 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st);
 int gemv_splits(int d_model, int n_tok);
 cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_model, int dim,
                                int n_tok, int splits, float* out, cudaStream_t st);
-// Decode-sized appends (at most 8 tokens, rows fitting one block's shared
-// memory) run as one launch: split-K GEMV, then the last block reduces the
-// splits in order and stores the rows.
+// Decode-sized appends (at most 8 tokens whose partial sums fit one block's
+// shared memory) run as one launch: split-K GEMV, then the last block
+// reduces the splits in order and stores the rows.
+int append_fused_splits(int d_model, int dim);
 bool append_fusable(int n_tok, int dim, int splits);
 cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
                                 int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,

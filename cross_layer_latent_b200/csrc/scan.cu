@@ -139,17 +139,6 @@ struct SegWalk {
   }
 };
 
-// Swizzled byte offset inside a K-major tile whose rows are `swz` bytes.
-__device__ __forceinline__ uint32_t swizzle(uint32_t off, uint32_t swz) {
-  return off ^ (((off >> 7) & ((swz >> 4) - 1u)) << 4);
-}
-
-// 16-byte cp.async reading src_bytes (0..16) and zero-filling the rest.
-__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst_smem, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-
 // 4-byte cp.async reading src_bytes (0 or 4).
 __device__ __forceinline__ void cp_async_4_zfill(uint32_t dst_smem, const void* src, int src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
@@ -257,11 +246,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     mbar_init(s.drain, 1);
     *s.abort_flag = 0;
     fence_barrier_init();
+    tma_prefetch_desc(&a.map_a);
+    tma_prefetch_desc(&a.map_b);
   }
   if (warp == 1) {
     tmem_alloc(s.tmem_base, a.tmem_cols);
     tmem_relinquish();
   }
+  // everything above touches only this CTA's own resources; the lengths,
+  // queries and cache rows below may come from the previous kernel
+  pdl_begin();
   // Items per segment, then an exclusive prefix over segments.
   for (int i = tid; i < a.n_segments; i += blockDim.x) {
     s.prefix[i + 1] = segment_items<GATHER>(a, i);
@@ -301,8 +295,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const int k_R = a.R, k_MB = a.MB, k_KS = a.KS, k_spi = a.stages_per_item;
   const uint32_t k_a_stage_bytes = a.a_stage_bytes, k_b_slot_bytes = a.b_slot_bytes, k_idesc = a.idesc;
   const uint32_t k_meta_bytes = a.meta_bytes;
-  const int64_t k_row_bytes = a.row_bytes, k_score_stride = a.score_stride;
-  const uint8_t* const k_cache = a.cache;
+  const int64_t k_score_stride = a.score_stride;
   const float* const k_cache_scale = a.cache_scale;
   const int* const k_lengths = a.lengths;
   const int* const k_q_pos = a.q_pos;
@@ -330,8 +323,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   if (warp == 0 && !GATHER) {
     // ------------------------------------------------------------ loader (TMA), one lane
     if (lane == 0) {
-      tma_prefetch_desc(&a.map_a);
-      tma_prefetch_desc(&a.map_b);
       Ring st, bs, ms;
       uint32_t n_st = 0, n_bs = 0, n_ms = 0;
       SegWalk w{s.prefix, n_groups};
@@ -681,8 +672,7 @@ cudaError_t launch_one(const ScanArgs& a, int grid, cudaStream_t st) {
   auto k = scan_kernel<KIND, GATHER>;
   const cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(k), a.smem_bytes);
   if (e != cudaSuccess) return e;
-  k<<<grid, kScanThreads, a.smem_bytes, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(grid), dim3(kScanThreads), a.smem_bytes, st, 1, a);
 }
 
 }  // namespace

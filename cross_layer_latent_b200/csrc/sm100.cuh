@@ -152,6 +152,19 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Every kernel of the library is launched with programmatic stream
+// serialisation, so it may start while the previous kernel on the stream is
+// finishing.  pdl_begin() waits until that kernel has completed and its
+// memory is visible (no global memory is touched before it), then lets the
+// next kernel start its own prologue.  Without the launch attribute both are
+// no-ops.
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {

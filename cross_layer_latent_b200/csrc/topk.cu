@@ -112,6 +112,7 @@ __device__ void find_bucket_asc(const unsigned* h, int nbins, int need, int* scr
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const TopkArgs a) {
+  pdl_begin();
   __shared__ unsigned h[kHistBins];
   const int r = blockIdx.y, c = blockIdx.x;
   const int n = row_len(a, r);
@@ -128,6 +129,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_hist_kernel(const TopkArgs 
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_filter_kernel(const TopkArgs a) {
+  pdl_begin();
   __shared__ unsigned h[kHistBins];
   __shared__ int scratch[32];
   __shared__ int res[2];
@@ -189,6 +191,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_filter_kernel(const TopkArg
 constexpr int kSelectThreads = 1024;
 
 __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(const TopkArgs a) {
+  pdl_begin();
   __shared__ unsigned h[kHistBins];
   __shared__ int scratch[32];
   __shared__ int res[2];
@@ -293,6 +296,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(const TopkA
 constexpr int kEmitPerThread = kTopkChunk / kTopkThreads;   // 16
 
 __global__ void __launch_bounds__(kTopkThreads) topk_emit_kernel(const TopkArgs a) {
+  pdl_begin();
   __shared__ int scratch[32];
   const int r = blockIdx.y, c = blockIdx.x;
   const int* info = a.rowinfo + static_cast<int64_t>(r) * 16;
@@ -340,10 +344,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_emit_kernel(const TopkArgs 
 cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
   const dim3 grid_chunks(a.n_chunks, a.rows);
   switch (stage) {
-    case 0: topk_hist_kernel<<<grid_chunks, kTopkThreads, 0, st>>>(a); break;
-    case 1: topk_filter_kernel<<<grid_chunks, kTopkThreads, 0, st>>>(a); break;
-    case 2: topk_select_kernel<<<a.rows, kSelectThreads, 0, st>>>(a); break;
-    case 3: topk_emit_kernel<<<grid_chunks, kTopkThreads, 0, st>>>(a); break;
+    case 0: return launch_pdl(topk_hist_kernel, grid_chunks, dim3(kTopkThreads), 0, st, 1, a);
+    case 1: return launch_pdl(topk_filter_kernel, grid_chunks, dim3(kTopkThreads), 0, st, 1, a);
+    case 2: return launch_pdl(topk_select_kernel, dim3(a.rows), dim3(kSelectThreads), 0, st, 1, a);
+    case 3: return launch_pdl(topk_emit_kernel, grid_chunks, dim3(kTopkThreads), 0, st, 1, a);
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -500,6 +504,7 @@ __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, un
 
 template <int PT, bool CL>
 __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const TopkArgs a) {
+  pdl_begin();
   constexpr int NW = kClusterThreads / 32;
   constexpr int NSLAB = PT / 4;
   __shared__ __align__(16) unsigned H1[2048];                       // top 11 bits
@@ -687,23 +692,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
 
 template <int PT>
 cudaError_t launch_radix_pt(const TopkArgs& a, int cs, cudaStream_t st) {
-  if (cs == 1) {
-    topk_radix_kernel<PT, false><<<dim3(1, a.rows, 1), kClusterThreads, 0, st>>>(a);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cs, a.rows, 1);
-  cfg.blockDim = dim3(kClusterThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_radix_kernel<PT, true>, a);
+  if (cs == 1) return launch_pdl(topk_radix_kernel<PT, false>, dim3(1, a.rows, 1), dim3(kClusterThreads), 0, st, 1, a);
+  return launch_pdl(topk_radix_kernel<PT, true>, dim3(cs, a.rows, 1), dim3(kClusterThreads), 0, st, cs, a);
 }
 
 }  // namespace
