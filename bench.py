@@ -261,15 +261,17 @@ def scan_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kind):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source."""
+def profiled_traffic(group):
+    """DRAM bytes per scan launch, averaged over a step's launches (the
+    anchor's latent scan and `group` DSA key scans) like the achieved rate,
+    from the committed ncu capture -- None unless it was taken on the current
+    kernel source."""
     try:
         with open(os.path.join(ROOT, "profiles", "scan_traffic.json")) as f:
             t = json.load(f)
         if t.get("source_hash") != scan_source_hash():
             return None
-        return t.get(kind)
+        return (t["anchor_dram_bytes_per_launch"] + group * t["dsa_dram_bytes_per_launch"]) / (group + 1)
     except Exception:
         return None
 
@@ -495,7 +497,7 @@ def main():
     scan_ms = sum(r["ms"] for r in scans)
     peak, peak_kind = measured_peaks()
     achieved = alg_bytes / (scan_ms / 1e3) / 1e9 if scan_ms > 0 else 0.0
-    traffic = profiled_traffic("scan_dram_bytes_per_launch")
+    traffic = profiled_traffic(wl.group) if args.workload == 3 else None
     by_kernel = {}
     for r in recs:
         d = by_kernel.setdefault(r["kernel"], {"launches": 0, "ms": 0.0})
@@ -515,6 +517,7 @@ def main():
                         "kernel": "scan (tcgen05 latent / key scan, fused ReLU-weighted head reduction)",
                         "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                         "alg_bytes_per_key": {"latent": row_latent, "dsa_key": row_key},
+                        "alg_bytes_per_launch": alg_bytes / max(len(scans), 1),
                         "launches_per_step": per_step, "scan_ms_per_step": scan_ms / args.steps,
                         "timing": "CUDA event pair around every launch on the launching stream, in a "
                                   "second timed pass of the same steps (eager, the GPU kept ahead of the host)"},

@@ -207,8 +207,11 @@ li_status check_ws(li_ctx* ctx, void* ws, size_t ws_bytes, const WsLayout& L, co
 
 // ------------------------------------------------------------------ tensor maps
 
+// Tiled loads stream whole rows and use 256-byte L2 promotion; row gathers
+// read scattered rows and ask for none (promotion would pull in neighbouring
+// sectors of every gathered row).
 li_status encode_map(li_ctx* ctx, CUtensorMap* m, li_dtype dt, int rank, void* base, const cuuint64_t* dims,
-                     const cuuint64_t* strides, const cuuint32_t* box, int swz) {
+                     const cuuint64_t* strides, const cuuint32_t* box, int swz, bool promote = true) {
   const CUtensorMapDataType t = dt == LI_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                 : dt == LI_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -217,7 +220,8 @@ li_status encode_map(li_ctx* ctx, CUtensorMap* m, li_dtype dt, int rank, void* b
                                             : CU_TENSOR_MAP_SWIZZLE_32B;
   const cuuint32_t es[3] = {1, 1, 1};
   const CUresult r = ctx->encode(m, t, rank, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                                 promote ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(ctx, LI_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return LI_OK;
 }
@@ -314,7 +318,7 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c->dim), static_cast<cuuint64_t>(c->batch) * c->capacity};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(swz / eb), 1};
-    li_status s = encode_map(ctx, &a.map_a, c->dtype, 2, c->data, dims, strides, box, swz);
+    li_status s = encode_map(ctx, &a.map_a, c->dtype, 2, c->data, dims, strides, box, swz, false);
     if (s != LI_OK) return s;
   } else {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(swz / eb), static_cast<cuuint64_t>(c->batch) * c->capacity,

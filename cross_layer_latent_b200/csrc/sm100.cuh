@@ -157,13 +157,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 // Every kernel of the library is launched with programmatic stream
 // serialisation, so it may start while the previous kernel on the stream is
 // finishing.  pdl_begin() waits until that kernel has completed and its
-// memory is visible (no global memory is touched before it), then lets the
-// next kernel start its own prologue.  Without the launch attribute both are
-// no-ops.
-__device__ __forceinline__ void pdl_begin() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
+// memory is visible (no global memory is touched before it).  Dependents
+// are not released early: they launch as this kernel's CTAs exit (released
+// early, a waiting dependent that fits beside this kernel's CTAs shares
+// their SMs and slows them down).  Without the launch attribute it is a
+// no-op.
+__device__ __forceinline__ void pdl_begin() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ------------------------------------------------------------------ TMA
 
