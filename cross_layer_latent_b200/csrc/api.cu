@@ -268,38 +268,64 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   a.idesc = make_instr_desc(fmt, 128, N);
   a.b_slot_bytes = static_cast<uint32_t>(a.n_kchunks) * N * swz;
   // Work item of R rows (two M=128 blocks when both accumulators of every
-  // in-flight item fit tensor memory), stage of KS K-chunks: the largest
-  // stage that still leaves a pipeline of several stages.
+  // in-flight item fit tensor memory), stage of KS K-chunks.  Among the
+  // layouts that fit, the one with the deepest pipeline wins: items in
+  // flight = min(stages / stages_per_item, metadata slots - 2), so the
+  // metadata ring never throttles the stage ring; then more query slots.
   const bool has_meta = gather || c->dtype == LI_E4M3;
-  const size_t fixed_misc = 1024 + 16 + (kMaxSegments + 1) * 4 + 16 + kEpiWarps * (3 * N + 16) * 4 +
-                            (gather ? 2 * kMaxSegments * 4 : 0);
+  const int ep_stride = (q->beta ? 3 * N : N) + 16;
+  // barriers (2 x kMaxStages + 2 + 2 + 8 + 8 + 2 x kMetaSlots + 2) x 8 B,
+  // tensor-memory base, abort flag, prefix, epilogue parameters, gather limits
+  const size_t fixed_misc = static_cast<size_t>(2 * kMaxStages + 22 + 2 * kMetaSlots) * 8 + 16 +
+                            static_cast<size_t>(n_seg + 1) * 4 + 16 + static_cast<size_t>(kEpiWarps) * ep_stride * 4 +
+                            (gather ? static_cast<size_t>(2 * n_seg) * 4 : 0) + 64;
   const size_t budget = static_cast<size_t>(ctx->max_smem_optin) - 1024;
   const size_t kStageCap = 48 * 1024;
   bool planned = false;
   for (int R = (2 * N <= 256 && !gather) ? 256 : 128; R >= 128 && !planned; R -= 128) {
-    const size_t meta = has_meta ? static_cast<size_t>(kMetaSlots) * 8 * R : 0;
+    const uint32_t meta_bytes = has_meta ? static_cast<uint32_t>((gather ? 8 : 4) * R) : 0u;
     for (int KS = a.n_kchunks; KS >= 1 && !planned; --KS) {
       if (a.n_kchunks % KS) continue;
       const size_t stage = static_cast<size_t>(R) * swz * KS;
       if (stage > kStageCap && KS > 1) continue;
-      for (int bslots = 2; bslots >= 1 && !planned; --bslots) {
-        const int64_t room = static_cast<int64_t>(budget) - static_cast<int64_t>(bslots) * a.b_slot_bytes -
-                             static_cast<int64_t>(meta + fixed_misc);
-        const int stages = room > 0 ? static_cast<int>(std::min<int64_t>(kMaxStages, room / stage)) : 0;
-        const int need = KS < a.n_kchunks ? 4 : 3;
-        if (stages < need) continue;
-        a.R = R;
-        a.MB = R / 128;
-        a.KS = KS;
-        a.stages_per_item = a.n_kchunks / KS;
-        a.n_stages = stages;
-        a.n_bslots = bslots;
-        a.a_stage_bytes = static_cast<uint32_t>(stage);
-        a.meta_bytes = static_cast<uint32_t>(8 * R);
-        a.misc_offset = static_cast<uint32_t>(stages * stage + bslots * a.b_slot_bytes + meta);
-        a.smem_bytes = static_cast<uint32_t>(std::max<size_t>(1024 + a.misc_offset + fixed_misc, 120 * 1024));
-        planned = true;
+      const int spi = a.n_kchunks / KS;
+      const int need = KS < a.n_kchunks ? 4 : 3;
+      // Two query slots let a CTA whose items cross into the next segment
+      // load its queries ahead; one slot is taken only with a single segment
+      // (or when two leave no room for the minimum ring).
+      int best_depth = -1, best_stages = 0, best_bslots = 0, best_meta = 0;
+      for (int bslots = 2; bslots >= 1; --bslots) {
+        if (bslots == 1 && n_seg > 1 && best_stages >= need) break;
+        for (int nm = has_meta ? kMetaSlots : 0; nm >= (has_meta ? 4 : 0); --nm) {
+          const int64_t room = static_cast<int64_t>(budget) - static_cast<int64_t>(bslots) * a.b_slot_bytes -
+                               static_cast<int64_t>(nm) * meta_bytes - static_cast<int64_t>(fixed_misc);
+          const int stages = room > 0 ? static_cast<int>(std::min<int64_t>(kMaxStages, room / stage)) : 0;
+          // stages the metadata ring lets the loader run ahead
+          const int depth = has_meta ? std::min(stages, (nm - 2) * spi) : stages;
+          if (depth > best_depth) {
+            best_depth = depth;
+            best_stages = stages;
+            best_bslots = bslots;
+            best_meta = nm;
+          }
+          if (!has_meta) break;
+        }
       }
+      if (best_stages < need) continue;
+      a.R = R;
+      a.MB = R / 128;
+      a.KS = KS;
+      a.stages_per_item = spi;
+      a.n_stages = best_stages;
+      a.n_bslots = best_bslots;
+      a.n_meta = best_meta;
+      a.ep_stride = ep_stride;
+      a.a_stage_bytes = static_cast<uint32_t>(stage);
+      a.meta_bytes = meta_bytes;
+      a.misc_offset = static_cast<uint32_t>(best_stages * stage + best_bslots * a.b_slot_bytes +
+                                            static_cast<size_t>(best_meta) * meta_bytes);
+      a.smem_bytes = static_cast<uint32_t>(std::max<size_t>(1024 + a.misc_offset + fixed_misc, 120 * 1024));
+      planned = true;
     }
   }
   if (!planned || a.smem_bytes > static_cast<uint32_t>(ctx->max_smem_optin))

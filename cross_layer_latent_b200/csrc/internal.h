@@ -11,7 +11,10 @@ namespace li {
 
 constexpr int kTileM = 128;          // cache rows per MMA tile (UMMA M)
 constexpr int kEpiWarps = 8;         // two epilogue warpgroups, alternating tiles
-constexpr int kScanThreads = 64 + 32 * kEpiWarps;   // warp 0 loads, warp 1 issues MMAs
+// warp 0 loads, warps 1 and 2 + kEpiWarps issue the MMAs of the two M blocks,
+// warps 2 .. 1 + kEpiWarps run the epilogue
+constexpr int kScanThreads = 96 + 32 * kEpiWarps;
+constexpr int kMmaWarp2 = 2 + kEpiWarps;
 constexpr int kMetaSlots = 8;        // ring of per-item row metadata (fp8 scales, gathered rows)
 constexpr int kMaxItemRows = 256;    // rows of one work item (two M=128 MMA blocks)
 constexpr int kMaxSegments = 1024;   // (sequence, query group) segments per scan launch
@@ -42,7 +45,8 @@ struct alignas(64) ScanArgs {
   int swz, n_kchunks, elt_bytes;
   int R, MB;                  // rows per work item (128 or 256) and M=128 blocks per item
   int KS, stages_per_item;    // K-chunks per stage, stages per item
-  int n_stages, n_bslots, n_acc;
+  int n_stages, n_bslots, n_acc, n_meta;
+  int ep_stride;              // floats of epilogue parameters per epilogue warp
   uint32_t tmem_cols, idesc;
   uint32_t a_stage_bytes, b_slot_bytes, meta_bytes, misc_offset, smem_bytes;
   int n_segments;

@@ -40,7 +40,7 @@ constexpr uint64_t kDrainNs = 200ull * 1000ull * 1000ull;   // 0.2 s
 struct ScanSmem {
   uint8_t* a_stages;
   uint8_t* b_slots;
-  uint8_t* meta;        // kMetaSlots x meta_bytes: scale[R] then tok[R]
+  uint8_t* meta;        // n_meta x meta_bytes: scale[R] (then tok[R] when gathering)
   uint64_t* full;
   uint64_t* empty;
   uint64_t* bfull;
@@ -52,12 +52,14 @@ struct ScanSmem {
   uint64_t* drain;
   uint32_t* tmem_base;
   int* abort_flag;
-  int* prefix;          // [kMaxSegments + 1]
-  float* ep;            // kEpiWarps x (3 * N + 16) floats
-  int* seg_n;           // gather: [kMaxSegments] candidates of each segment (clamped)
-  int* seg_len;         // gather: [kMaxSegments] valid length of the segment's sequence
+  int* prefix;          // [n_segments + 1]
+  float* ep;            // kEpiWarps x ep_stride floats
+  int* seg_n;           // gather: [n_segments] candidates of each segment (clamped)
+  int* seg_len;         // gather: [n_segments] valid length of the segment's sequence
 };
 
+// Shared-memory layout; scan_misc_bytes() on the host sizes the part after
+// misc_offset the same way.
 __device__ __forceinline__ ScanSmem carve(uint8_t* base, const ScanArgs& a) {
   ScanSmem s;
   s.a_stages = base;
@@ -68,18 +70,18 @@ __device__ __forceinline__ ScanSmem carve(uint8_t* base, const ScanArgs& a) {
   s.empty = s.full + kMaxStages;
   s.bfull = s.empty + kMaxStages;
   s.bempty = s.bfull + 2;
-  s.accfull = s.bempty + 2;
-  s.accempty = s.accfull + 4;
-  s.mfull = s.accempty + 4;
+  s.accfull = s.bempty + 2;               // [accumulator slot][M block]
+  s.accempty = s.accfull + 8;
+  s.mfull = s.accempty + 8;
   s.mempty = s.mfull + kMetaSlots;
-  s.drain = s.mempty + kMetaSlots;
-  s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.drain = s.mempty + kMetaSlots;        // one per MMA issuer
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 2);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
   s.prefix = s.abort_flag + 2;
   // 16-byte aligned parameter arrays (read four at a time)
-  s.ep = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s.prefix + kMaxSegments + 1) + 15) & ~uintptr_t(15));
-  s.seg_n = reinterpret_cast<int*>(s.ep + kEpiWarps * (3 * a.N + 16));
-  s.seg_len = s.seg_n + kMaxSegments;
+  s.ep = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s.prefix + a.n_segments + 1) + 15) & ~uintptr_t(15));
+  s.seg_n = reinterpret_cast<int*>(s.ep + kEpiWarps * a.ep_stride);
+  s.seg_len = s.seg_n + a.n_segments;
   return s;
 }
 
@@ -234,16 +236,19 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const bool has_meta = GATHER || e4;
 
   if (tid == 0) {
-    for (int i = 0; i < a.n_stages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
-    for (int i = 0; i < a.n_bslots; ++i) { mbar_init(&s.bfull[i], 1); mbar_init(&s.bempty[i], 1); }
-    for (int i = 0; i < a.n_acc; ++i) { mbar_init(&s.accfull[i], 1); mbar_init(&s.accempty[i], 4 * a.MB); }
+    // every MMA issuer (one per M block) releases stages and query slots
+    for (int i = 0; i < a.n_stages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], a.MB); }
+    for (int i = 0; i < a.n_bslots; ++i) { mbar_init(&s.bfull[i], 1); mbar_init(&s.bempty[i], a.MB); }
+    // accumulator (slot, M block): one issuer fills it, one warpgroup drains it
+    for (int i = 0; i < 2 * a.n_acc; ++i) { mbar_init(&s.accfull[i], 1); mbar_init(&s.accempty[i], 4); }
     for (int i = 0; i < kMetaSlots; ++i) {
       // gather: every loader lane arrives once after storing its token ids
       // and once (asynchronously) when its scale copies have landed
       mbar_init(&s.mfull[i], GATHER ? 64 : 1);
       mbar_init(&s.mempty[i], 4 * a.MB);
     }
-    mbar_init(s.drain, 1);
+    mbar_init(&s.drain[0], 1);
+    mbar_init(&s.drain[1], 1);
     *s.abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&a.map_a);
@@ -316,6 +321,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const uint32_t S = static_cast<uint32_t>(a.n_stages);
   const uint32_t NB = static_cast<uint32_t>(a.n_bslots);
   const uint32_t NA = static_cast<uint32_t>(a.n_acc);
+  const uint32_t NM = static_cast<uint32_t>(a.n_meta);
   const int elt_per_chunk = k_swz / a.elt_bytes;
   const int n_groups = GATHER ? k_T : a.n_groups;
   const uint32_t chunk_region = static_cast<uint32_t>(k_R * k_swz);   // one K-chunk of a stage
@@ -353,7 +359,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           mbar_arrive_expect_tx(&s.mfull[ms.i], bytes);
           bulk_load(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes,
                     k_cache_scale + static_cast<int64_t>(w.b) * k_capacity + it * k_R, bytes, &s.mfull[ms.i]);
-          ms.step(kMetaSlots);
+          ms.step(NM);
           ++n_ms;
         }
         const int row0 = w.b * k_capacity + it * k_R;
@@ -374,7 +380,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         // let every copy already issued land before the CTA exits
         drain_ring(s.full, S, n_st);
         drain_ring(s.bfull, NB, n_bs);
-        drain_ring(s.mfull, kMetaSlots, n_ms);
+        drain_ring(s.mfull, NM, n_ms);
       }
     }
   } else if (warp == 0) {
@@ -448,7 +454,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       cp_async_arrive_noinc(&s.mfull[ms.i]);
       mbar_arrive(&s.mfull[ms.i]);
       __syncwarp();
-      ms.step(kMetaSlots);
+      ms.step(NM);
       bool ok = true;
       for (int sp = 0; sp < k_spi; ++sp) {
         if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
@@ -475,9 +481,14 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         drain_ring(s.bfull, NB, n_bs);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer, one lane
-    if (lane == 0) {
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    // ------------------------------------------------------------ MMA issuers, one lane each
+    // Issuer mi issues the MMAs of M block mi of every item (with one M
+    // block per item only warp 1 works): each waits for the stage and for its
+    // accumulator, issues and commits on its own, so the per-item waits and
+    // the MMA issue of the two blocks overlap.
+    const int mi = warp == 1 ? 0 : 1;
+    if (lane == 0 && mi < k_MB) {
       Ring st, bs, acc;
       SegWalk w{s.prefix, n_groups};
       bool first = true;
@@ -486,7 +497,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       // K-major swizzled descriptors: everything but the start address is
       // fixed, so only the address field is added per MMA.
       const uint64_t desc_hi = make_smem_desc(0, static_cast<uint32_t>(k_swz));
-      const uint32_t m_stride = static_cast<uint32_t>(128 * k_swz);     // next M block in a chunk
+      const uint32_t m_off = static_cast<uint32_t>(mi * 128 * k_swz);   // this M block within a chunk
       const uint32_t ksteps = static_cast<uint32_t>(k_swz >> 5);
       for (int item = begin; item < end; ++item, ++lt) {
         if (*s.abort_flag) break;
@@ -499,34 +510,36 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           slot = static_cast<int>(bs.i);
           bs.step(NB);
         }
-        if (!bounded_wait(&s.accempty[acc.i], acc.ph ^ 1u, wc)) break;
+        uint64_t* accf = &s.accfull[2 * acc.i + mi];
+        if (!bounded_wait(&s.accempty[2 * acc.i + mi], acc.ph ^ 1u, wc)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem + acc.i * static_cast<uint32_t>(k_MB * k_N);
+        const uint32_t d0 = tmem + (acc.i * static_cast<uint32_t>(k_MB) + static_cast<uint32_t>(mi)) *
+                                       static_cast<uint32_t>(k_N);
         const uint32_t b_base = smem_addr(s.b_slots + static_cast<size_t>(slot) * k_b_slot_bytes);
         bool ok = true;
         for (int sp = 0; sp < k_spi; ++sp) {
-          if (sp == 0) trace_event(k_trace, lt, 6);
+          if (sp == 0 && mi == 0) trace_event(k_trace, lt, 6);
           if (!bounded_wait(&s.full[st.i], st.ph, wc)) { ok = false; break; }
-          if (sp == 0) trace_event(k_trace, lt, 2);
+          if (sp == 0 && mi == 0) trace_event(k_trace, lt, 2);
           tc_fence_after();
-          const uint32_t a_base = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
+          const uint32_t a_base = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes) + m_off;
           for (int c = 0; c < k_KS; ++c) {
             const int kc = sp * k_KS + c;
-            issue_chunk_rt<KIND>(static_cast<int>(ksteps), k_MB, d0, a_base + static_cast<uint32_t>(c) * chunk_region,
-                                 b_base + static_cast<uint32_t>(kc * k_N * k_swz), desc_hi, m_stride,
+            issue_chunk_rt<KIND>(static_cast<int>(ksteps), 1, d0, a_base + static_cast<uint32_t>(c) * chunk_region,
+                                 b_base + static_cast<uint32_t>(kc * k_N * k_swz), desc_hi, 0u,
                                  static_cast<uint32_t>(k_N), k_idesc, kc == 0);
           }
           umma_commit(&s.empty[st.i]);
           st.step(S);
         }
         if (!ok) break;
-        umma_commit(&s.accfull[acc.i]);
-        trace_event(k_trace, lt, 3);
+        umma_commit(accf);
+        if (mi == 0) trace_event(k_trace, lt, 3);
         acc.step(NA);
       }
       if (*s.abort_flag) {
-        umma_commit(s.drain);
-        drain_wait(s.drain, 0, kDrainNs);
+        umma_commit(&s.drain[mi]);
+        drain_wait(&s.drain[mi], 0, kDrainNs);
       }
     }
   } else {
@@ -539,14 +552,16 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     const int mb = k_MB == 2 ? wg : 0;
     const int istep = k_MB == 2 ? 1 : 2;
     const int r = mb * 128 + quad * 32 + lane;   // row of the item
-    float* ep_w = s.ep + ew * (3 * k_N + 16);
+    const bool has_beta = k_beta != nullptr;
+    // per-warp parameters: folded weights; with a bias also the query scales
+    // and the bias terms; then the valid lengths of the group's queries
+    float* ep_w = s.ep + ew * a.ep_stride;
     float* ep_qs = ep_w + k_N;
     float* ep_beta = ep_qs + k_N;
-    int* ep_len = reinterpret_cast<int*>(ep_beta + k_N);
-    const bool has_beta = k_beta != nullptr;
+    int* ep_len = reinterpret_cast<int*>(ep_w + (has_beta ? 3 * k_N : k_N));
     Ring acc, ms;
     const uint32_t first_item = k_MB == 2 ? 0u : static_cast<uint32_t>(wg);
-    acc.i = first_item;                      // n_acc, kMetaSlots >= 2
+    acc.i = first_item;                      // n_acc, n_meta >= 2
     ms.i = first_item;
     SegWalk w{s.prefix, n_groups};
     bool first = true;
@@ -574,8 +589,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
             // Without a bias, fold the query scale into the weight (ReLU is
             // positively homogeneous and the scales are positive).
             ep_w[i0 + h] = has_beta ? wv : wv * qs;
-            ep_qs[i0 + h] = qs;
-            ep_beta[i0 + h] = be;
+            if (has_beta) {
+              ep_qs[i0 + h] = qs;
+              ep_beta[i0 + h] = be;
+            }
           }
         }
         if (lane < 16) {
@@ -606,7 +623,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (GATHER) tok = reinterpret_cast<const int*>(mscale + k_R)[r];
         if (e4 && tok >= 0) cs = mscale[r];    // rows past the valid prefix read a stale value, unused
       }
-      if (!bounded_wait(&s.accfull[acc.i], acc.ph, wc)) break;
+      if (!bounded_wait(&s.accfull[2 * acc.i + mb], acc.ph, wc)) break;
       if (lane == 0 && (ew & 3) == 0) trace_event(k_trace, lt, 4);
       tc_fence_after();
 
@@ -653,11 +670,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) {
         if ((ew & 3) == 0) trace_event(k_trace, lt, 5);
-        mbar_arrive(&s.accempty[acc.i]);
+        mbar_arrive(&s.accempty[2 * acc.i + mb]);
         if (has_meta) mbar_arrive(&s.mempty[ms.i]);
       }
       acc.step_by(static_cast<uint32_t>(istep), NA);
-      if (has_meta) ms.step_by(static_cast<uint32_t>(istep), kMetaSlots);
+      if (has_meta) ms.step_by(static_cast<uint32_t>(istep), NM);
     }
   }
 
