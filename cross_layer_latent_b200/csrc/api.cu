@@ -240,7 +240,16 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   memset(&a, 0, sizeof(a));
   const int eb = elt_bytes(c->dtype);
   const int64_t row_bytes = static_cast<int64_t>(c->dim) * eb;
-  const int swz = row_bytes % 128 == 0 ? 128 : (row_bytes % 64 == 0 ? 64 : 32);
+  int swz = row_bytes % 128 == 0 ? 128 : (row_bytes % 64 == 0 ? 64 : 32);
+  int n_kchunks = static_cast<int>(row_bytes / swz);
+  if (gather && swz < 128 && row_bytes > 128) {
+    // Row gathers are bound by the number of TMA operations, so gather whole
+    // 128-byte chunks: K is padded to a multiple of 128 bytes, and the bytes
+    // past the row's end lie outside both tensor maps and arrive as zeros
+    // (cache and queries alike), which adds exact zeros to every product.
+    swz = 128;
+    n_kchunks = static_cast<int>((row_bytes + 127) / 128);
+  }
   const int H_pad = (q->H + 15) / 16 * 16;
   const int Qg = gather ? 1 : std::max(1, std::min(256 / H_pad, q->T));
   const int N = Qg * H_pad;
@@ -260,7 +269,7 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   a.n_segments = n_seg;
   a.swz = swz;
   a.elt_bytes = eb;
-  a.n_kchunks = static_cast<int>(row_bytes / swz);
+  a.n_kchunks = n_kchunks;
   a.row_bytes = row_bytes;
   a.cand_stride = cand_stride;
   const int kind = c->dtype == LI_F32 ? kKindTF32 : (c->dtype == LI_BF16 ? kKindBF16 : kKindE4M3);
