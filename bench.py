@@ -48,6 +48,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-other-contexts", action="store_true")
+    p.add_argument("--no-prefill", action="store_true")
     return p.parse_args()
 
 
@@ -407,6 +408,56 @@ def profiled_steps(step, steps, flush, stream, lead_ms=4.0):
     return recs, hs_ms, dsa_ms
 
 
+def prefill_leg(li, ctx, args, rank, dev):
+    """Full LatentIndex scoring and per-query top-k for the prefill chunk:
+    each layer's call is timed with CUDA events, and the scan kernel alone
+    from the launch profile; FLOPs = 2 * H * d_c per (query, valid position)."""
+    wl = workload(4)
+    inp = generate(wl, seed=wl.seed + 1000 * rank)
+    g = li.GroupIndexer(ctx, batch=wl.batch, capacity=wl.capacity, d_c=wl.d_c, H=wl.heads, d_k=wl.d_k,
+                        G=wl.group, dtype=li.LI_BF16, k=wl.k, B=0, T=wl.queries, dsa=False, device=dev)
+    g.load(inp.lengths, inp.W_K, inp.q, inp.w, latent=inp.latent, q_pos=inp.q_pos, dsa_keys=False)
+    pairs = int(sum(min(int(inp.lengths[b]), int(p) + 1) for b in range(wl.batch) for p in inp.q_pos[b]))
+    flop = 2.0 * wl.heads * wl.d_c * pairs
+    for l in range(wl.group):
+        g.score_topk(l)
+    torch.cuda.synchronize()
+    li.li_profile_reset(ctx)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(wl.group)]
+    li.li_profile_enable(ctx, True)
+    for l in range(wl.group):
+        ev[l][0].record()
+        g.score_topk(l)
+        ev[l][1].record()
+    li.li_profile_enable(ctx, False)
+    torch.cuda.synchronize()
+    recs = li.li_profile_read(ctx)
+    li.li_profile_reset(ctx)
+    st = li.li_device_status(ctx, g.ws)
+    if st != "LI_OK":
+        raise RuntimeError(f"device status after the prefill leg: {st}")
+    call_ms = [a.elapsed_time(b) for a, b in ev]
+    scan_ms = [r["ms"] for r in recs if r["kernel"] == "scan"]
+    sel_ms = [r["ms"] for r in recs if r["kernel"].startswith("topk")]
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    scan_tflops = flop / (statistics.mean(scan_ms) / 1e3) / 1e12 if scan_ms else None
+    return {"workload": f"{wl.name}: {wl.queries} queries at positions {int(inp.q_pos.min())}..{int(inp.q_pos.max())}"
+                        f" of a {wl.capacity}-position bf16 prefix, H {wl.heads}, d_c {wl.d_c}, k {wl.k}",
+            "pairs_per_layer": pairs, "tflop_per_layer": flop / 1e12,
+            "layer_ms": statistics.mean(call_ms), "scan_ms": statistics.mean(scan_ms) if scan_ms else None,
+            "select_ms": sum(sel_ms) / max(len(call_ms), 1),
+            "roofline": {"bound": "tensor", "achieved": scan_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": (scan_tflops / peak) if scan_tflops else None,
+                         "peak_source": "measured cuBLAS bf16 GEMM, sustained (MEASURED_PEAKS.json)"},
+            "keys_per_s": wl.group * pairs / (sum(call_ms) / 1e3)}
+
+
 def max_over_ranks(x, dist, dev):
     """The slowest rank's value (every rank gets it)."""
     t = torch.tensor([x], device=dev, dtype=torch.float64)
@@ -605,6 +656,11 @@ def main():
             del s2
             torch.cuda.empty_cache()
         out["paths"]["other_contexts"] = other
+
+    # ---- prefill-chunk scoring (the tensor-bound contraction): 1024 queries
+    #      against their causal prefix of 65536 positions, per layer
+    if not args.no_prefill:
+        out["prefill"] = prefill_leg(li, ctx, args, rank, dev)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, step.hnew, step.Wd, step.Wk)
