@@ -451,7 +451,11 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   t.cand = at<uint2>(ws, L.cand);
   if (static_cast<int64_t>(t.rows) * t.n > static_cast<int64_t>((L.scores - L.cand) / 8))
     return fail(ctx, LI_ERR_WORKSPACE, "selection of %d x %d exceeds the workspace candidate buffer", t.rows, t.n);
-  if (t.n <= kClusterMaxN && t.rows <= 65535) {
+  // The cluster kernel minimises latency for a few rows; once its CTAs
+  // (rows x cluster size) exceed about one wave, the chunked path, which
+  // spreads every row over many small blocks, has the better throughput.
+  const int64_t cs = std::min<int64_t>(kClusterMaxSize, std::max<int64_t>(1, (t.n + 8191) / 8192));
+  if (t.n <= kClusterMaxN && static_cast<int64_t>(t.rows) * cs <= 2 * static_cast<int64_t>(ctx->num_sms)) {
     int cs = 0;
     Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);
     const cudaError_t e = launch_topk_cluster(t, st, &cs);
