@@ -385,7 +385,17 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   a.q_scale = q->dtype == LI_E4M3 ? q->q_scale : nullptr;
   a.beta = q->beta;
   P->kind = kind;
-  const int64_t tiles_per_seg = (static_cast<int64_t>(gather ? cand_stride : c->capacity) + a.R - 1) / a.R;
+  a.RI = a.R;
+  if (gather) {
+    // gathered rows per item: the largest of 128 / 64 / 32 that still gives
+    // every SM an item (the gather is bound by TMA operations per SM; the
+    // MMA block stays 128 rows, the rows past RI are neither gathered nor
+    // stored)
+    a.RI = 32;
+    for (int ri = a.R; ri >= 32; ri >>= 1)
+      if (static_cast<int64_t>(n_seg) * ((cand_stride + ri - 1) / ri) >= ctx->num_sms) { a.RI = ri; break; }
+  }
+  const int64_t tiles_per_seg = (static_cast<int64_t>(gather ? cand_stride : c->capacity) + a.RI - 1) / a.RI;
   P->grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ctx->num_sms, n_seg * tiles_per_seg)));
   return LI_OK;
 }

@@ -44,6 +44,7 @@ struct alignas(64) ScanArgs {
   int cand_stride;
   int swz, n_kchunks, elt_bytes;
   int R, MB;                  // rows per work item (128 or 256) and M=128 blocks per item
+  int RI;                     // gather: candidate rows gathered per item (32, 64 or 128 <= R)
   int KS, stages_per_item;    // K-chunks per stage, stages per item
   int n_stages, n_bslots, n_acc, n_meta;
   int ep_stride;              // floats of epilogue parameters per epilogue warp

@@ -91,7 +91,7 @@ __device__ __forceinline__ int segment_items(const ScanArgs& a, int seg) {
   if (GATHER) {
     int n = a.cand_n[seg];
     n = n < 0 ? 0 : (n > a.cand_stride ? a.cand_stride : n);
-    return (n + a.R - 1) / a.R;
+    return (n + a.RI - 1) / a.RI;
   }
   const int b = seg / a.n_groups, g = seg % a.n_groups;
   int len = a.lengths[b];
@@ -298,6 +298,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const int k_capacity = a.capacity, k_T = a.T, k_H = a.H, k_H_pad = a.H_pad, k_Qg = a.Qg, k_N = a.N;
   const int k_cand_stride = a.cand_stride, k_swz = a.swz, k_n_kchunks = a.n_kchunks;
   const int k_R = a.R, k_MB = a.MB, k_KS = a.KS, k_spi = a.stages_per_item;
+  const int k_RI = GATHER ? a.RI : a.R;      // rows an item covers (gather: fewer than the M block)
   const uint32_t k_a_stage_bytes = a.a_stage_bytes, k_b_slot_bytes = a.b_slot_bytes, k_idesc = a.idesc;
   const uint32_t k_meta_bytes = a.meta_bytes;
   const int64_t k_score_stride = a.score_stride;
@@ -397,7 +398,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     constexpr int kIdsPerLane = kMaxItemRows / 32;
     uint32_t n_st = 0, n_bs = 0;
     const int rows_per_lane = k_R >> 5;
-    const int groups = k_R >> 2;                   // 4-row gathers per K-chunk
+    const int groups = k_RI >> 2;                  // 4-row gathers per K-chunk
+    const uint32_t stage_tx = static_cast<uint32_t>(k_RI * k_swz * k_KS);   // bytes gathered per stage
     Ring st, bs, ms;
     SegWalk w{s.prefix, n_groups};
     SegWalk wn{s.prefix, n_groups};                // one item ahead
@@ -409,8 +411,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
 #pragma unroll
       for (int i = 0; i < kIdsPerLane; ++i) {
         out[i] = -1;
-        const int j = itn * k_R + lane + 32 * i;
-        if (i < rows_per_lane && j < k_cand_stride) out[i] = k_cand[static_cast<int64_t>(sg) * k_cand_stride + j];
+        const int r = lane + 32 * i;
+        const int j = itn * k_RI + r;
+        if (i < rows_per_lane && r < k_RI && j < k_cand_stride)
+          out[i] = k_cand[static_cast<int64_t>(sg) * k_cand_stride + j];
       }
     };
     if (begin < end) fetch_ids(begin, wn, ids);
@@ -444,8 +448,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       for (int i = 0; i < kIdsPerLane; ++i) {
         if (i < rows_per_lane) {
           const int r = lane + 32 * i;
-          const int j = it * k_R + r;
-          int t = j < cn ? cur[i] : -1;
+          const int j = it * k_RI + r;
+          int t = (r < k_RI && j < cn) ? cur[i] : -1;
           if (j < cn && (t < 0 || t >= len)) t = -2;     // invalid candidate
           mtok[r] = t;
           if (e4) cp_async_4_zfill(smem_addr(mscale + r), k_cache_scale + seq_row + (t >= 0 ? t : 0), t >= 0 ? 4 : 0);
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       bool ok = true;
       for (int sp = 0; sp < k_spi; ++sp) {
         if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(&s.full[st.i], k_a_stage_bytes);
+        if (lane == 0) mbar_arrive_expect_tx(&s.full[st.i], stage_tx);
         __syncwarp();
         const uint32_t stage = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
         for (int u = lane; u < groups * k_KS; u += 32) {
@@ -614,7 +618,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         }
         __syncwarp();
       }
-      const int j = it * k_R + r;           // position (scan) or candidate slot (gather)
+      const int j = it * k_RI + r;          // position (scan) or candidate slot (gather)
+      const bool row_in_item = !GATHER || r < k_RI;
       int tok = j;
       float cs = 1.f;
       if (has_meta) {
@@ -657,7 +662,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (qi == 0 && lane == 0 && (ew & 3) == 0) trace_event(k_trace, lt, 7);
         float sc = (part[0] + part[1]) + (part[2] + part[3]);
         if (!has_beta && e4) sc *= cs;
-        if (j < ep_len[qi]) {
+        if (row_in_item && j < ep_len[qi]) {
           if (GATHER && tok < 0) {
             sc = -INFINITY;
             record_status(k_status, kStatusIndex);
