@@ -60,6 +60,29 @@ struct ProfRec {
   int grid, block, smem;
 };
 
+struct ScanPlan {
+  ScanArgs a;
+  int kind;
+  int grid;
+};
+
+// Everything a scan plan depends on (zero-filled, compared bytewise).
+struct PlanKey {
+  const void* data;
+  const float* scale;
+  const int32_t* lengths;
+  const void* q;
+  const float* q_scale;
+  const float* beta;
+  const float* w;
+  const int32_t* q_pos;
+  const uint64_t* trace;
+  uint64_t wait_ns;
+  int32_t batch, capacity, dim, dtype;
+  int32_t q_dtype, T, H, gather;
+  int32_t cand_stride, pad;
+};
+
 struct li_ctx {
   int device = 0;
   int num_sms = 0;
@@ -71,6 +94,13 @@ struct li_ctx {
   uint64_t* trace = nullptr;
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> free_events;
+  // Recently built scan plans (tensor maps included): a decode loop calls
+  // the same entry points on the same buffers every step.
+  static constexpr int kPlanCache = 16;
+  PlanKey plan_key[kPlanCache] = {};
+  ScanPlan plan_val[kPlanCache];
+  bool plan_used[kPlanCache] = {};
+  int plan_next = 0;
 };
 
 namespace {
@@ -228,14 +258,52 @@ li_status encode_map(li_ctx* ctx, CUtensorMap* m, li_dtype dt, int rank, void* b
 
 // ------------------------------------------------------------------ scan plan
 
-struct ScanPlan {
-  ScanArgs a;
-  int kind;
-  int grid;
-};
 
+li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, bool gather, int cand_stride,
+                          ScanPlan* P, const char* what);
+
+// The plan of a scan launch, from the context's cache when the same buffers
+// and shapes were planned before (the tensor maps hold the buffer addresses).
 li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gather, int cand_stride,
                     ScanPlan* P, const char* what) {
+  PlanKey k;
+  memset(&k, 0, sizeof(k));
+  k.data = c->data;
+  k.scale = c->scale;
+  k.lengths = c->lengths;
+  k.q = q->q;
+  k.q_scale = q->q_scale;
+  k.beta = q->beta;
+  k.w = q->w;
+  k.q_pos = q->q_pos;
+  k.trace = ctx->trace;
+  k.wait_ns = ctx->wait_ns;
+  k.batch = c->batch;
+  k.capacity = c->capacity;
+  k.dim = c->dim;
+  k.dtype = static_cast<int32_t>(c->dtype);
+  k.q_dtype = static_cast<int32_t>(q->dtype);
+  k.T = q->T;
+  k.H = q->H;
+  k.gather = gather ? 1 : 0;
+  k.cand_stride = cand_stride;
+  for (int i = 0; i < li_ctx::kPlanCache; ++i)
+    if (ctx->plan_used[i] && memcmp(&ctx->plan_key[i], &k, sizeof(k)) == 0) {
+      *P = ctx->plan_val[i];
+      return LI_OK;
+    }
+  li_status s = plan_scan_build(ctx, c, q, gather, cand_stride, P, what);
+  if (s != LI_OK) return s;
+  const int slot = ctx->plan_next;
+  ctx->plan_next = (slot + 1) % li_ctx::kPlanCache;
+  ctx->plan_key[slot] = k;
+  ctx->plan_val[slot] = *P;
+  ctx->plan_used[slot] = true;
+  return LI_OK;
+}
+
+li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, bool gather, int cand_stride,
+                          ScanPlan* P, const char* what) {
   ScanArgs& a = P->a;
   memset(&a, 0, sizeof(a));
   const int eb = elt_bytes(c->dtype);
