@@ -128,9 +128,11 @@ __device__ __forceinline__ void write_row(const float (&v)[8], float amax, int l
 // output over the splits in order.  Used when the partials fit in the
 // block's shared memory.
 constexpr int kFuseMaxPartials = 16384;   // floats of partial sums (64 KB)
+constexpr int kAppendWarps = 16;          // 512-thread blocks: few arrivals on the completion counter
+constexpr int kStagePer = kFuseMaxPartials / (kAppendWarps * 32);   // partial sums each thread stages
 
 template <typename T>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* __restrict__ h,
+__global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T* __restrict__ h,
                                                                       const T* __restrict__ W, int d_model,
                                                                       int dim, int n_tok, int splits,
                                                                       float* __restrict__ part, int batch, int T_tok,
@@ -141,9 +143,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* _
   extern __shared__ __align__(16) float ps[];       // [splits][n_tok * dim], then cs [n_tok * dim]
   __shared__ unsigned last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int task = blockIdx.x * kGemvWarps + warp;
-  if (task < dim * splits) {
-    const int j = task / splits, sp = task % splits;
+  // block b takes split b % splits for kAppendWarps consecutive outputs, so
+  // its warps share one slice of the hidden states (read once, then from L1)
+  const int sp = static_cast<int>(blockIdx.x) % splits;
+  const int j = (static_cast<int>(blockIdx.x) / splits) * kAppendWarps + warp;
+  if (j < dim) {
     const int len = d_model / splits;
     const int i0 = sp * len, i1 = i0 + len;
     float acc[kGemvTok];
@@ -180,17 +184,18 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* _
   __syncthreads();
   if (!last) return;
   __threadfence();
-  const int nx = n_tok * dim, np = splits * nx;
-  for (int base = threadIdx.x; base < np; base += blockDim.x * 8) {
-    float v[8];
+  const int nx = n_tok * dim, np = splits * nx;   // np <= kStagePer * blockDim.x
+  {
+    // every partial sum in flight at once
+    float v[kStagePer];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const int idx = base + m * static_cast<int>(blockDim.x);
+    for (int m = 0; m < kStagePer; ++m) {
+      const int idx = static_cast<int>(threadIdx.x) + m * kAppendWarps * 32;
       v[m] = idx < np ? __ldcg(part + idx) : 0.f;
     }
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const int idx = base + m * static_cast<int>(blockDim.x);
+    for (int m = 0; m < kStagePer; ++m) {
+      const int idx = static_cast<int>(threadIdx.x) + m * kAppendWarps * 32;
       if (idx < np) ps[idx] = v[m];
     }
   }
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_append_kernel(const T* _
     cs[x] = sum;
   }
   __syncthreads();
-  for (int m = warp; m < n_tok; m += kGemvWarps) {
+  for (int m = warp; m < n_tok; m += kAppendWarps) {
     const int b = m / T_tok, t = m % T_tok;
     const int len = lengths[b];
     if (len < 0 || len + T_tok > capacity) {
@@ -522,19 +527,19 @@ cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d
                                 int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
                                 int dtype, unsigned int* done, int* status, cudaStream_t st) {
   const int n_tok = batch * T;
-  const int grid = (dim * splits + kGemvWarps - 1) / kGemvWarps;
+  const int grid = splits * ((dim + kAppendWarps - 1) / kAppendWarps);
   const size_t smem = static_cast<size_t>(splits + 1) * n_tok * dim * sizeof(float);
   cudaError_t e;
   if (h_dtype == LI_BF16) {
     auto k = gemv_append_kernel<__nv_bfloat16>;
     if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
-    return launch_pdl(k, dim3(grid), dim3(kGemvWarps * 32), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(h),
+    return launch_pdl(k, dim3(grid), dim3(kAppendWarps * 32), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(h),
                       reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim, n_tok, splits, part, batch, T, data,
                       scale, lengths, capacity, dtype, done, status);
   } else {
     auto k = gemv_append_kernel<float>;
     if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
-    return launch_pdl(k, dim3(grid), dim3(kGemvWarps * 32), smem, st, 1, reinterpret_cast<const float*>(h),
+    return launch_pdl(k, dim3(grid), dim3(kAppendWarps * 32), smem, st, 1, reinterpret_cast<const float*>(h),
                       reinterpret_cast<const float*>(W), d_model, dim, n_tok, splits, part, batch, T, data, scale,
                       lengths, capacity, dtype, done, status);
   }
