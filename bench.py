@@ -49,6 +49,7 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-other-contexts", action="store_true")
     p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--no-fused", action="store_true")
     return p.parse_args()
 
 
@@ -491,6 +492,54 @@ def prefill_leg(li, ctx, args, rank, dev):
             "keys_per_s": wl.group * pairs / (sum(call_ms) / 1e3)}
 
 
+def fused_leg(step, args, flush, stream, dist, dev, world):
+    """Scoring + selection of all G layers over the full prefix: G per-layer
+    scans of the shared latent, against one scan with the G layers' absorbed
+    queries stacked (G * H MMA columns; queries from the anchor's hidden state
+    in the training-aware instantiation).  Both from captured graphs, L2
+    flushed before each, CUDA events on the stream."""
+    g, wl = step.g, step.wl
+    step.reset()
+    step.hs_path()                       # absorbed queries of every layer
+    torch.cuda.synchronize()
+
+    def per_layer():
+        for l in range(wl.group):
+            g.score_topk(l)
+
+    graphs = []
+    for fn in (per_layer, g.fused_group_score_topk):
+        fn()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        graphs.append(gr)
+    times = []
+    for gr in graphs:
+        for _ in range(args.warmup):
+            gr.replay()
+        ms = []
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        times.append(max_over_ranks(statistics.mean(ms), dist, dev))
+    del graphs
+    keys = wl.group * int(sum(int(n) for n in step.inp.lengths))
+    lat_bytes = int(sum(int(n) for n in step.inp.lengths)) * row_bytes(wl, wl.d_c)
+    return {"per_layer_ms": times[0], "fused_ms": times[1], "fused_speedup": times[0] / times[1],
+            "keys_per_step": keys, "per_layer_keys_per_s": world * keys / (times[0] / 1e3),
+            "fused_keys_per_s": world * keys / (times[1] / 1e3),
+            "fused_latent_gb_per_s": lat_bytes / (times[1] / 1e3) / 1e9,
+            "mode": f"{wl.group} layers x (scan + top-{wl.k}) of {wl.batch} sequences; fused: one scan, "
+                    f"{wl.group} x {wl.heads} MMA columns"}
+
+
 def max_over_ranks(x, dist, dev):
     """The slowest rank's value (every rank gets it)."""
     t = torch.tensor([x], device=dev, dtype=torch.float64)
@@ -663,6 +712,11 @@ def main():
                       "eager_value": whole_job_rate(world, keys, args.steps, te_eager),
                       "eager_ms_per_step": te_eager / args.steps,
                       "eager_mode": "the same with every library call issued eagerly"}
+
+    # ---- full LatentIndex for the whole group: 4 per-layer scans of the shared
+    #      latent against one fused scan with the 4 layers' queries stacked
+    if not args.no_fused:
+        out["paths"]["full_latentindex"] = fused_leg(step, args, flush, stream, dist, dev, world)
 
     # ---- HS against DSA-style at the shorter contexts (same library, same protocol)
     if not args.no_other_contexts:

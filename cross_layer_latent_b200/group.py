@@ -42,12 +42,17 @@ class GroupIndexer:
         dev, tdt = self.device, TORCH_DTYPE[dtype]
         self.latent = _cache(batch, capacity, d_c, dtype, dev)
         self.keys: List[Cache] = [_cache(batch, capacity, d_k, dtype, dev) for _ in range(G)] if dsa else []
-        self.q_abs = [torch.zeros(batch, T, H, d_c, dtype=tdt, device=dev) for _ in range(G)]
-        self.q_raw = [torch.zeros(batch, T, H, d_k, dtype=tdt, device=dev) for _ in range(G)] if dsa else []
+        # layer-major storage: layer l's queries are the contiguous slice [l],
+        # and the fused group scan restacks all layers with one copy each
         e4 = dtype == LI_E4M3
-        self.q_abs_scale = [torch.ones(batch, T, H, device=dev) if e4 else None for _ in range(G)]
+        self.q_abs_all = torch.zeros(G, batch, T, H, d_c, dtype=tdt, device=dev)
+        self.q_abs_scale_all = torch.ones(G, batch, T, H, device=dev) if e4 else None
+        self.w_all = torch.zeros(G, batch, T, H, device=dev)
+        self.q_abs = list(self.q_abs_all.unbind(0))
+        self.q_abs_scale = list(self.q_abs_scale_all.unbind(0)) if e4 else [None] * G
+        self.w = list(self.w_all.unbind(0))
+        self.q_raw = [torch.zeros(batch, T, H, d_k, dtype=tdt, device=dev) for _ in range(G)] if dsa else []
         self.q_raw_scale = [torch.ones(batch, T, H, device=dev) if e4 else None for _ in range(G)] if dsa else []
-        self.w = [torch.zeros(batch, T, H, device=dev) for _ in range(G)]
         self.beta: List[Optional[torch.Tensor]] = [None] * G
         self.q_pos: Optional[torch.Tensor] = None
         self.idx = [torch.full((batch, T, k), -1, dtype=torch.int32, device=dev) for _ in range(G)]
@@ -134,6 +139,35 @@ class GroupIndexer:
         li_score_topk(self.ctx, self.latent, self.query(layer), self.k, self.idx[layer], self.score[layer], dump,
                       self.ws, stream)
         return self.idx[layer]
+
+    def fused_group_score_topk(self, dump: Optional[torch.Tensor] = None, stream=None):
+        """Full LatentIndex for all G layers of a decode token with one pass
+        over the shared latent: the layers' absorbed queries are stacked as G
+        query rows of each sequence (training-aware instantiation, Sec. D.2:
+        every layer's query comes from the anchor's hidden state, so all exist
+        at once).  The scan takes up to 256 // H of them per MMA (G * H columns
+        at G = 4, H = 64: one read of the latent for the whole group).
+        Selections land in idx_group [batch, G, k]; dump, if given, is
+        [batch, G, capacity]."""
+        if self.T != 1:
+            raise ValueError("the fused group scan stacks decode queries (T = 1)")
+        if not hasattr(self, "q_group"):
+            dev, G, b = self.device, self.G, self.batch
+            self.q_group = torch.empty_like(self.q_abs_all[:, :, 0].transpose(0, 1).contiguous())
+            self.q_group_scale = (torch.empty(b, G, self.H, device=dev)
+                                  if self.q_abs_scale_all is not None else None)
+            self.w_group = torch.empty(b, G, self.H, device=dev)
+            self.idx_group = torch.full((b, G, self.k), -1, dtype=torch.int32, device=dev)
+            self.score_group = torch.zeros(b, G, self.k, device=dev)
+            self.ws_group = workspace(self.ctx, b, G, self.capacity, self.H, self.k, 0, device=dev)
+        # layer-major [G, b, H, ...] to sequence-major [b, G, H, ...]: one copy per array
+        self.q_group.copy_(self.q_abs_all[:, :, 0].transpose(0, 1))
+        self.w_group.copy_(self.w_all[:, :, 0].transpose(0, 1))
+        if self.q_group_scale is not None:
+            self.q_group_scale.copy_(self.q_abs_scale_all[:, :, 0].transpose(0, 1))
+        q = Query(q=self.q_group, w=self.w_group, q_scale=self.q_group_scale, beta=None, q_pos=None, dtype=self.dtype)
+        li_score_topk(self.ctx, self.latent, q, self.k, self.idx_group, self.score_group, dump, self.ws_group, stream)
+        return self.idx_group
 
     def hs_anchor(self, layer: int = 0, dump: Optional[torch.Tensor] = None, stream=None):
         li_hs_anchor_candidates(self.ctx, self.latent, self.query(layer), self.B, self.k, self.cand, self.cand_n,

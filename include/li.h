@@ -200,7 +200,14 @@ LI_API li_status li_absorb_query(li_ctx* ctx, const void* q, li_dtype q_dtype, i
  * out_idx   [batch][T][k] int32 (see "Selections").
  * out_score [batch][T][k] fp32 selected scores, or NULL.
  * scores_dump [batch][T][capacity] fp32, or NULL: receives every valid score
- *           (positions past the valid prefix are not written).            */
+ *           (positions past the valid prefix are not written).
+ * The T query rows of a sequence share every read of the cache: up to
+ * 256 / H of them go into one MMA.  Stacking the G layers' absorbed decode
+ * queries of a group as T = G rows (possible when all of them exist at
+ * once, as in the training-aware instantiation of Sec. D.2, where every
+ * layer's query comes from the anchor's hidden state) scores the whole
+ * group with one pass over the latent; each row's scores and selection are
+ * the same as with that row alone.                                        */
 LI_API li_status li_score_topk(li_ctx* ctx, const li_cache* cache, const li_query* q, int k,
                         int32_t* out_idx, float* out_score, float* scores_dump, void* ws,
                         size_t ws_bytes, void* stream);
