@@ -15,10 +15,14 @@ printed in the summary (tests/golden/printed_numbers.json), an independent
 pure-Python brute force that reconstructs every key explicitly, the method's
 invariants (absorption exactness, HS with B >= L equals full selection, a
 one-layer group with an identity decoder is DSA-style scoring), and the
-codecs against torch's bf16 / float8_e4m3fn conversions.  The pages print no
+codecs against torch's bf16 / float8_e4m3fn conversions.  The two-branch
+latent (rope.py: rotary rotation, LayerNorm, native rotated keys) is pinned
+by plane geometry, the rotation group laws, torch's float64 layer_norm and
+the exactness of absorbing frequency-wise complex decoders into post-RoPE
+queries (tests/test_oracle_rope.py).  The pages print no
 score values of their own, so the score arithmetic is pinned by hand
 arithmetic and brute force rather than by a published example.
 """
-from . import codecs, counters, indexer, bruteforce
+from . import codecs, counters, indexer, bruteforce, rope
 
-__all__ = ["codecs", "counters", "indexer", "bruteforce"]
+__all__ = ["codecs", "counters", "indexer", "bruteforce", "rope"]

@@ -53,3 +53,35 @@ def assert_selection_close(gpu_idx, ref_scores, M, k, n, rtol, what=""):
     assert len(bad) == 0, (f"{what}: {len(bad)} of {len(diff)} differing positions are not near the boundary; "
                            f"first {bad[:5]}, gap {gap[gap > tol][:5]}, tol {tol[gap > tol][:5]}")
     return len(diff)
+
+
+# ------------------------------------------------------------------ two-branch (RoPE + NoPE) latent
+
+def latent_format(ri):
+    """The oracle's LatentFormat for generated RopeInputs."""
+    from oracle.rope import LatentFormat
+    return LatentFormat(rope_offset=ri.rope_offset, rope_dim=ri.rope_dim, sources=ri.sources,
+                        inv_freq=ri.inv_freq, norm_offset=ri.norm_offset, norm_dim=ri.norm_dim,
+                        gamma=ri.gamma, beta=ri.beta, eps=ri.eps)
+
+
+def rope_decoder_matrix(ri, layer: int, d_k: int, d_c: int):
+    """Layer `layer`'s decoder as one real matrix W [d_k, d_c] (key = W c) plus
+    its bias [d_k], the form the absorption entry point takes.  Native key
+    slot f (reals 2f, 2f+1) gets sum_j d[f, j] * latent slot (f, j): the
+    complex product (a + ib)(x + iy) is the real block [[a, -b], [b, a]]
+    acting on (x, y).  The NoPE rows take W_nope on the NoPE columns."""
+    F, r = ri.d_re[layer].shape
+    W = np.zeros((d_k, d_c), np.float32)
+    for f in range(F):
+        for j in range(r):
+            a, b = ri.d_re[layer][f, j], ri.d_im[layer][f, j]
+            col = ri.rope_offset + 2 * (f * r + j)
+            W[2 * f, col], W[2 * f, col + 1] = a, -b
+            W[2 * f + 1, col], W[2 * f + 1, col + 1] = b, a
+    d_nope = d_k - 2 * F
+    W[2 * F:, ri.norm_offset:ri.norm_offset + ri.norm_dim] = ri.W_nope[layer]
+    bias = np.zeros(d_k, np.float32)
+    bias[2 * F:] = ri.b_nope[layer]
+    assert ri.W_nope[layer].shape == (d_nope, ri.norm_dim)
+    return W, bias

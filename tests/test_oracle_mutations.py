@@ -77,3 +77,54 @@ def test_planted_mistake_is_caught(monkeypatch, name, attr, bad):
         except AssertionError:
             failures += 1
     assert failures > 0, f"no pin caught: {name}"
+
+
+# ------------------------------------------------------------------ two-branch latent (oracle/rope.py)
+
+import oracle.rope as rp  # noqa: E402
+from tests import test_oracle_rope as rope_pins  # noqa: E402
+
+_rotate = rp.rotate
+
+
+def _rotate_wrong_sign(x, pos, inv_freq, sources=1):
+    return _rotate(x, -np.asarray(pos), inv_freq, sources)
+
+
+def _rotate_slot_frequency(x, pos, inv_freq, sources=1):
+    # a slip: slot p takes frequency p instead of p // sources
+    z = rp.as_slots(x)
+    P = z.shape[-1]
+    freq = np.resize(np.asarray(inv_freq, float), P)
+    pos = np.asarray(pos, float)
+    angle = pos[..., None] * freq if pos.ndim else pos * freq
+    return rp.from_slots(z * np.exp(1j * angle))
+
+
+def _layer_norm_unbiased(x, gamma=None, beta=None, eps=1e-6):
+    x = np.asarray(x, float)
+    y = (x - x.mean(axis=-1, keepdims=True)) / np.sqrt(x.var(axis=-1, ddof=1, keepdims=True) + eps)
+    if gamma is not None:
+        y = y * gamma
+    return y if beta is None else y + beta
+
+
+ROPE_PINS = [rope_pins.test_quarter_turn_of_a_unit_pair, rope_pins.test_rotation_laws,
+             rope_pins.test_sources_of_one_frequency_share_its_phase, rope_pins.test_layer_norm_matches_torch,
+             lambda: rope_pins.test_absorbed_scoring_of_rotated_latent_equals_native_rotated_keys(2)]
+
+
+@pytest.mark.parametrize("name,attr,bad", [
+    ("rotation the wrong way", "rotate", _rotate_wrong_sign),
+    ("slot frequency ignores the sources", "rotate", _rotate_slot_frequency),
+    ("LayerNorm with the unbiased variance", "layer_norm", _layer_norm_unbiased),
+])
+def test_planted_rope_mistake_is_caught(monkeypatch, name, attr, bad):
+    monkeypatch.setattr(rp, attr, bad)
+    failures = 0
+    for pin in ROPE_PINS:
+        try:
+            pin()
+        except AssertionError:
+            failures += 1
+    assert failures > 0, f"no pin caught: {name}"

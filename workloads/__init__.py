@@ -3,7 +3,7 @@
 Data synthesis only; none of the indexer's arithmetic lives here.
 """
 from .configs import WORKLOADS, Workload, workload
-from .gen import Inputs, generate, shrunk, construction_inputs
+from .gen import Inputs, RopeInputs, construction_inputs, generate, rope_inputs, shrunk
 
 __all__ = ["WORKLOADS", "Workload", "workload", "Inputs", "generate", "shrunk",
-           "construction_inputs"]
+           "construction_inputs", "RopeInputs", "rope_inputs"]

@@ -137,3 +137,53 @@ def construction_inputs(wl: Workload, seed: Optional[int] = None):
     W_k = [(rng.standard_normal((wl.d_k, wl.d_model), dtype=np.float32) * s)
            for _ in range(wl.group)]
     return h_new.astype(np.float32), W_down.astype(np.float32), [x.astype(np.float32) for x in W_k]
+
+
+@dataclass
+class RopeInputs:
+    """Parameters of a two-branch (RoPE + NoPE) latent and of layer decoders
+    that are frequency-wise complex on the rotary branch.
+
+    Layout (this build's reading of "RoPE64/NoPE128"): the latent row is
+    [rotary rope_dim | NoPE norm_dim]; a layer's native key is
+    [rotary 2F | NoPE d_k - 2F] with F = rope_dim / (2 sources) frequencies.
+    Recipe: inv_freq[f] = base^(-f / F) with base 10000 (float32); LayerNorm
+    gamma = 1 + 0.1 N(0, 1), beta = 0.1 N(0, 1), eps 1e-6; complex decoder
+    coefficients d[l][f, j] with real and imaginary parts
+    N(0, sqrt(d_model / (2 sources))) (std), which gives rotary key
+    components of unit variance from latents of std 1/sqrt(d_model); NoPE
+    decoders W_nope[l] ~ N(0, 1/sqrt(norm_dim)), biases b_nope[l] ~ 0.1 N(0, 1).
+    The queries of the workload serve as post-RoPE queries."""
+    rope_offset: int
+    rope_dim: int
+    sources: int
+    inv_freq: np.ndarray          # float32 [F]
+    norm_offset: int
+    norm_dim: int
+    gamma: np.ndarray             # float32 [norm_dim]
+    beta: np.ndarray              # float32 [norm_dim]
+    eps: float
+    d_re: List[np.ndarray]        # per layer float32 [F, sources]
+    d_im: List[np.ndarray]
+    W_nope: List[np.ndarray]      # per layer float32 [d_k - 2F, norm_dim]
+    b_nope: List[np.ndarray]      # per layer float32 [d_k - 2F]
+
+
+def rope_inputs(wl: Workload, sources: int = 1, rope_dim: int = 64, seed: Optional[int] = None) -> RopeInputs:
+    rng = np.random.default_rng((wl.seed if seed is None else seed) + 2000 + sources)
+    F = rope_dim // (2 * sources)
+    norm_dim = wl.d_c - rope_dim
+    d_nope = wl.d_k - 2 * F
+    inv_freq = (10000.0 ** (-np.arange(F, dtype=np.float64) / F)).astype(np.float32)
+    gamma = (1.0 + 0.1 * rng.standard_normal(norm_dim)).astype(np.float32)
+    beta = (0.1 * rng.standard_normal(norm_dim)).astype(np.float32)
+    sd = math.sqrt(wl.d_model / (2.0 * sources))
+    d_re, d_im, W_nope, b_nope = [], [], [], []
+    for _ in range(wl.group):
+        d_re.append((rng.standard_normal((F, sources)) * sd).astype(np.float32))
+        d_im.append((rng.standard_normal((F, sources)) * sd).astype(np.float32))
+        W_nope.append((rng.standard_normal((d_nope, norm_dim)) / math.sqrt(norm_dim)).astype(np.float32))
+        b_nope.append((0.1 * rng.standard_normal(d_nope)).astype(np.float32))
+    return RopeInputs(rope_offset=0, rope_dim=rope_dim, sources=sources, inv_freq=inv_freq,
+                      norm_offset=rope_dim, norm_dim=norm_dim, gamma=gamma, beta=beta, eps=1e-6,
+                      d_re=d_re, d_im=d_im, W_nope=W_nope, b_nope=b_nope)
