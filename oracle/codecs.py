@@ -128,3 +128,21 @@ def e4m3_quantize_rows(c: np.ndarray):
 
 def e4m3_dequantize_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return e4m3_decode(codes).astype(np.float64) * np.asarray(scale, np.float64)[..., None]
+
+
+def e4m3_quantize_rows_segmented(c: np.ndarray, split: int):
+    """Segmented fp8 (LatentIndex summary, Sec. B.2 and Sec. C.1): each row
+    [..., d] is quantised as two independent segments, elements [0, split)
+    and [split, d), each with its own per-row scale (the two branches of
+    the latent keep their own range).  Returns (codes uint8 [..., d],
+    scale float32 [..., 2])."""
+    c = np.asarray(c, dtype=np.float32)
+    c0, s0 = e4m3_quantize_rows(c[..., :split])
+    c1, s1 = e4m3_quantize_rows(c[..., split:])
+    return np.concatenate([c0, c1], axis=-1), np.stack([s0, s1], axis=-1)
+
+
+def e4m3_dequantize_rows_segmented(codes: np.ndarray, scale: np.ndarray, split: int) -> np.ndarray:
+    scale = np.asarray(scale, np.float64)
+    return np.concatenate([e4m3_dequantize_rows(codes[..., :split], scale[..., 0]),
+                           e4m3_dequantize_rows(codes[..., split:], scale[..., 1])], axis=-1)

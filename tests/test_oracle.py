@@ -316,3 +316,29 @@ def test_e4m3_row_quantisation_properties():
     err = np.abs(dq - c)
     bound = np.maximum(np.abs(c) * 2.0 ** -4, 2.0 ** -10 * scale[:, None]) * (1 + 1e-6)
     assert np.all(err <= bound)
+
+
+def test_segmented_e4m3_keeps_each_branch_range():
+    """Segmented fp8: the small-range branch keeps its resolution next to a
+    large-range one; scaling one segment by a power of two scales its scale
+    exactly and changes no code; each element decodes within half an e4m3
+    spacing of its own segment; torch's float8_e4m3fn gives the same codes."""
+    rng = np.random.default_rng(3)
+    c = rng.standard_normal((32, 192)).astype(np.float32)
+    c[:, :64] *= 2e-6                          # a rotary branch far smaller than the NoPE branch
+    codes, scale = codecs.e4m3_quantize_rows_segmented(c, 64)
+    assert codes.shape == (32, 192) and scale.shape == (32, 2)
+    dq = codecs.e4m3_dequantize_rows_segmented(codes, scale, 64)
+    for a, b, k in ((0, 64, 0), (64, 192, 1)):
+        bound = np.maximum(np.abs(c[:, a:b]) * 2.0 ** -4, 2.0 ** -10 * scale[:, k:k + 1]) * (1 + 1e-6)
+        assert np.all(np.abs(dq[:, a:b] - c[:, a:b]) <= bound)
+        ref = (torch.from_numpy(c[:, a:b]) / torch.from_numpy(scale[:, k:k + 1])).to(torch.float8_e4m3fn)
+        assert np.array_equal(codes[:, a:b], ref.view(torch.uint8).numpy())
+    # one scale per row would lose the small branch: most of its codes flush to zero
+    one, _ = codecs.e4m3_quantize_rows(c)
+    assert np.mean((one[:, :64] & 0x7F) == 0) > 0.9 and np.mean((codes[:, :64] & 0x7F) == 0) < 0.05
+    c2 = c.copy()
+    c2[:, 64:] *= 4
+    codes2, scale2 = codecs.e4m3_quantize_rows_segmented(c2, 64)
+    assert np.array_equal(codes2, codes)
+    assert np.array_equal(scale2[:, 0], scale[:, 0]) and np.array_equal(scale2[:, 1], 4 * scale[:, 1])
