@@ -40,7 +40,13 @@ class LiError(RuntimeError):
 class c_li_cache(ctypes.Structure):
     _fields_ = [("data", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("lengths", ctypes.c_void_p),
                 ("batch", ctypes.c_int32), ("capacity", ctypes.c_int32), ("dim", ctypes.c_int32),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("scale_split", ctypes.c_int32)]
+
+
+class c_li_latent_transform(ctypes.Structure):
+    _fields_ = [("rope_offset", ctypes.c_int32), ("rope_dim", ctypes.c_int32), ("rope_sources", ctypes.c_int32),
+                ("inv_freq", ctypes.c_void_p), ("norm_offset", ctypes.c_int32), ("norm_dim", ctypes.c_int32),
+                ("norm_gamma", ctypes.c_void_p), ("norm_beta", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
 
 
 class c_li_query(ctypes.Structure):
@@ -67,6 +73,8 @@ _sigs = {
     "li_device_status": (_I, [_P, _P, _P, ctypes.POINTER(_I)]),
     "li_set_wait_limit": (_I, [_P, ctypes.c_uint64]),
     "li_append_latent": (_I, [_P, ctypes.POINTER(c_li_cache), _P, _I, _I, _P, _I, _P, _SZ, _P]),
+    "li_append_latent_ex": (_I, [_P, ctypes.POINTER(c_li_cache), _P, _I, _I, _P, _I,
+                                 ctypes.POINTER(c_li_latent_transform), _P, _SZ, _P]),
     "li_absorb_query": (_I, [_P, _P, _I, _I, _I, _I, _P, _I64, _P, _I64, _I, _I, _P, _P, _P, _P]),
     "li_score_topk": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _I, _P, _P, _P, _P,
                            _SZ, _P]),
@@ -139,17 +147,42 @@ class Context:
 @dataclass
 class Cache:
     """A latent or key cache: data [batch, capacity, dim] (float32, bfloat16 or
-    uint8 e4m3 codes), scale [batch, capacity] float32 (e4m3 only), lengths
-    [batch] int32."""
+    uint8 e4m3 codes), scale [batch, capacity] float32 (e4m3 only; with
+    segmented fp8, scale_split > 0, [batch, capacity, 2]), lengths [batch]
+    int32."""
     data: torch.Tensor
     lengths: torch.Tensor
     scale: Optional[torch.Tensor] = None
     dtype: Optional[int] = None
+    scale_split: int = 0
 
     def c(self) -> c_li_cache:
         b, cap, dim = self.data.shape
         dt = self.dtype if self.dtype is not None else _dtype(self.data)
-        return c_li_cache(_ptr(self.data), _ptr(self.scale), _ptr(self.lengths), b, cap, dim, dt)
+        return c_li_cache(_ptr(self.data), _ptr(self.scale), _ptr(self.lengths), b, cap, dim, dt,
+                          int(self.scale_split))
+
+
+@dataclass
+class LatentTransform:
+    """The two-branch latent's row transforms (li_latent_transform): rotary
+    range [rope_offset, rope_offset + rope_dim) with inv_freq [rope_dim /
+    (2 rope_sources)] float32, LayerNorm range [norm_offset, norm_offset +
+    norm_dim) with optional gamma / beta [norm_dim] float32."""
+    rope_offset: int = 0
+    rope_dim: int = 0
+    rope_sources: int = 1
+    inv_freq: Optional[torch.Tensor] = None
+    norm_offset: int = 0
+    norm_dim: int = 0
+    gamma: Optional[torch.Tensor] = None
+    beta: Optional[torch.Tensor] = None
+    eps: float = 1e-6
+
+    def c(self) -> c_li_latent_transform:
+        return c_li_latent_transform(self.rope_offset, self.rope_dim, self.rope_sources, _ptr(self.inv_freq),
+                                     self.norm_offset, self.norm_dim, _ptr(self.gamma), _ptr(self.beta),
+                                     float(self.eps))
 
 
 @dataclass
@@ -211,6 +244,16 @@ def li_append_latent(ctx: Context, cache: Cache, h: torch.Tensor, W_down: Option
     cc = cache.c()
     ctx.check(_lib.li_append_latent(ctx.handle, ctypes.byref(cc), _ptr(h), _dtype(h), d_model, _ptr(W_down),
                                     int(T), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def li_append_latent_ex(ctx: Context, cache: Cache, h: torch.Tensor, W_down: Optional[torch.Tensor], T: int,
+                        tf: Optional[LatentTransform], ws: torch.Tensor, stream=None):
+    d_model = h.shape[-1]
+    cc = cache.c()
+    ct = tf.c() if tf is not None else None
+    ctx.check(_lib.li_append_latent_ex(ctx.handle, ctypes.byref(cc), _ptr(h), _dtype(h), d_model, _ptr(W_down),
+                                       int(T), ctypes.byref(ct) if ct is not None else None, _ptr(ws), ws.numel(),
+                                       _stream(stream)))
 
 
 def li_absorb_query(ctx: Context, q: torch.Tensor, W_K: Optional[torch.Tensor], d_c: int, out_dtype: int,

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -80,7 +81,7 @@ struct PlanKey {
   uint64_t wait_ns;
   int32_t batch, capacity, dim, dtype;
   int32_t q_dtype, T, H, gather;
-  int32_t cand_stride, pad;
+  int32_t cand_stride, scale_split;
 };
 
 struct li_ctx {
@@ -208,6 +209,13 @@ li_status check_cache(li_ctx* ctx, const li_cache* c, const char* what) {
     return fail(ctx, LI_ERR_SHAPE, "%s: dim %d must be a multiple of %d in [%d, 256]", what, c->dim, kmul, kmul);
   if (!aligned(c->data, 16)) return fail(ctx, LI_ERR_ALIGN, "%s: cache data not 16-byte aligned", what);
   if (c->scale && !aligned(c->scale, 16)) return fail(ctx, LI_ERR_ALIGN, "%s: scale not 16-byte aligned", what);
+  if (c->scale_split != 0) {
+    if (c->dtype != LI_E4M3)
+      return fail(ctx, LI_ERR_ARG, "%s: scale_split is only for E4M3 caches (got %d)", what, c->scale_split);
+    if (c->scale_split < 0 || c->scale_split >= c->dim || c->scale_split % 32)
+      return fail(ctx, LI_ERR_SHAPE, "%s: scale_split %d must be a multiple of 32 in (0, dim = %d)", what,
+                  c->scale_split, c->dim);
+  }
 
   return LI_OK;
 }
@@ -287,6 +295,7 @@ li_status plan_scan(li_ctx* ctx, const li_cache* c, const li_query* q, bool gath
   k.H = q->H;
   k.gather = gather ? 1 : 0;
   k.cand_stride = cand_stride;
+  k.scale_split = c->scale_split;
   for (int i = 0; i < li_ctx::kPlanCache; ++i)
     if (ctx->plan_used[i] && memcmp(&ctx->plan_key[i], &k, sizeof(k)) == 0) {
       *P = ctx->plan_val[i];
@@ -318,8 +327,13 @@ li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, boo
     swz = 128;
     n_kchunks = static_cast<int>((row_bytes + 127) / 128);
   }
+  // segmented fp8: two scales per row and two accumulators per item, so at
+  // most 128 MMA columns per accumulator
+  const int nsc = c->dtype == LI_E4M3 && c->scale_split > 0 ? 2 : 1;
   const int H_pad = (q->H + 15) / 16 * 16;
-  const int Qg = gather ? 1 : std::max(1, std::min(256 / H_pad, q->T));
+  if (H_pad * nsc > 256)
+    return fail(ctx, LI_ERR_UNSUPPORTED, "%s: H = %d exceeds %d heads with segmented scales", what, q->H, 256 / nsc);
+  const int Qg = gather ? 1 : std::max(1, std::min(256 / nsc / H_pad, q->T));
   const int N = Qg * H_pad;
   const int n_groups = (q->T + Qg - 1) / Qg;
   const int n_seg = gather ? c->batch * q->T : c->batch * n_groups;
@@ -359,8 +373,9 @@ li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, boo
   const size_t budget = static_cast<size_t>(ctx->max_smem_optin) - 1024;
   const size_t kStageCap = 48 * 1024;
   bool planned = false;
-  for (int R = (2 * N <= 256 && !gather) ? 256 : 128; R >= 128 && !planned; R -= 128) {
-    const uint32_t meta_bytes = has_meta ? static_cast<uint32_t>((gather ? 8 : 4) * R) : 0u;
+  for (int R = (2 * N * nsc <= 256 && !gather) ? 256 : 128; R >= 128 && !planned; R -= 128) {
+    // metadata slot: R x nsc scales, then (gather) R token ids
+    const uint32_t meta_bytes = has_meta ? static_cast<uint32_t>((4 * nsc + (gather ? 4 : 0)) * R) : 0u;
     for (int KS = a.n_kchunks; KS >= 1 && !planned; --KS) {
       if (a.n_kchunks % KS) continue;
       const size_t stage = static_cast<size_t>(R) * swz * KS;
@@ -407,9 +422,10 @@ li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, boo
   }
   if (!planned || a.smem_bytes > static_cast<uint32_t>(ctx->max_smem_optin))
     return fail(ctx, LI_ERR_UNSUPPORTED, "%s: operands too large for shared memory (N=%d, dim=%d)", what, N, c->dim);
-  a.n_acc = std::min(4, 512 / (a.MB * N));
+  a.n_acc = std::min(4, 512 / (a.MB * N * nsc));
+  a.seg_kstep = nsc == 2 ? c->scale_split / 32 : 0;
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(a.n_acc * a.MB * N)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(a.n_acc * a.MB * N * nsc)) cols <<= 1;
   a.tmem_cols = cols;
   a.wait_ns = ctx->wait_ns;
   a.trace = ctx->trace;
@@ -687,10 +703,51 @@ li_status li_set_wait_limit(li_ctx* c, uint64_t ns) {
 
 li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_dtype h_dtype, int d_model,
                            const void* W_down, int T, void* ws, size_t ws_bytes, void* stream) {
-  const char* what = "li_append_latent";
+  return li_append_latent_ex(c, cache, h, h_dtype, d_model, W_down, T, nullptr, ws, ws_bytes, stream);
+}
+
+li_status li_append_latent_ex(li_ctx* c, const li_cache* cache, const void* h, li_dtype h_dtype, int d_model,
+                              const void* W_down, int T, const li_latent_transform* tfp, void* ws, size_t ws_bytes,
+                              void* stream) {
+  const char* what = tfp ? "li_append_latent_ex" : "li_append_latent";
   if (!c) return LI_ERR_ARG;
   li_status s = check_cache(c, cache, what);
   if (s != LI_OK) return s;
+  RowTransform tf;
+  memset(&tf, 0, sizeof(tf));
+  if (tfp) {
+    const int dim = cache->dim;
+    if (tfp->rope_dim < 0 || tfp->norm_dim < 0) return fail(c, LI_ERR_SHAPE, "%s: negative branch width", what);
+    if (tfp->rope_dim > 0) {
+      if (tfp->rope_sources < 1) return fail(c, LI_ERR_ARG, "%s: rope_sources must be >= 1", what);
+      if (tfp->rope_offset < 0 || tfp->rope_offset % 2 || tfp->rope_dim % (2 * tfp->rope_sources) ||
+          tfp->rope_offset + tfp->rope_dim > dim)
+        return fail(c, LI_ERR_SHAPE,
+                    "%s: rotary range [%d, %d) must start even, lie in the row of %d and hold whole frequencies "
+                    "of %d sources", what, tfp->rope_offset, tfp->rope_offset + tfp->rope_dim, dim,
+                    tfp->rope_sources);
+      if (!tfp->inv_freq) return fail(c, LI_ERR_ARG, "%s: inv_freq is NULL", what);
+      tf.rope_offset = tfp->rope_offset;
+      tf.rope_dim = tfp->rope_dim;
+      tf.rope_sources = tfp->rope_sources;
+      tf.inv_freq = tfp->inv_freq;
+    }
+    if (tfp->norm_dim > 0) {
+      if (tfp->norm_offset < 0 || tfp->norm_offset + tfp->norm_dim > dim)
+        return fail(c, LI_ERR_SHAPE, "%s: NoPE range [%d, %d) outside the row of %d", what, tfp->norm_offset,
+                    tfp->norm_offset + tfp->norm_dim, dim);
+      if (!(tfp->norm_eps >= 0.f) || !std::isfinite(tfp->norm_eps))
+        return fail(c, LI_ERR_ARG, "%s: norm_eps must be finite and >= 0", what);
+      tf.norm_offset = tfp->norm_offset;
+      tf.norm_dim = tfp->norm_dim;
+      tf.gamma = tfp->norm_gamma;
+      tf.beta = tfp->norm_beta;
+      tf.eps = tfp->norm_eps;
+    }
+    if (tf.rope_dim > 0 && tf.norm_dim > 0 && tf.rope_offset < tf.norm_offset + tf.norm_dim &&
+        tf.norm_offset < tf.rope_offset + tf.rope_dim)
+      return fail(c, LI_ERR_SHAPE, "%s: the rotary and NoPE ranges overlap", what);
+  }
   if (!h) return fail(c, LI_ERR_ARG, "%s: h is NULL", what);
   if (T < 1) return fail(c, LI_ERR_SHAPE, "%s: T must be >= 1", what);
   if (T > cache->capacity) return fail(c, LI_ERR_SHAPE, "%s: T = %d exceeds the capacity", what, T);
@@ -712,7 +769,7 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
     Launch Ls(c, st, "append_store", 0, 256, 0);
     const cudaError_t e = launch_append_store(static_cast<const float*>(h), dim, 0, 1, cache->batch, T, 0, T, true,
                                               cache->data, cache->scale, cache->lengths, cache->capacity, dim,
-                                              cache->dtype, done, status, st);
+                                              cache->dtype, cache->scale_split, tf, done, status, st);
     Ls.done();
     return e == cudaSuccess ? LI_OK : cuda_fail(c, e, "append store launch");
   }
@@ -727,7 +784,7 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
       Launch Lg(c, st, "append", 0, 256, 0);
       const cudaError_t e = launch_append_fused(h, h_dtype, W_down, d_model, dim, cache->batch, T, splits, tmp,
                                                 cache->data, cache->scale, cache->lengths, cache->capacity,
-                                                cache->dtype, done, status, st);
+                                                cache->dtype, cache->scale_split, tf, done, status, st);
       Lg.done();
       return e == cudaSuccess ? LI_OK : cuda_fail(c, e, "append launch");
     }
@@ -757,7 +814,7 @@ li_status li_append_latent(li_ctx* c, const li_cache* cache, const void* h, li_d
     const cudaError_t e = launch_append_store(tmp, dim, static_cast<int64_t>(cache->batch) * tn * dim, splits,
                                               cache->batch, tn, t0, T, t0 + tn >= T, cache->data,
                                               cache->scale, cache->lengths, cache->capacity, dim, cache->dtype,
-                                              done, status, st);
+                                              cache->scale_split, tf, done, status, st);
     Ls.done();
     if (e != cudaSuccess) return cuda_fail(c, e, "append store launch");
   }

@@ -94,10 +94,82 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const T* __restri
       out[(static_cast<int64_t>(sp) * n_tok + m0 + t) * dim + j] = acc[t];
 }
 
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// The two-branch latent's row transforms (LatentIndex summary, Sec. 3.1,
+// Sec. A.2, Sec. D.2) on one fp32 row held by a warp (lane holds elements
+// lane + 32 e): LayerNorm of the NoPE range (biased variance, correctly
+// rounded division and square root), and rotation of the rotary range at
+// position `pos`: slot p = (x[2p], x[2p+1]) of the range turns by
+// pos * inv_freq[p / sources], the angle formed exactly and its cosine and
+// sine taken in double precision, then rounded to fp32.  Slot partners are
+// adjacent lanes (the range starts on an even element).
+__device__ __forceinline__ void transform_row(float (&v)[8], int lane, int64_t pos, const RowTransform& tf) {
+  if (tf.norm_dim > 0) {
+    const int a = tf.norm_offset, b = tf.norm_offset + tf.norm_dim;
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = lane + 32 * e;
+      if (i >= a && i < b) s += v[e];
+    }
+    const float mean = __fdiv_rn(warp_sum(s), static_cast<float>(tf.norm_dim));
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = lane + 32 * e;
+      if (i >= a && i < b) {
+        const float d = v[e] - mean;
+        ss = fmaf(d, d, ss);
+      }
+    }
+    const float sd = __fsqrt_rn(__fdiv_rn(warp_sum(ss), static_cast<float>(tf.norm_dim)) + tf.eps);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = lane + 32 * e;
+      if (i >= a && i < b) {
+        float y = __fdiv_rn(v[e] - mean, sd);
+        if (tf.gamma) y *= __ldg(tf.gamma + (i - a));
+        if (tf.beta) y += __ldg(tf.beta + (i - a));
+        v[e] = y;
+      }
+    }
+  }
+  if (tf.rope_dim > 0) {
+    const int a = tf.rope_offset, b = tf.rope_offset + tf.rope_dim;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = lane + 32 * e;
+      const float partner = __shfl_xor_sync(0xffffffffu, v[e], 1);
+      if (i >= a && i < b) {
+        const int f = ((i - a) >> 1) / tf.rope_sources;
+        double sn, cs;
+        sincos(static_cast<double>(pos) * static_cast<double>(__ldg(tf.inv_freq + f)), &sn, &cs);
+        const float c = static_cast<float>(cs), sf = static_cast<float>(sn);
+        v[e] = ((i - a) & 1) == 0 ? v[e] * c - partner * sf : partner * sf + v[e] * c;
+      }
+    }
+  }
+}
+
 // Write one fp32 row (lane holds elements lane + 32 e) into the cache at
-// `row` in the cache dtype; e4m3 rows also get their scale amax / 448.
-__device__ __forceinline__ void write_row(const float (&v)[8], float amax, int lane, int64_t row, int dim, int dtype,
-                                          void* data, float* scale) {
+// `row` (sequence position `pos`) in the cache dtype, after the row
+// transforms.  E4M3 rows get scale amax / 448 per row, or, with
+// scale_split > 0, one per segment: elements [0, scale_split) and
+// [scale_split, dim), stored as scale[2 row] and scale[2 row + 1].
+__device__ __forceinline__ void write_row(float (&v)[8], int lane, int64_t row, int64_t pos, int dim, int dtype,
+                                          int scale_split, const RowTransform& tf, void* data, float* scale) {
+  transform_row(v, lane, pos, tf);
   if (dtype == LI_F32) {
     float* dst = reinterpret_cast<float*>(data) + row * dim;
 #pragma unroll
@@ -109,14 +181,33 @@ __device__ __forceinline__ void write_row(const float (&v)[8], float amax, int l
     for (int e = 0; e < 8; ++e)
       if (lane + 32 * e < dim) dst[lane + 32 * e] = __float2bfloat16_rn(v[e]);
   } else {
+    float am0 = 0.f, am1 = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    for (int e = 0; e < 8; ++e) {
+      const int i = lane + 32 * e;
+      if (i < dim) {
+        if (scale_split > 0 && i >= scale_split) am1 = fmaxf(am1, fabsf(v[e]));
+        else am0 = fmaxf(am0, fabsf(v[e]));
+      }
+    }
+    am0 = warp_max(am0);
+    am1 = warp_max(am1);
+    const float sc0 = am0 > 0.f ? __fdiv_rn(am0, 448.f) : 1.f;
+    const float sc1 = am1 > 0.f ? __fdiv_rn(am1, 448.f) : 1.f;
     uint8_t* dst = reinterpret_cast<uint8_t*>(data) + row * dim;
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (lane + 32 * e < dim) dst[lane + 32 * e] = to_e4m3(__fdiv_rn(v[e], sc));
-    if (lane == 0) scale[row] = sc;
+    for (int e = 0; e < 8; ++e) {
+      const int i = lane + 32 * e;
+      if (i < dim) dst[i] = to_e4m3(__fdiv_rn(v[e], scale_split > 0 && i >= scale_split ? sc1 : sc0));
+    }
+    if (lane == 0) {
+      if (scale_split > 0) {
+        scale[2 * row] = sc0;
+        scale[2 * row + 1] = sc1;
+      } else {
+        scale[row] = sc0;
+      }
+    }
   }
 }
 
@@ -137,8 +228,9 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
                                                                       int dim, int n_tok, int splits,
                                                                       float* __restrict__ part, int batch, int T_tok,
                                                                       void* data, float* scale, int32_t* lengths,
-                                                                      int capacity, int dtype,
-                                                                      unsigned int* done, int* status) {
+                                                                      int capacity, int dtype, int scale_split,
+                                                                      RowTransform tf, unsigned int* done,
+                                                                      int* status) {
   pdl_begin();
   extern __shared__ __align__(16) float ps[];       // [splits][n_tok * dim], then cs [n_tok * dim]
   __shared__ unsigned last;
@@ -215,14 +307,13 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
       continue;
     }
     float v[8];
-    float amax = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = lane + 32 * e;
       v[e] = i < dim ? cs[m * dim + i] : 0.f;
-      amax = fmaxf(amax, fabsf(v[e]));
     }
-    write_row(v, amax, lane, static_cast<int64_t>(b) * capacity + len + t, dim, dtype, data, scale);
+    write_row(v, lane, static_cast<int64_t>(b) * capacity + len + t, len + t, dim, dtype, scale_split, tf, data,
+              scale);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -242,8 +333,8 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
                                                     int64_t split_stride, int splits,
                                                     int batch, int T_chunk, int t0, int T_total, int bump,
                                                     void* data, float* scale, int32_t* lengths,
-                                                    int capacity, int dim, int dtype,
-                                                    unsigned int* done, int* status) {
+                                                    int capacity, int dim, int dtype, int scale_split,
+                                                    RowTransform tf, unsigned int* done, int* status) {
   pdl_begin();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok = blockIdx.x * 8 + warp;
@@ -256,7 +347,6 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
       const int64_t row = static_cast<int64_t>(b) * capacity + len + t0 + t;
       const float* src = c + static_cast<int64_t>(tok) * c_tok_stride;
       float v[8];
-      float amax = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int i = lane + 32 * e;
@@ -272,9 +362,8 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
             if (sp < splits) x += part[sp];
         }
         v[e] = x;
-        amax = fmaxf(amax, fabsf(v[e]));
       }
-      write_row(v, amax, lane, row, dim, dtype, data, scale);
+      write_row(v, lane, row, len + t0 + t, dim, dtype, scale_split, tf, data, scale);
     }
   }
   if (!bump) return;
@@ -525,7 +614,8 @@ bool append_fusable(int n_tok, int dim, int splits) {
 
 cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
                                 int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
-                                int dtype, unsigned int* done, int* status, cudaStream_t st) {
+                                int dtype, int scale_split, const RowTransform& tf, unsigned int* done, int* status,
+                                cudaStream_t st) {
   const int n_tok = batch * T;
   const int grid = splits * ((dim + kAppendWarps - 1) / kAppendWarps);
   const size_t smem = static_cast<size_t>(splits + 1) * n_tok * dim * sizeof(float);
@@ -535,24 +625,25 @@ cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d
     if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
     return launch_pdl(k, dim3(grid), dim3(kAppendWarps * 32), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(h),
                       reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim, n_tok, splits, part, batch, T, data,
-                      scale, lengths, capacity, dtype, done, status);
+                      scale, lengths, capacity, dtype, scale_split, tf, done, status);
   } else {
     auto k = gemv_append_kernel<float>;
     if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
     return launch_pdl(k, dim3(grid), dim3(kAppendWarps * 32), smem, st, 1, reinterpret_cast<const float*>(h),
                       reinterpret_cast<const float*>(W), d_model, dim, n_tok, splits, part, batch, T, data, scale,
-                      lengths, capacity, dtype, done, status);
+                      lengths, capacity, dtype, scale_split, tf, done, status);
   }
 }
 
 cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits, int batch,
                                 int T_chunk, int t0, int T_total, bool bump, void* data, float* scale,
-                                int32_t* lengths, int capacity, int dim, int dtype, unsigned int* done_counter,
-                                int* status, cudaStream_t st) {
+                                int32_t* lengths, int capacity, int dim, int dtype, int scale_split,
+                                const RowTransform& tf, unsigned int* done_counter, int* status, cudaStream_t st) {
   const int n_tok = batch * T_chunk;
   const int grid = (n_tok + 7) / 8;
   return launch_pdl(store_kernel, dim3(grid), dim3(256), 0, st, 1, c, c_tok_stride, split_stride, splits, batch, T_chunk,
-                    t0, T_total, bump ? 1 : 0, data, scale, lengths, capacity, dim, dtype, done_counter, status);
+                    t0, T_total, bump ? 1 : 0, data, scale, lengths, capacity, dim, dtype, scale_split, tf,
+                    done_counter, status);
 }
 
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,

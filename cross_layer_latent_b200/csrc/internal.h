@@ -27,7 +27,7 @@ struct alignas(64) ScanArgs {
   CUtensorMap map_a;          // cache rows: dims {swz/elt, batch*capacity, n_kchunks}, box {swz/elt, R, KS};
                               // gather: dims {dim, batch*capacity}, box {swz/elt, 1}
   CUtensorMap map_b;          // queries: dims {dim, H, batch*T}, box {swz/elt, H_pad, Qg}
-  const float* cache_scale;   // [batch*capacity] or null
+  const float* cache_scale;   // [batch*capacity] (segmented: [batch*capacity][2]) or null
   const int* lengths;         // [batch]
   const int* q_pos;           // [batch*T] or null
   const float* w;             // [batch*T*H]
@@ -51,6 +51,7 @@ struct alignas(64) ScanArgs {
   uint32_t tmem_cols, idesc;
   uint32_t a_stage_bytes, b_slot_bytes, meta_bytes, misc_offset, smem_bytes;
   int n_segments;
+  int seg_kstep;              // segmented fp8: first K step (32 bytes) of the second scale's segment; 0: one scale
   uint64_t* trace;            // per-tile event times of the first kTraceCtas CTAs, or null
 };
 
@@ -150,6 +151,17 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st);
 
 // Split count of the construction GEMV for n_tok tokens of width d_model.
 int gemv_splits(int d_model, int n_tok);
+// Per-row transforms of the two-branch latent, applied after c = W_down h
+// and before quantisation (see li_latent_transform).  All zero: none.
+struct RowTransform {
+  int rope_offset, rope_dim, rope_sources;
+  const float* inv_freq;
+  int norm_offset, norm_dim;
+  const float* gamma;
+  const float* beta;
+  float eps;
+};
+
 cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_model, int dim,
                                int n_tok, int splits, float* out, cudaStream_t st);
 // Decode-sized appends (at most 8 tokens whose partial sums fit one block's
@@ -159,11 +171,12 @@ int append_fused_splits(int d_model, int dim);
 bool append_fusable(int n_tok, int dim, int splits);
 cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
                                 int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
-                                int dtype, unsigned int* done, int* status, cudaStream_t st);
+                                int dtype, int scale_split, const RowTransform& tf, unsigned int* done, int* status,
+                                cudaStream_t st);
 cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits,
                                 int batch, int T_chunk, int t0, int T_total, bool bump, void* data,
-                                float* scale, int32_t* lengths, int capacity, int dim, int dtype,
-                                unsigned int* done_counter, int* status, cudaStream_t st);
+                                float* scale, int32_t* lengths, int capacity, int dim, int dtype, int scale_split,
+                                const RowTransform& tf, unsigned int* done_counter, int* status, cudaStream_t st);
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
                           int out_dtype, void* q_abs, float* q_abs_scale, float* beta,

@@ -40,7 +40,7 @@ constexpr uint64_t kDrainNs = 200ull * 1000ull * 1000ull;   // 0.2 s
 struct ScanSmem {
   uint8_t* a_stages;
   uint8_t* b_slots;
-  uint8_t* meta;        // n_meta x meta_bytes: scale[R] (then tok[R] when gathering)
+  uint8_t* meta;        // n_meta x meta_bytes: scale[R x scales per row] (then tok[R] when gathering)
   uint64_t* full;
   uint64_t* empty;
   uint64_t* bfull;
@@ -147,6 +147,11 @@ __device__ __forceinline__ void cp_async_4_zfill(uint32_t dst_smem, const void* 
                : "memory");
 }
 
+__device__ __forceinline__ void cp_async_8_zfill(uint32_t dst_smem, const void* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
 // Bulk (non-tensor) global -> shared copy completing on an mbarrier;
 // addresses and size must be multiples of 16 bytes.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -206,6 +211,8 @@ __device__ __forceinline__ void issue_chunk_rt(int ksteps, int mbs, uint32_t d0,
     case 1 * 4 + 2: issue_chunk<KIND, 1, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
     case 2 * 4 + 1: issue_chunk<KIND, 2, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
     case 2 * 4 + 2: issue_chunk<KIND, 2, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 3 * 4 + 1: issue_chunk<KIND, 3, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 3 * 4 + 2: issue_chunk<KIND, 3, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
     case 4 * 4 + 1: issue_chunk<KIND, 4, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
     default: issue_chunk<KIND, 4, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
   }
@@ -303,6 +310,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const uint32_t k_meta_bytes = a.meta_bytes;
   const int64_t k_score_stride = a.score_stride;
   const float* const k_cache_scale = a.cache_scale;
+  const int k_SK = a.seg_kstep;              // > 0: two scales per row, two accumulators per (slot, M block)
+  const int k_nsc = k_SK > 0 ? 2 : 1;
   const int* const k_lengths = a.lengths;
   const int* const k_q_pos = a.q_pos;
   const float* const k_w = a.w;
@@ -356,10 +365,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           // capacity are not read: the epilogue ignores them)
           if (!bounded_wait(&s.mempty[ms.i], ms.ph ^ 1u, wc)) break;
           const int rows = min(k_R, k_capacity - it * k_R);
-          const uint32_t bytes = static_cast<uint32_t>(rows) * 4u;
+          const uint32_t bytes = static_cast<uint32_t>(rows * k_nsc) * 4u;
           mbar_arrive_expect_tx(&s.mfull[ms.i], bytes);
           bulk_load(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes,
-                    k_cache_scale + static_cast<int64_t>(w.b) * k_capacity + it * k_R, bytes, &s.mfull[ms.i]);
+                    k_cache_scale + (static_cast<int64_t>(w.b) * k_capacity + it * k_R) * k_nsc, bytes,
+                    &s.mfull[ms.i]);
           ms.step(NM);
           ++n_ms;
         }
@@ -442,7 +452,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       const int len = s.seg_len[seg], cn = s.seg_n[seg];
       if (!bounded_wait(&s.mempty[ms.i], ms.ph ^ 1u, wc)) break;
       float* mscale = reinterpret_cast<float*>(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes);
-      int* mtok = reinterpret_cast<int*>(mscale + k_R);
+      int* mtok = reinterpret_cast<int*>(mscale + k_R * k_nsc);
       const int seq_row = w.b * k_capacity;
 #pragma unroll
       for (int i = 0; i < kIdsPerLane; ++i) {
@@ -452,7 +462,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           int t = (r < k_RI && j < cn) ? cur[i] : -1;
           if (j < cn && (t < 0 || t >= len)) t = -2;     // invalid candidate
           mtok[r] = t;
-          if (e4) cp_async_4_zfill(smem_addr(mscale + r), k_cache_scale + seq_row + (t >= 0 ? t : 0), t >= 0 ? 4 : 0);
+          if (e4) {
+            const int64_t srow = seq_row + (t >= 0 ? t : 0);
+            if (k_nsc == 2) cp_async_8_zfill(smem_addr(mscale + 2 * r), k_cache_scale + 2 * srow, t >= 0 ? 8 : 0);
+            else cp_async_4_zfill(smem_addr(mscale + r), k_cache_scale + srow, t >= 0 ? 4 : 0);
+          }
         }
       }
       cp_async_arrive_noinc(&s.mfull[ms.i]);
@@ -518,7 +532,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (!bounded_wait(&s.accempty[2 * acc.i + mi], acc.ph ^ 1u, wc)) break;
         tc_fence_after();
         const uint32_t d0 = tmem + (acc.i * static_cast<uint32_t>(k_MB) + static_cast<uint32_t>(mi)) *
-                                       static_cast<uint32_t>(k_N);
+                                       static_cast<uint32_t>(k_N * k_nsc);
         const uint32_t b_base = smem_addr(s.b_slots + static_cast<size_t>(slot) * k_b_slot_bytes);
         bool ok = true;
         for (int sp = 0; sp < k_spi; ++sp) {
@@ -529,9 +543,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           const uint32_t a_base = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes) + m_off;
           for (int c = 0; c < k_KS; ++c) {
             const int kc = sp * k_KS + c;
-            issue_chunk_rt<KIND>(static_cast<int>(ksteps), 1, d0, a_base + static_cast<uint32_t>(c) * chunk_region,
-                                 b_base + static_cast<uint32_t>(kc * k_N * k_swz), desc_hi, 0u,
-                                 static_cast<uint32_t>(k_N), k_idesc, kc == 0);
+            const uint32_t a_c = a_base + static_cast<uint32_t>(c) * chunk_region;
+            const uint32_t b_c = b_base + static_cast<uint32_t>(kc * k_N * k_swz);
+            if (k_SK == 0) {
+              issue_chunk_rt<KIND>(static_cast<int>(ksteps), 1, d0, a_c, b_c, desc_hi, 0u,
+                                   static_cast<uint32_t>(k_N), k_idesc, kc == 0);
+            } else {
+              // segmented scales: K steps before k_SK accumulate into the
+              // first accumulator, the rest into the second (N columns on)
+              const int g0 = kc * static_cast<int>(ksteps);
+              const int n0 = max(0, min(static_cast<int>(ksteps), k_SK - g0));
+              if (n0 > 0)
+                issue_chunk_rt<KIND>(n0, 1, d0, a_c, b_c, desc_hi, 0u, static_cast<uint32_t>(k_N), k_idesc, kc == 0);
+              if (n0 < static_cast<int>(ksteps))
+                issue_chunk_rt<KIND>(static_cast<int>(ksteps) - n0, 1, d0 + static_cast<uint32_t>(k_N),
+                                     a_c + static_cast<uint32_t>(n0) * 32u, b_c + static_cast<uint32_t>(n0) * 32u,
+                                     desc_hi, 0u, static_cast<uint32_t>(k_N), k_idesc, g0 + n0 == k_SK);
+            }
           }
           umma_commit(&s.empty[st.i]);
           st.step(S);
@@ -621,19 +649,31 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       const int j = it * k_RI + r;          // position (scan) or candidate slot (gather)
       const bool row_in_item = !GATHER || r < k_RI;
       int tok = j;
-      float cs = 1.f;
+      float cs = 1.f, cs1 = 0.f;
       if (has_meta) {
         if (!bounded_wait(&s.mfull[ms.i], ms.ph, wc)) break;
         const float* mscale = reinterpret_cast<const float*>(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes);
-        if (GATHER) tok = reinterpret_cast<const int*>(mscale + k_R)[r];
-        if (e4 && tok >= 0) cs = mscale[r];    // rows past the valid prefix read a stale value, unused
+        if (GATHER) tok = reinterpret_cast<const int*>(mscale + k_R * k_nsc)[r];
+        // rows past the valid prefix read stale values, unused
+        if (e4 && tok >= 0) {
+          if (k_nsc == 2) {
+            cs = mscale[2 * r];
+            cs1 = mscale[2 * r + 1];
+          } else {
+            cs = mscale[r];
+          }
+        }
       }
       if (!bounded_wait(&s.accfull[2 * acc.i + mb], acc.ph, wc)) break;
       if (lane == 0 && (ew & 3) == 0) trace_event(k_trace, lt, 4);
       tc_fence_after();
 
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
-                             (acc.i * static_cast<uint32_t>(k_MB) + static_cast<uint32_t>(mb)) * static_cast<uint32_t>(k_N);
+                             (acc.i * static_cast<uint32_t>(k_MB) + static_cast<uint32_t>(mb)) *
+                                 static_cast<uint32_t>(k_N * k_nsc);
+      // segmented scales: head h's product is cs * D0_h + cs1 * D1_h; without
+      // a bias cs is factored out (cs > 0) and D0_h + (cs1 / cs) D1_h summed
+      const float rho = k_nsc == 2 ? cs1 / cs : 0.f;
       for (int qi = 0; qi < k_Qg; ++qi) {
         const int t = g * k_Qg + qi;
         if (t >= k_T) break;
@@ -642,6 +682,22 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         const float* qs = ep_qs + qi * k_H_pad;
         const float* be = ep_beta + qi * k_H_pad;
         int h0 = 0;
+        if (k_nsc == 2) {
+          for (; h0 + 16 <= k_H_pad; h0 += 16) {
+            float v[16], v1[16];
+            tmem_load16x2_sync(tbase + static_cast<uint32_t>(qi * k_H_pad + h0),
+                               tbase + static_cast<uint32_t>(k_N + qi * k_H_pad + h0), v, v1);
+            if (!has_beta) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = fmaf(rho, v1[e], v[e]);
+              relu_dot16(v, wq + h0, part);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = fmaf(cs1, v1[e], cs * v[e]);
+              relu_dot16_beta(v, wq + h0, qs + h0, be + h0, 1.f, part);
+            }
+          }
+        }
         for (; h0 + 32 <= k_H_pad; h0 += 32) {
           float v[32];
           tmem_load32_sync(tbase + static_cast<uint32_t>(qi * k_H_pad + h0), v);

@@ -14,18 +14,21 @@ from typing import List, Optional
 
 import torch
 
-from ._binding import (LI_BF16, LI_E4M3, LI_F32, Cache, Context, Query, li_absorb_query, li_append_latent,
-                       li_dsa_score_topk, li_hs_anchor_candidates, li_hs_follower_refine, li_score_topk,
+from ._binding import (LI_BF16, LI_E4M3, LI_F32, Cache, Context, LatentTransform, Query, li_absorb_query,
+                       li_append_latent, li_append_latent_ex, li_dsa_score_topk, li_hs_anchor_candidates, li_hs_follower_refine, li_score_topk,
                        workspace)
 
 TORCH_DTYPE = {LI_F32: torch.float32, LI_BF16: torch.bfloat16, LI_E4M3: torch.uint8}
 
 
-def _cache(batch, capacity, dim, dtype, device) -> Cache:
+def _cache(batch, capacity, dim, dtype, device, scale_split: int = 0) -> Cache:
+    scale = None
+    if dtype == LI_E4M3:
+        shape = (batch, capacity, 2) if scale_split else (batch, capacity)
+        scale = torch.ones(*shape, dtype=torch.float32, device=device)
     return Cache(data=torch.zeros(batch, capacity, dim, dtype=TORCH_DTYPE[dtype], device=device),
-                 lengths=torch.zeros(batch, dtype=torch.int32, device=device),
-                 scale=torch.ones(batch, capacity, dtype=torch.float32, device=device) if dtype == LI_E4M3 else None,
-                 dtype=dtype)
+                 lengths=torch.zeros(batch, dtype=torch.int32, device=device), scale=scale, dtype=dtype,
+                 scale_split=scale_split)
 
 
 class GroupIndexer:
@@ -34,13 +37,19 @@ class GroupIndexer:
 
     def __init__(self, ctx: Context, *, batch: int, capacity: int, d_c: int, H: int, d_k: int, G: int = 4,
                  dtype: int = LI_BF16, k: int = 2048, B: Optional[int] = None, T: int = 1, dsa: bool = False,
-                 device: Optional[str] = None):
+                 device: Optional[str] = None, transform: Optional[LatentTransform] = None,
+                 scale_split: int = 0):
+        """transform: the two-branch latent's row transforms applied by every
+        append to the shared latent (rotary branch rotated at the row's
+        position, LayerNorm on the NoPE branch); scale_split > 0 stores the
+        latent as segmented fp8 (E4M3 only)."""
         self.ctx = ctx
+        self.transform = transform
         self.device = device or f"cuda:{ctx.device}"
         self.batch, self.capacity, self.d_c, self.H, self.d_k = batch, capacity, d_c, H, d_k
         self.G, self.dtype, self.k, self.B, self.T = G, dtype, k, B, T
         dev, tdt = self.device, TORCH_DTYPE[dtype]
-        self.latent = _cache(batch, capacity, d_c, dtype, dev)
+        self.latent = _cache(batch, capacity, d_c, dtype, dev, scale_split)
         self.keys: List[Cache] = [_cache(batch, capacity, d_k, dtype, dev) for _ in range(G)] if dsa else []
         # layer-major storage: layer l's queries are the contiguous slice [l],
         # and the fused group scan restacks all layers with one copy each
@@ -98,7 +107,7 @@ class GroupIndexer:
         """Append T new tokens per sequence to the shared latent cache:
         h [batch, T, d_model] with W_down [d_c, d_model], or the fp32 latent
         [batch, T, d_c] itself when W_down is None."""
-        li_append_latent(self.ctx, self.latent, h, W_down, h.shape[1], self.ws, stream)
+        li_append_latent_ex(self.ctx, self.latent, h, W_down, h.shape[1], self.transform, self.ws, stream)
 
     def append_keys(self, layer: int, h: torch.Tensor, W_k: Optional[torch.Tensor] = None, stream=None):
         """Append to layer `layer`'s DSA key cache (key = W_k h)."""

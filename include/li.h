@@ -92,7 +92,13 @@ typedef struct li_ctx li_ctx;
  *         device by li_append_latent).
  * dim: multiple of 8 (F32), 16 (BF16) or 32 (E4M3), at most 256.  Scanning
  * an E4M3 cache (li_score_topk, li_hs_anchor_candidates, li_dsa_score_topk)
- * needs capacity % 4 == 0 and a 16-byte aligned scale array.                */
+ * needs capacity % 4 == 0 and a 16-byte aligned scale array.
+ * scale_split: 0 for one scale per row.  For E4M3 caches, a value in
+ *         (0, dim) that is a multiple of 32 selects segmented fp8 (Sec. B.2,
+ *         Sec. C.1): two scales per row, scale [batch][capacity][2], the
+ *         first for elements [0, scale_split) (the rotary branch) and the
+ *         second for [scale_split, dim) (the NoPE branch).  Must be 0 for
+ *         F32 and BF16 caches.                                            */
 typedef struct {
   void* data;
   float* scale;
@@ -101,6 +107,7 @@ typedef struct {
   int32_t capacity;
   int32_t dim;
   li_dtype dtype;
+  int32_t scale_split;
 } li_cache;
 
 /* The queries of one layer for every sequence of the batch.
@@ -170,6 +177,49 @@ LI_API li_status li_set_wait_limit(li_ctx* ctx, uint64_t ns);
 LI_API li_status li_append_latent(li_ctx* ctx, const li_cache* cache, const void* h, li_dtype h_dtype,
                            int d_model, const void* W_down, int T, void* ws, size_t ws_bytes,
                            void* stream);
+
+/* The two-branch latent (Sec. 3.1: RoPE and NoPE branches concatenated and
+ * cached once per group; Sec. A.2: the rotary branch is rotated before
+ * caching; Sec. A.4: one or more complex sources per rotary frequency;
+ * Sec. D.2: LayerNorm on the NoPE branch only).  li_append_latent_ex applies
+ * these to each new row after c = W_down h and before quantisation.
+ * Rotary branch: elements [rope_offset, rope_offset + rope_dim) hold
+ *   rope_dim / 2 complex slots, slot p = (x[2p], x[2p+1]) counted from
+ *   rope_offset, of frequency f = p / rope_sources.  The row written at
+ *   cache row s (its sequence position) has slot p multiplied by
+ *   exp(i s inv_freq[f]): x' = x cos - y sin, y' = x sin + y cos, with the
+ *   angle formed exactly and its cosine and sine taken in double precision,
+ *   rounded to fp32.  rope_dim = 0 disables it; otherwise rope_offset and
+ *   rope_dim are even, rope_dim is a multiple of 2 * rope_sources and
+ *   inv_freq is a device array of rope_dim / (2 rope_sources) fp32.
+ *   Decoders must be frequency-wise complex on this branch (each layer's
+ *   rotary key slot f a complex combination of the sources of frequency f),
+ *   so that absorbing them into post-RoPE queries scores the rotated latent
+ *   exactly; the native key layout they target is the caller's choice.
+ * NoPE branch: elements [norm_offset, norm_offset + norm_dim) are replaced
+ *   by (x - mean) / sqrt(var + norm_eps) * gamma + beta (biased variance,
+ *   fp32, correctly rounded division and square root); gamma and beta are
+ *   device arrays of norm_dim fp32, or NULL for 1 and 0.  norm_dim = 0
+ *   disables it.
+ * The two ranges must lie inside the row and must not overlap.            */
+typedef struct {
+  int32_t rope_offset;
+  int32_t rope_dim;
+  int32_t rope_sources;
+  const float* inv_freq;
+  int32_t norm_offset;
+  int32_t norm_dim;
+  const float* norm_gamma;
+  const float* norm_beta;
+  float norm_eps;
+} li_latent_transform;
+
+/* li_append_latent with the two-branch transforms; tf NULL is
+ * li_append_latent.  Errors: LI_ERR_ARG / LI_ERR_SHAPE for an invalid
+ * transform (checked on the host before anything is enqueued).           */
+LI_API li_status li_append_latent_ex(li_ctx* ctx, const li_cache* cache, const void* h, li_dtype h_dtype,
+                              int d_model, const void* W_down, int T, const li_latent_transform* tf,
+                              void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------- a2: absorb */
 
