@@ -32,7 +32,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from workloads import construction_inputs, generate, workload  # noqa: E402
+from workloads import construction_inputs, generate, rope_inputs, workload  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
 METRIC = "decode indexer keys scored/s and % HBM roofline at 8K-128K ctx; HS vs DSA path"
@@ -50,6 +50,7 @@ def parse():
     p.add_argument("--no-other-contexts", action="store_true")
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-fused", action="store_true")
+    p.add_argument("--no-two-branch", action="store_true")
     return p.parse_args()
 
 
@@ -492,23 +493,12 @@ def prefill_leg(li, ctx, args, rank, dev):
             "keys_per_s": wl.group * pairs / (sum(call_ms) / 1e3)}
 
 
-def fused_leg(step, args, flush, stream, dist, dev, world):
-    """Scoring + selection of all G layers over the full prefix: G per-layer
-    scans of the shared latent, against one scan with the G layers' absorbed
-    queries stacked (G * H MMA columns; queries from the anchor's hidden state
-    in the training-aware instantiation).  Both from captured graphs, L2
-    flushed before each, CUDA events on the stream."""
-    g, wl = step.g, step.wl
-    step.reset()
-    step.hs_path()                       # absorbed queries of every layer
-    torch.cuda.synchronize()
-
-    def per_layer():
-        for l in range(wl.group):
-            g.score_topk(l)
-
+def graph_times(fns, args, flush, stream, dist, dev):
+    """Mean device time (ms, slowest rank) of each callable, captured once as
+    a CUDA graph and replayed: W warm-up replays, then K timed ones, each
+    after an L2 flush and between CUDA events on the stream."""
     graphs = []
-    for fn in (per_layer, g.fused_group_score_topk):
+    for fn in fns:
         fn()
         torch.cuda.synchronize()
         gr = torch.cuda.CUDAGraph()
@@ -530,6 +520,70 @@ def fused_leg(step, args, flush, stream, dist, dev, world):
             ms.append(e0.elapsed_time(e1))
         times.append(max_over_ranks(statistics.mean(ms), dist, dev))
     del graphs
+    return times
+
+
+def two_branch_leg(step, args, flush, stream, dist, dev):
+    """The pages' inference format for the same workload: the two-branch
+    latent (rotary branch [0, 64) rotated at each row's position, LayerNorm on
+    the NoPE branch [64, 192)) stored as segmented fp8 (one e4m3 scale per
+    branch, 200 bytes a row), against the single-scale latent of the main
+    step.  Times the decode append (projection + transforms + quantisation),
+    the HS anchor (scan + both selections) and one follower."""
+    li, g, wl, inp = step.li, step.g, step.wl, step.inp
+    ri = rope_inputs(wl)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)  # noqa: E731
+    tf = li.LatentTransform(rope_offset=ri.rope_offset, rope_dim=ri.rope_dim, rope_sources=ri.sources,
+                            inv_freq=t(ri.inv_freq), norm_offset=ri.norm_offset, norm_dim=ri.norm_dim,
+                            gamma=t(ri.gamma), beta=t(ri.beta), eps=ri.eps)
+    g2 = li.GroupIndexer(step.ctx, batch=wl.batch, capacity=wl.capacity, d_c=wl.d_c, H=wl.heads, d_k=wl.d_k,
+                         G=wl.group, dtype=li.LI_E4M3, k=wl.k, B=wl.B, device=dev, transform=tf, scale_split=64)
+    g2.load(inp.lengths, inp.W_K, inp.q, inp.w, latent=inp.latent)
+    step.reset()
+    step.hs_path()                       # the main group's queries and candidates
+    torch.cuda.synchronize()
+    before = step.len_before
+
+    def append(grp):
+        def fn():
+            grp.latent.lengths.copy_(before)
+            grp.append(step.h_anchor, step.W_down)
+        return fn
+
+    fns = [append(g), append(g2), lambda: g.hs_anchor(0), lambda: g2.hs_anchor(0),
+           lambda: g.hs_follower(1), lambda: g2.hs_follower(1)]
+    t_ms = graph_times(fns, args, flush, stream, dist, dev)
+    for grp in (g, g2):
+        grp.latent.lengths.copy_(torch.from_numpy(inp.lengths).to(dev))
+    st = li.li_device_status(step.ctx, g2.ws)
+    if st != "LI_OK":
+        raise RuntimeError(f"device status after the two-branch leg: {st}")
+    n_rows = int(sum(int(n) for n in inp.lengths))
+    out = {"mode": "rotary 64 + NoPE 128 (LayerNorm), segmented e4m3 (2 scales, 200 B/row) vs one scale (196 B/row)"}
+    for name, (a, b) in {"append": (0, 1), "anchor": (2, 3), "follower": (4, 5)}.items():
+        out[f"{name}_ms"] = t_ms[b]
+        out[f"{name}_single_scale_ms"] = t_ms[a]
+    out["anchor_latent_gb_per_s"] = n_rows * 200 / (t_ms[3] / 1e3) / 1e9
+    del g2
+    return out
+
+
+def fused_leg(step, args, flush, stream, dist, dev, world):
+    """Scoring + selection of all G layers over the full prefix: G per-layer
+    scans of the shared latent, against one scan with the G layers' absorbed
+    queries stacked (G * H MMA columns; queries from the anchor's hidden state
+    in the training-aware instantiation).  Both from captured graphs, L2
+    flushed before each, CUDA events on the stream."""
+    g, wl = step.g, step.wl
+    step.reset()
+    step.hs_path()                       # absorbed queries of every layer
+    torch.cuda.synchronize()
+
+    def per_layer():
+        for l in range(wl.group):
+            g.score_topk(l)
+
+    times = graph_times([per_layer, g.fused_group_score_topk], args, flush, stream, dist, dev)
     keys = wl.group * int(sum(int(n) for n in step.inp.lengths))
     lat_bytes = int(sum(int(n) for n in step.inp.lengths)) * row_bytes(wl, wl.d_c)
     return {"per_layer_ms": times[0], "fused_ms": times[1], "fused_speedup": times[0] / times[1],
@@ -717,6 +771,10 @@ def main():
     #      latent against one fused scan with the 4 layers' queries stacked
     if not args.no_fused:
         out["paths"]["full_latentindex"] = fused_leg(step, args, flush, stream, dist, dev, world)
+
+    # ---- the two-branch latent in segmented fp8 (the pages' inference format)
+    if not args.no_two_branch:
+        out["paths"]["two_branch_segmented_fp8"] = two_branch_leg(step, args, flush, stream, dist, dev)
 
     # ---- HS against DSA-style at the shorter contexts (same library, same protocol)
     if not args.no_other_contexts:

@@ -167,9 +167,10 @@ __device__ __forceinline__ void transform_row(float (&v)[8], int lane, int64_t p
 // transforms.  E4M3 rows get scale amax / 448 per row, or, with
 // scale_split > 0, one per segment: elements [0, scale_split) and
 // [scale_split, dim), stored as scale[2 row] and scale[2 row + 1].
+template <bool TF>
 __device__ __forceinline__ void write_row(float (&v)[8], int lane, int64_t row, int64_t pos, int dim, int dtype,
                                           int scale_split, const RowTransform& tf, void* data, float* scale) {
-  transform_row(v, lane, pos, tf);
+  if constexpr (TF) transform_row(v, lane, pos, tf);
   if (dtype == LI_F32) {
     float* dst = reinterpret_cast<float*>(data) + row * dim;
 #pragma unroll
@@ -222,7 +223,7 @@ constexpr int kFuseMaxPartials = 16384;   // floats of partial sums (64 KB)
 constexpr int kAppendWarps = 16;          // 512-thread blocks: few arrivals on the completion counter
 constexpr int kStagePer = kFuseMaxPartials / (kAppendWarps * 32);   // partial sums each thread stages
 
-template <typename T>
+template <typename T, bool TF>
 __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T* __restrict__ h,
                                                                       const T* __restrict__ W, int d_model,
                                                                       int dim, int n_tok, int splits,
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
       const int i = lane + 32 * e;
       v[e] = i < dim ? cs[m * dim + i] : 0.f;
     }
-    write_row(v, lane, static_cast<int64_t>(b) * capacity + len + t, len + t, dim, dtype, scale_split, tf, data,
+    write_row<TF>(v, lane, static_cast<int64_t>(b) * capacity + len + t, len + t, dim, dtype, scale_split, tf, data,
               scale);
   }
   __syncthreads();
@@ -329,6 +330,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
 // One warp per new token: write c (fp32 rows) into the cache at row
 // lengths[b] + t0 + t in the cache dtype.  The last block to finish advances
 // lengths[b] by T_total when `bump` is set (all blocks read lengths first).
+template <bool TF>
 __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c, int64_t c_tok_stride,
                                                     int64_t split_stride, int splits,
                                                     int batch, int T_chunk, int t0, int T_total, int bump,
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
         }
         v[e] = x;
       }
-      write_row(v, lane, row, len + t0 + t, dim, dtype, scale_split, tf, data, scale);
+      write_row<TF>(v, lane, row, len + t0 + t, dim, dtype, scale_split, tf, data, scale);
     }
   }
   if (!bump) return;
@@ -612,27 +614,41 @@ bool append_fusable(int n_tok, int dim, int splits) {
   return splits >= 1 && n_tok <= kGemvTok && dim <= 256 && (splits + 1) * n_tok * dim <= kFuseMaxPartials;
 }
 
-cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
-                                int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
-                                int dtype, int scale_split, const RowTransform& tf, unsigned int* done, int* status,
-                                cudaStream_t st) {
+template <bool TF>
+cudaError_t launch_append_fused_tf(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
+                                   int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
+                                   int dtype, int scale_split, const RowTransform& tf, unsigned int* done,
+                                   int* status, cudaStream_t st) {
   const int n_tok = batch * T;
   const int grid = splits * ((dim + kAppendWarps - 1) / kAppendWarps);
   const size_t smem = static_cast<size_t>(splits + 1) * n_tok * dim * sizeof(float);
   cudaError_t e;
   if (h_dtype == LI_BF16) {
-    auto k = gemv_append_kernel<__nv_bfloat16>;
+    auto k = gemv_append_kernel<__nv_bfloat16, TF>;
     if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
     return launch_pdl(k, dim3(grid), dim3(kAppendWarps * 32), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(h),
                       reinterpret_cast<const __nv_bfloat16*>(W), d_model, dim, n_tok, splits, part, batch, T, data,
                       scale, lengths, capacity, dtype, scale_split, tf, done, status);
   } else {
-    auto k = gemv_append_kernel<float>;
+    auto k = gemv_append_kernel<float, TF>;
     if ((e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem))) != cudaSuccess) return e;
     return launch_pdl(k, dim3(grid), dim3(kAppendWarps * 32), smem, st, 1, reinterpret_cast<const float*>(h),
                       reinterpret_cast<const float*>(W), d_model, dim, n_tok, splits, part, batch, T, data, scale,
                       lengths, capacity, dtype, scale_split, tf, done, status);
   }
+}
+
+bool has_transform(const RowTransform& tf) { return tf.rope_dim > 0 || tf.norm_dim > 0; }
+
+cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
+                                int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
+                                int dtype, int scale_split, const RowTransform& tf, unsigned int* done, int* status,
+                                cudaStream_t st) {
+  return has_transform(tf)
+             ? launch_append_fused_tf<true>(h, h_dtype, W, d_model, dim, batch, T, splits, part, data, scale, lengths,
+                                            capacity, dtype, scale_split, tf, done, status, st)
+             : launch_append_fused_tf<false>(h, h_dtype, W, d_model, dim, batch, T, splits, part, data, scale, lengths,
+                                             capacity, dtype, scale_split, tf, done, status, st);
 }
 
 cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t split_stride, int splits, int batch,
@@ -641,9 +657,9 @@ cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t sp
                                 const RowTransform& tf, unsigned int* done_counter, int* status, cudaStream_t st) {
   const int n_tok = batch * T_chunk;
   const int grid = (n_tok + 7) / 8;
-  return launch_pdl(store_kernel, dim3(grid), dim3(256), 0, st, 1, c, c_tok_stride, split_stride, splits, batch, T_chunk,
-                    t0, T_total, bump ? 1 : 0, data, scale, lengths, capacity, dim, dtype, scale_split, tf,
-                    done_counter, status);
+  return launch_pdl(has_transform(tf) ? store_kernel<true> : store_kernel<false>, dim3(grid), dim3(256), 0, st, 1, c,
+                    c_tok_stride, split_stride, splits, batch, T_chunk, t0, T_total, bump ? 1 : 0, data, scale, lengths,
+                    capacity, dim, dtype, scale_split, tf, done_counter, status);
 }
 
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,

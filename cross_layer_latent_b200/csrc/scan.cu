@@ -233,7 +233,7 @@ __device__ __forceinline__ void drain_ring(uint64_t* bars, uint32_t n, uint32_t 
   }
 }
 
-template <int KIND, bool GATHER>
+template <int KIND, bool GATHER, bool SEG>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_constant__ ScanArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -310,8 +310,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const uint32_t k_meta_bytes = a.meta_bytes;
   const int64_t k_score_stride = a.score_stride;
   const float* const k_cache_scale = a.cache_scale;
-  const int k_SK = a.seg_kstep;              // > 0: two scales per row, two accumulators per (slot, M block)
-  const int k_nsc = k_SK > 0 ? 2 : 1;
+  // SEG: two scales per row (segmented fp8), two accumulators per (slot, M block)
+  const int k_SK = SEG ? a.seg_kstep : 0;
+  constexpr int k_nsc = SEG ? 2 : 1;
   const int* const k_lengths = a.lengths;
   const int* const k_q_pos = a.q_pos;
   const float* const k_w = a.w;
@@ -464,7 +465,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           mtok[r] = t;
           if (e4) {
             const int64_t srow = seq_row + (t >= 0 ? t : 0);
-            if (k_nsc == 2) cp_async_8_zfill(smem_addr(mscale + 2 * r), k_cache_scale + 2 * srow, t >= 0 ? 8 : 0);
+            if constexpr (SEG) cp_async_8_zfill(smem_addr(mscale + 2 * r), k_cache_scale + 2 * srow, t >= 0 ? 8 : 0);
             else cp_async_4_zfill(smem_addr(mscale + r), k_cache_scale + srow, t >= 0 ? 4 : 0);
           }
         }
@@ -545,7 +546,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
             const int kc = sp * k_KS + c;
             const uint32_t a_c = a_base + static_cast<uint32_t>(c) * chunk_region;
             const uint32_t b_c = b_base + static_cast<uint32_t>(kc * k_N * k_swz);
-            if (k_SK == 0) {
+            if constexpr (!SEG) {
               issue_chunk_rt<KIND>(static_cast<int>(ksteps), 1, d0, a_c, b_c, desc_hi, 0u,
                                    static_cast<uint32_t>(k_N), k_idesc, kc == 0);
             } else {
@@ -656,7 +657,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         if (GATHER) tok = reinterpret_cast<const int*>(mscale + k_R * k_nsc)[r];
         // rows past the valid prefix read stale values, unused
         if (e4 && tok >= 0) {
-          if (k_nsc == 2) {
+          if constexpr (SEG) {
             cs = mscale[2 * r];
             cs1 = mscale[2 * r + 1];
           } else {
@@ -673,7 +674,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
                                  static_cast<uint32_t>(k_N * k_nsc);
       // segmented scales: head h's product is cs * D0_h + cs1 * D1_h; without
       // a bias cs is factored out (cs > 0) and D0_h + (cs1 / cs) D1_h summed
-      const float rho = k_nsc == 2 ? cs1 / cs : 0.f;
+      float rho = 0.f;
+      if constexpr (SEG) rho = cs1 / cs;
       for (int qi = 0; qi < k_Qg; ++qi) {
         const int t = g * k_Qg + qi;
         if (t >= k_T) break;
@@ -682,7 +684,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         const float* qs = ep_qs + qi * k_H_pad;
         const float* be = ep_beta + qi * k_H_pad;
         int h0 = 0;
-        if (k_nsc == 2) {
+        if constexpr (SEG) {
           for (; h0 + 16 <= k_H_pad; h0 += 16) {
             float v[16], v1[16];
             tmem_load16x2_sync(tbase + static_cast<uint32_t>(qi * k_H_pad + h0),
@@ -745,9 +747,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   if (warp == 1) tmem_dealloc(tmem, a.tmem_cols);
 }
 
-template <int KIND, bool GATHER>
+template <int KIND, bool GATHER, bool SEG = false>
 cudaError_t launch_one(const ScanArgs& a, int grid, cudaStream_t st) {
-  auto k = scan_kernel<KIND, GATHER>;
+  auto k = scan_kernel<KIND, GATHER, SEG>;
   const cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(k), a.smem_bytes);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, dim3(grid), dim3(kScanThreads), a.smem_bytes, st, 1, a);
@@ -761,8 +763,10 @@ cudaError_t launch_scan_kernel(int kind, bool gather, const ScanArgs& a, int gri
     case kKindTF32 * 2 + 1: return launch_one<kKindTF32, true>(a, grid, st);
     case kKindBF16 * 2: return launch_one<kKindBF16, false>(a, grid, st);
     case kKindBF16 * 2 + 1: return launch_one<kKindBF16, true>(a, grid, st);
-    case kKindE4M3 * 2: return launch_one<kKindE4M3, false>(a, grid, st);
-    case kKindE4M3 * 2 + 1: return launch_one<kKindE4M3, true>(a, grid, st);
+    case kKindE4M3 * 2:
+      return a.seg_kstep > 0 ? launch_one<kKindE4M3, false, true>(a, grid, st) : launch_one<kKindE4M3, false>(a, grid, st);
+    case kKindE4M3 * 2 + 1:
+      return a.seg_kstep > 0 ? launch_one<kKindE4M3, true, true>(a, grid, st) : launch_one<kKindE4M3, true>(a, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
