@@ -19,10 +19,13 @@ codecs against torch's bf16 / float8_e4m3fn conversions.  The two-branch
 latent (rope.py: rotary rotation, LayerNorm, native rotated keys) is pinned
 by plane geometry, the rotation group laws, torch's float64 layer_norm and
 the exactness of absorbing frequency-wise complex decoders into post-RoPE
-queries (tests/test_oracle_rope.py).  The pages print no
+queries (tests/test_oracle_rope.py).  The selection-quality metrics
+(recall.py: attention-mass recall per head and of the head average, the
+IndexCache comparator) are pinned by a hand-computed example, a brute force
+over all size-K sets and scipy's softmax (tests/test_oracle_recall.py).  The pages print no
 score values of their own, so the score arithmetic is pinned by hand
 arithmetic and brute force rather than by a published example.
 """
-from . import codecs, counters, indexer, bruteforce, rope
+from . import bruteforce, codecs, counters, indexer, recall, rope
 
-__all__ = ["codecs", "counters", "indexer", "bruteforce", "rope"]
+__all__ = ["codecs", "counters", "indexer", "bruteforce", "recall", "rope"]
