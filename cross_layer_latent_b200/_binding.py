@@ -87,6 +87,8 @@ _sigs = {
     "li_dsa_score_topk": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _I, _P, _P, _P, _P,
                                _SZ, _P]),
     "li_topk": (_I, [_P, _P, _I, _I, _I64, _P, _I, _P, _P, _P, _SZ, _P]),
+    "li_recall_workspace_bytes": (_SZ, [_P, _I, _I, _I, _I]),
+    "li_attention_recall": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "li_set_trace": (_I, [_P, _P, _SZ]),
     "li_profile_enable": (_I, [_P, _I]),
     "li_profile_read": (_I, [_P, ctypes.POINTER(c_li_profile_record), _I, ctypes.POINTER(_I)]),
@@ -318,6 +320,23 @@ def li_topk(ctx: Context, scores: torch.Tensor, k: int, out_idx: torch.Tensor, o
     n = stride if n is None else n
     ctx.check(_lib.li_topk(ctx.handle, _ptr(scores), rows, int(n), int(scores.stride(0)), _ptr(lengths), int(k),
                            _ptr(out_idx), _ptr(out_score), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def li_attention_recall(ctx: Context, probs: torch.Tensor, sel: torch.Tensor, K: int,
+                        lengths: Optional[torch.Tensor] = None, mean: bool = True, ws: Optional[torch.Tensor] = None,
+                        stream=None):
+    """probs [rows, H, N] float32, sel [rows, k] int32 (-1 padded).  Returns
+    (recall [rows, H], mean_recall [rows] or None) as device tensors."""
+    rows, H, N = probs.shape
+    k = sel.shape[-1]
+    need = int(_lib.li_recall_workspace_bytes(ctx.handle, rows, H, N, int(K)))
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=probs.device)
+    rec = torch.empty(rows, H, device=probs.device)
+    mrec = torch.empty(rows, device=probs.device) if mean else None
+    ctx.check(_lib.li_attention_recall(ctx.handle, _ptr(probs), rows, H, N, _ptr(lengths), _ptr(sel), int(k), int(K),
+                                       _ptr(rec), _ptr(mrec), _ptr(ws), ws.numel(), _stream(stream)))
+    return rec, mrec
 
 
 def li_set_trace(ctx: Context, buf: Optional[torch.Tensor]):

@@ -953,6 +953,83 @@ li_status li_topk(li_ctx* c, const float* scores, int rows, int n, int64_t row_s
   return run_topk(c, t, ws, L, st);
 }
 
+// ------------------------------------------------------------------ selection quality
+
+namespace {
+struct RecallLayout {
+  WsLayout L;
+  size_t top_idx, top_val, pbar, total;
+};
+RecallLayout recall_layout(int64_t rows, int64_t H, int64_t N, int64_t K) {
+  RecallLayout R;
+  R.L = ws_layout(rows * H, N, 0);
+  size_t off = R.L.total;
+  auto take = [&](size_t bytes) { size_t o = off; off += up256(bytes); return o; };
+  R.top_idx = take(rows * H * K * 4);
+  R.top_val = take(rows * H * K * 4);
+  R.pbar = take(rows * N * 4);
+  R.total = off;
+  return R;
+}
+}  // namespace
+
+size_t li_recall_workspace_bytes(const li_ctx*, int rows, int H, int N, int K) {
+  if (rows < 1 || H < 1 || N < 1 || K < 1) return 0;
+  return recall_layout(rows, H, N, std::min(K, N)).total;
+}
+
+li_status li_attention_recall(li_ctx* c, const float* probs, int rows, int H, int N, const int32_t* lengths,
+                              const int32_t* sel, int k, int K, float* recall, float* mean_recall, void* ws,
+                              size_t ws_bytes, void* stream) {
+  const char* what = "li_attention_recall";
+  if (!c) return LI_ERR_ARG;
+  if (!probs || !sel || !recall) return fail(c, LI_ERR_ARG, "%s: probs, sel and recall must be non-NULL", what);
+  if (rows < 1 || H < 1 || N < 1 || k < 1 || K < 1)
+    return fail(c, LI_ERR_SHAPE, "%s: rows, H, N, k and K must be >= 1", what);
+  if (static_cast<int64_t>(rows) * H > 65535)
+    return fail(c, LI_ERR_UNSUPPORTED, "%s: rows x H = %lld exceeds 65535", what,
+                static_cast<long long>(rows) * H);
+  const int KK = std::min(K, N);
+  const RecallLayout R = recall_layout(rows, H, N, KK);
+  if (!ws || ws_bytes < R.total)
+    return fail(c, LI_ERR_WORKSPACE, "%s: workspace of %zu bytes, %zu needed", what, ws_bytes, R.total);
+  if (!aligned(ws, 256)) return fail(c, LI_ERR_ALIGN, "%s: workspace must be 256-byte aligned", what);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* top_idx = at<int32_t>(ws, R.top_idx);
+  float* top_val = at<float>(ws, R.top_val);
+  // each head's best size-K mass: the exact top-K of its row
+  TopkArgs t = topk_args(probs, N, rows * H, N, KK);
+  t.lengths = lengths;
+  t.len_div = H;
+  t.out_idx = top_idx;
+  t.out_score = top_val;
+  li_status s = run_topk(c, t, ws, R.L, st);
+  if (s != LI_OK) return s;
+  {
+    Launch Lr(c, st, "recall", 0, 256, 0);
+    const cudaError_t e = launch_recall(probs, rows, H, N, lengths, sel, k, top_idx, top_val, KK, recall, st);
+    Lr.done();
+    if (e != cudaSuccess) return cuda_fail(c, e, "recall launch");
+  }
+  if (!mean_recall) return LI_OK;
+  float* pbar = at<float>(ws, R.pbar);
+  {
+    Launch Lm(c, st, "head_mean", 0, 256, 0);
+    const cudaError_t e = launch_head_mean(probs, rows, H, N, lengths, pbar, c->num_sms, st);
+    Lm.done();
+    if (e != cudaSuccess) return cuda_fail(c, e, "head mean launch");
+  }
+  TopkArgs t2 = topk_args(pbar, N, rows, N, KK);
+  t2.lengths = lengths;
+  t2.out_idx = top_idx;
+  t2.out_score = top_val;
+  if ((s = run_topk(c, t2, ws, R.L, st)) != LI_OK) return s;
+  Launch Lr(c, st, "recall", 0, 256, 0);
+  const cudaError_t e = launch_recall(pbar, rows, 1, N, lengths, sel, k, top_idx, top_val, KK, mean_recall, st);
+  Lr.done();
+  return e == cudaSuccess ? LI_OK : cuda_fail(c, e, "recall launch");
+}
+
 li_status li_set_trace(li_ctx* c, void* buf, size_t bytes) {
   if (!c) return LI_ERR_ARG;
   if (buf && bytes < static_cast<size_t>(kTraceCtas) * kTraceTiles * kTraceEvents * 8)

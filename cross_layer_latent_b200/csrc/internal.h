@@ -182,4 +182,10 @@ cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k,
                           int out_dtype, void* q_abs, float* q_abs_scale, float* beta,
                           cudaStream_t st);
 
+// ---- selection quality
+cudaError_t launch_head_mean(const float* probs, int rows, int H, int N, const int32_t* lengths, float* pbar,
+                             int num_sms, cudaStream_t st);
+cudaError_t launch_recall(const float* vals, int rows, int Hh, int N, const int32_t* lengths, const int32_t* sel,
+                          int k, const int32_t* top_idx, const float* top_val, int K, float* out, cudaStream_t st);
+
 }  // namespace li

@@ -345,6 +345,33 @@ LI_API li_status li_topk(li_ctx* ctx, const float* scores, int rows, int n, int6
                   const int32_t* lengths, int k, int32_t* out_idx, float* out_score, void* ws,
                   size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------ selection quality */
+
+/* Attention-mass recall of a selection (Sec. 4.1 and Table 1; Sec. D.3:
+ * the mass a selection captures relative to each head's own top-K set, from
+ * each layer's dense attention; Sec. C.2: averaged over heads; Sec. C.3:
+ * mean-attention recall against the best shared size-K set of the head
+ * average).  For query row r with valid prefix n_r (lengths[r], or N when
+ * lengths is NULL) and head h:
+ *   recall[r][h] = (sum of probs[r][h][s] over selected s = sel[r][j] with
+ *                   0 <= s < n_r) / (sum of the min(K, n_r) largest
+ *                   probs[r][h][s], s < n_r), or 0 when that sum is 0;
+ *   mean_recall[r] = the same for pbar[r][s] = (sum_h probs[r][h][s]) / H.
+ * The best sets are exact (the library's top-k); masses are summed in fp32.
+ * probs [rows][H][N] fp32 device (entries at s >= n_r are ignored);
+ * sel [rows][k] int32 device, -1 padded (a selection output);
+ * recall [rows][H] fp32 device; mean_recall [rows] fp32 device or NULL.
+ * ws: li_recall_workspace_bytes(ctx, rows, H, N, K) bytes, 256-byte
+ * aligned, zero-filled before first use (status word at offset 0).
+ * Needs rows * H <= 65535.  An IndexCache follower (Sec. 1, Sec. 2) reuses
+ * the anchor's selection unchanged: pass the anchor's out_idx as sel.
+ * Evaluation tooling: no counterpart on the decode path.                  */
+LI_API size_t li_recall_workspace_bytes(const li_ctx* ctx, int rows, int H, int N, int K);
+LI_API li_status li_attention_recall(li_ctx* ctx, const float* probs, int rows, int H, int N,
+                              const int32_t* lengths, const int32_t* sel, int k, int K,
+                              float* recall, float* mean_recall, void* ws, size_t ws_bytes,
+                              void* stream);
+
 /* ------------------------------------------------------------- profiling */
 
 /* Launch profile: when enabled, every kernel launch (and workspace clear) of
