@@ -18,6 +18,7 @@ Multi-GPU: one process per GPU (torchrun); every rank runs the same step on
 its own sequences (weak scaling, no collective on the data path).
 """
 import argparse
+from dataclasses import replace
 import hashlib
 import json
 import math
@@ -51,6 +52,7 @@ def parse():
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-fused", action="store_true")
     p.add_argument("--no-two-branch", action="store_true")
+    p.add_argument("--no-recall", action="store_true")
     return p.parse_args()
 
 
@@ -568,6 +570,76 @@ def two_branch_leg(step, args, flush, stream, dist, dev):
     return out
 
 
+def recall_leg(step, dev):
+    """Selection quality of the step's selectors on a synthetic dense
+    attention (the pages measure recall on real models; weights are out of
+    reach here).  Layer l's attention for head h: the native logits q_h . k_s
+    (keys W_K c from the fp32 latent) standardised over the prefix and
+    sharpened by 2.5 before the softmax.  Selectors: DSA-style (own keys),
+    full LatentIndex, HS, and IndexCache (followers reuse the anchor's
+    selection).  Recall is li_attention_recall: per-head mass over the best
+    size-K mass, and the same for the head average."""
+    li, ctx = step.li, step.ctx
+    # the same workload with layer-specific relevant tokens (1% per layer)
+    # beside the shared ones, so that the layers' best sets differ
+    wl = replace(step.wl, layer_specific_frac=0.01)
+    inp = generate(wl)
+    g = li.GroupIndexer(ctx, batch=wl.batch, capacity=wl.capacity, d_c=wl.d_c, H=wl.heads, d_k=wl.d_k,
+                        G=wl.group, dtype=step.g.dtype, k=wl.k, B=wl.B, dsa=True, device=dev)
+    g.load(inp.lengths, inp.W_K, inp.q, inp.w, latent=inp.latent)
+    lengths = torch.from_numpy(inp.lengths).to(dev)
+    sels = {"dsa": [], "full": [], "hs": [], "index_cache": []}
+    for l in range(wl.group):
+        g.dsa_score_topk(l)
+        sels["dsa"].append(g.idx[l][:, 0].clone())
+        g.score_topk(l)
+        sels["full"].append(g.idx[l][:, 0].clone())
+    g.hs_anchor(0)
+    anchor = g.idx[0][:, 0].clone()
+    sels["hs"].append(anchor)
+    sels["index_cache"].append(anchor)
+    for l in range(1, wl.group):
+        g.hs_follower(l)
+        sels["hs"].append(g.idx[l][:, 0].clone())
+        sels["index_cache"].append(anchor)
+    torch.cuda.synchronize()
+    lat = torch.from_numpy(inp.latent).to(dev)
+    out = {m: {"head_recall": [], "mean_recall": []} for m in sels}
+    ws = None
+    t_ms = []
+    for l in range(wl.group):
+        keys = lat @ torch.from_numpy(inp.W_K[l]).to(dev).T                    # [b, cap, d_k]
+        q = torch.from_numpy(inp.q[l][:, 0]).to(dev)                             # [b, H, d_k]
+        logits = torch.bmm(q, keys.transpose(1, 2))                             # [b, H, cap]
+        del keys
+        z = (logits - logits.mean(dim=2, keepdim=True)) / logits.std(dim=2, keepdim=True)
+        del logits
+        p = torch.softmax(2.5 * z, dim=2).contiguous()
+        del z
+        for m, ss in sels.items():
+            if ws is None:
+                need = li._binding._lib.li_recall_workspace_bytes(ctx.handle, wl.batch, wl.heads, wl.capacity, wl.k)
+                ws = torch.zeros(int(need), dtype=torch.uint8, device=dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            rec, mrec = li.li_attention_recall(ctx, p, ss[l].contiguous(), wl.k, lengths=lengths, ws=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            t_ms.append(e0.elapsed_time(e1))
+            out[m]["head_recall"].append(float(rec.mean()))
+            out[m]["mean_recall"].append(float(mrec.mean()))
+        del p
+    res = {"attention": "synthetic: softmax over the prefix of 2.5 x the standardised native logits q_h . W_K c_s",
+           "workload": f"{wl.name} with 1% of tokens per layer relevant to that layer only",
+           "K": wl.k, "recall_ms": statistics.median(t_ms)}
+    for m, d in out.items():
+        res[m] = {"head_recall": statistics.mean(d["head_recall"]), "mean_recall": statistics.mean(d["mean_recall"]),
+                  "followers_head_recall": statistics.mean(d["head_recall"][1:]),
+                  "by_layer_head_recall": [round(x, 5) for x in d["head_recall"]]}
+    del g
+    return res
+
+
 def fused_leg(step, args, flush, stream, dist, dev, world):
     """Scoring + selection of all G layers over the full prefix: G per-layer
     scans of the shared latent, against one scan with the G layers' absorbed
@@ -775,6 +847,10 @@ def main():
     # ---- the two-branch latent in segmented fp8 (the pages' inference format)
     if not args.no_two_branch:
         out["paths"]["two_branch_segmented_fp8"] = two_branch_leg(step, args, flush, stream, dist, dev)
+
+    # ---- selection quality of the step's selectors (synthetic attention)
+    if not args.no_recall:
+        out["paths"]["recall"] = recall_leg(step, dev)
 
     # ---- HS against DSA-style at the shorter contexts (same library, same protocol)
     if not args.no_other_contexts:

@@ -32,6 +32,7 @@ class Workload:
     planted_frac: float      # fraction of tokens planted with high affinity
     outlier_channels: int = 0     # latent channels multiplied by outlier_mult
     outlier_mult: float = 1.0
+    layer_specific_frac: float = 0.0   # per layer, tokens planted along a direction only that layer favours
     d_model: int = 7168      # hidden width used for latent / key construction
     latent_from_hidden: bool = False   # True: c = W_down h is built by the append step
     queries: int = 1         # query tokens per sequence (1 = decode)

@@ -15,6 +15,10 @@ Recipe (all draws from ``numpy.random.default_rng(seed)``, float32):
 * Decoders W_K[l] = (G_l + sqrt(d_c) * v_l u^T) / sqrt(d_k), G_l ~ N(0, 1):
   Gaussian plus a rank-one spike that maps the latent direction u onto the
   key direction v_l.
+* Optional layer-specific relevance (``layer_specific_frac``): each layer's
+  decoder gains a second spike from its own direction u_l (orthogonal to u)
+  to the key direction that u already reaches, and that fraction of each
+  sequence's tokens is planted along u_l, relevant to layer l only.
 * Head weights w[l] ~ N(0, 1/sqrt(H)) (std); queries
   q[l] = (g + 2 sign(w[l]) v_l) / sqrt(d_k), g ~ N(0, 1), so heads with
   positive weight lean toward +v_l and heads with negative weight toward -v_l.
@@ -117,6 +121,24 @@ def generate(wl, seed: Optional[int] = None) -> Inputs:
         if latent is not None:
             latent[:, :, outl] *= np.float32(wl.outlier_mult)
         # (workloads built from h carry no outlier channels)
+
+    if wl.layer_specific_frac > 0 and latent is not None:
+        # Layer-specific relevance: layer l's decoder also maps a direction
+        # u_l (orthogonal to u) onto its key direction v_l, and a fraction of
+        # tokens per sequence is planted along u_l, so they matter to layer l
+        # only.  A separate stream keeps the other draws unchanged.
+        rl = np.random.default_rng(wl.seed + 3000)
+        s = 1.0 / math.sqrt(wl.d_model)
+        for l in range(G):
+            ul = rl.standard_normal(dc)
+            ul = _unit(ul - (ul @ u) * u)
+            # the key direction u already reaches (the queries lean toward it)
+            v = _unit(W_K[l].astype(np.float64) @ u.astype(np.float64))
+            W_K[l] = (W_K[l] + math.sqrt(dc) * np.outer(v, ul) / math.sqrt(dk)).astype(np.float32)
+            for i in range(b):
+                n_l = int(math.ceil(wl.layer_specific_frac * int(lengths[i])))
+                idx = rl.choice(int(lengths[i]), size=n_l, replace=False)
+                latent[i, idx, :] += np.float32(3.0 * s * math.sqrt(dc)) * ul
 
     q_pos = None
     if T > 1:
