@@ -463,6 +463,7 @@ li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, boo
     return fail(ctx, LI_ERR_SHAPE, "%s: scanning an E4M3 cache needs capacity %% 4 == 0 (got %d)", what,
                 c->capacity);
   a.cache_scale = c->dtype == LI_E4M3 ? c->scale : nullptr;
+  a.cache_data = static_cast<const uint8_t*>(c->data);
   a.lengths = c->lengths;
   a.q_pos = q->q_pos;
   a.w = q->w;

@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const T* __restri
                                                                int dim, int n_tok, int splits,
                                                                float* __restrict__ out) {
   pdl_begin();
+  pdl_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int task = blockIdx.x * kGemvWarps + warp;
   if (task >= dim * splits) return;
@@ -233,6 +234,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
                                                                       RowTransform tf, unsigned int* done,
                                                                       int* status) {
   pdl_begin();
+  pdl_release();
   extern __shared__ __align__(16) float ps[];       // [splits][n_tok * dim], then cs [n_tok * dim]
   __shared__ unsigned last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -338,6 +340,7 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
                                                     int capacity, int dim, int dtype, int scale_split,
                                                     RowTransform tf, unsigned int* done, int* status) {
   pdl_begin();
+  pdl_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok = blockIdx.x * 8 + warp;
   if (tok < batch * T_chunk) {
@@ -402,6 +405,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(const T* __restrict__ q, in
                                                      int out_dtype, void* q_abs, float* q_abs_scale,
                                                      float* beta) {
   pdl_begin();
+  pdl_release();
   __shared__ float qs[kAbsorbHeads][256];
   __shared__ float red[8][kAbsorbHeads];
   const int t = blockIdx.y, h0 = blockIdx.x * kAbsorbHeads;
@@ -505,6 +509,7 @@ __global__ void __launch_bounds__(256) absorb_shared_kernel(const T* __restrict_
                                                             int out_dtype, void* q_abs, float* q_abs_scale,
                                                             float* beta) {
   pdl_begin();
+  pdl_release();
   extern __shared__ __align__(16) unsigned char absorb_smem[];
   T* Ws = reinterpret_cast<T*>(absorb_smem);                                   // [d_k][d_c]
   float* qs = reinterpret_cast<float*>(absorb_smem + (static_cast<size_t>(d_k) * d_c * sizeof(T) + 15) / 16 * 16);

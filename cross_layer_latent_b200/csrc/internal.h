@@ -27,6 +27,7 @@ struct alignas(64) ScanArgs {
   CUtensorMap map_a;          // cache rows: dims {swz/elt, batch*capacity, n_kchunks}, box {swz/elt, R, KS};
                               // gather: dims {dim, batch*capacity}, box {swz/elt, 1}
   CUtensorMap map_b;          // queries: dims {dim, H, batch*T}, box {swz/elt, H_pad, Qg}
+  const uint8_t* cache_data;  // [batch*capacity][row_bytes] (the rows the cache map covers)
   const float* cache_scale;   // [batch*capacity] (segmented: [batch*capacity][2]) or null
   const int* lengths;         // [batch]
   const int* q_pos;           // [batch*T] or null

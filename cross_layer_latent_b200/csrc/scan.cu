@@ -265,6 +265,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     tmem_alloc(s.tmem_base, a.tmem_cols);
     tmem_relinquish();
   }
+  if (!GATHER && warp == 2 && lane == 0 && a.q_pos == nullptr) {
+    // Until the lengths are visible the CTA cannot know its first items; it
+    // guesses them from full-capacity segments (exact when every sequence
+    // is full) and prefetches their rows and scales into L2, so that the
+    // first tile loads after the prologue hit L2 instead of HBM.
+    const int ips = (a.capacity + a.R - 1) / a.R;
+    const int64_t total = static_cast<int64_t>(a.n_segments) * ips;
+    const int64_t b0 = total * blockIdx.x / gridDim.x, b1 = total * (blockIdx.x + 1) / gridDim.x;
+    const int nsc = SEG ? 2 : 1;
+    for (int64_t item = b0; item < b1 && item < b0 + 2; ++item) {
+      const int seg = static_cast<int>(item / ips), it = static_cast<int>(item % ips);
+      const int64_t row0 = static_cast<int64_t>(seg / a.n_groups) * a.capacity + static_cast<int64_t>(it) * a.R;
+      const int rows = min(a.R, a.capacity - it * a.R);
+      prefetch_l2_bulk(a.cache_data + row0 * a.row_bytes, static_cast<uint32_t>(rows * a.row_bytes));
+      if (a.cache_scale) prefetch_l2_bulk(a.cache_scale + row0 * nsc, static_cast<uint32_t>(rows * 4 * nsc));
+    }
+  }
   // everything above touches only this CTA's own resources; the lengths,
   // queries and cache rows below may come from the previous kernel
   pdl_begin();
@@ -350,6 +367,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         const bool moved = w.to(item) || first;
         first = false;
         const int it = item - s.prefix[w.seg];   // item index within the segment
+        // The item's first stage of rows goes first (the long HBM round
+        // trip), then its queries and scales, then its other stages.  The
+        // queries must precede the second stage: the MMA issuer cannot free
+        // a stage of this item before it has them, and the ring may hold
+        // fewer stages than an item has.
+        const int row0 = w.b * k_capacity + it * k_R;
+        auto load_stage = [&](int sp) -> bool {
+          if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) return false;
+          if (sp == 0) trace_event(k_trace, lt, 0);
+          mbar_arrive_expect_tx(&s.full[st.i], k_a_stage_bytes);
+          tma_load_3d(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes, &a.map_a, &s.full[st.i], 0, row0,
+                      sp * k_KS);
+          st.step(S);
+          ++n_st;
+          return true;
+        };
+        if (!load_stage(0)) break;
         if (moved) {
           if (!bounded_wait(&s.bempty[bs.i], bs.ph ^ 1u, wc)) break;
           mbar_arrive_expect_tx(&s.bfull[bs.i], k_b_slot_bytes);
@@ -374,17 +408,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           ms.step(NM);
           ++n_ms;
         }
-        const int row0 = w.b * k_capacity + it * k_R;
         bool ok = true;
-        for (int sp = 0; sp < k_spi; ++sp) {
-          if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
-          if (sp == 0) trace_event(k_trace, lt, 0);
-          mbar_arrive_expect_tx(&s.full[st.i], k_a_stage_bytes);
-          tma_load_3d(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes, &a.map_a, &s.full[st.i], 0, row0,
-                      sp * k_KS);
-          st.step(S);
-          ++n_st;
-        }
+        for (int sp = 1; sp < k_spi && ok; ++sp) ok = load_stage(sp);
         if (!ok) break;
         trace_event(k_trace, lt, 1);
       }

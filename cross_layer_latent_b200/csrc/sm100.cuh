@@ -157,12 +157,17 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 // Every kernel of the library is launched with programmatic stream
 // serialisation, so it may start while the previous kernel on the stream is
 // finishing.  pdl_begin() waits until that kernel has completed and its
-// memory is visible (no global memory is touched before it).  Dependents
-// are not released early: they launch as this kernel's CTAs exit (released
-// early, a waiting dependent that fits beside this kernel's CTAs shares
-// their SMs and slows them down).  Without the launch attribute it is a
-// no-op.
+// memory is visible (no global memory is touched before it).  The scan and
+// selection kernels do not release their dependents early: those launch as
+// their CTAs exit (released early, a waiting dependent that fits beside
+// their CTAs shares the SMs and slows them down).  The short construction
+// kernels release them right after their own wait (pdl_release), so the
+// next kernel's CTAs set up their barriers, tensor memory and L2 prefetches
+// while the construction finishes; everything before a kernel's own wait
+// is then complete, since the release follows that wait.  Without the
+// launch attribute both are no-ops.
 __device__ __forceinline__ void pdl_begin() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------------ TMA
 
@@ -193,6 +198,13 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst_smem, const CUtensorMap
 
 // Arrive on `bar` once every cp.async this thread has issued so far has
 // landed (the arrival counts toward the barrier's expected count).
+// Bulk prefetch of [src, src + bytes) into L2 (a hint: no data returns, so
+// it may run before the previous kernel's writes are visible; L2 keeps any
+// later write coherent).  src and bytes must be multiples of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
