@@ -549,7 +549,7 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   // The cluster kernel minimises latency for a few rows; once its CTAs
   // (rows x cluster size) exceed about one wave, the chunked path, which
   // spreads every row over many small blocks, has the better throughput.
-  const int64_t cs = std::min<int64_t>(kClusterMaxSize, std::max<int64_t>(1, (t.n + 8191) / 8192));
+  const int64_t cs = topk_cluster_size(t.n);
   if (t.n <= kClusterMaxN && static_cast<int64_t>(t.rows) * cs <= 2 * static_cast<int64_t>(ctx->num_sms)) {
     int cs = 0;
     Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);

@@ -136,6 +136,7 @@ struct TopkArgs {
 constexpr int kClusterThreads = 512;
 constexpr int kClusterMaxSize = 8;
 constexpr int kClusterMaxN = kClusterThreads * 32 * kClusterMaxSize;   // 131072
+int topk_cluster_size(int64_t n);   // CTAs per row of the single-launch selection
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size);
 
 constexpr int kTopkChunk = 4096;

@@ -698,10 +698,17 @@ cudaError_t launch_radix_pt(const TopkArgs& a, int cs, cudaStream_t st) {
 
 }  // namespace
 
+int topk_cluster_size(int64_t n) {
+  // As many CTAs as keep 4 keys a thread, up to a cluster of 8: short rows
+  // (the 8192 candidates of hierarchical selection) are latency-bound, and
+  // spreading them over more CTAs shortens every pass.
+  int64_t cs = (n + kClusterThreads * 4 - 1) / (kClusterThreads * 4);
+  return static_cast<int>(cs < 1 ? 1 : (cs > kClusterMaxSize ? kClusterMaxSize : cs));
+}
+
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size) {
   const int64_t n = a.n;
-  int cs = static_cast<int>((n + kClusterThreads * 16 - 1) / (kClusterThreads * 16));
-  cs = cs < 1 ? 1 : (cs > kClusterMaxSize ? kClusterMaxSize : cs);
+  const int cs = topk_cluster_size(n);
   const int64_t per_thread = (n + static_cast<int64_t>(cs) * kClusterThreads - 1) / (static_cast<int64_t>(cs) * kClusterThreads);
   if (cluster_size) *cluster_size = cs;
   if (per_thread <= 4) return launch_radix_pt<4>(a, cs, st);
