@@ -391,4 +391,10 @@ __device__ __forceinline__ uint32_t radix_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float a key came from (-0.0 comes back as +0.0, the value it was
+// ranked as).
+__device__ __forceinline__ float radix_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 }  // namespace li

@@ -676,7 +676,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
         if (rank < a.k) {
           const int64_t pos = run + j * 128 + 4 * lane + e;
           oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
-          if (osv) osv[rank] = row[pos];
+          if (osv) osv[rank] = radix_value(key[4 * j + e]);   // no reload: the key is the score
         }
       }
       g += gt ? 1 : 0;

@@ -41,7 +41,8 @@
  *   k_eff = min(k, n) positions with the largest scores, ordered by (score
  *   descending, position ascending) to decide who is in, and written in
  *   ascending position order; slots k_eff..k-1 hold -1 (indices) and -inf
- *   (scores).  -0.0 ranks equal to +0.0.  NaN scores are invalid input.
+ *   (scores).  -0.0 ranks equal to +0.0, and a selected -0.0 score may be
+ *   returned as +0.0.  NaN scores are invalid input.
  * Valid prefix.  In decode (q_pos == NULL) the query of sequence b sees
  *   positions [0, lengths[b]) -- the current token is appended before it
  *   scores.  With q_pos, query (b, t) sees [0, min(lengths[b], q_pos[b][t]+1)).
