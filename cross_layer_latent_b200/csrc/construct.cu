@@ -107,6 +107,28 @@ __device__ __forceinline__ float warp_max(float x) {
   return x;
 }
 
+// Per-lane constants of the row transforms (the same for every row): the
+// LayerNorm affine terms and the rotary frequency of each element the lane
+// holds.  Loaded once per warp, before the rows are ready, so that no global
+// read sits between a row's reduction and its store.
+struct TfLane {
+  float g[8], b[8], f[8];
+};
+
+__device__ __forceinline__ TfLane load_tf_lane(const RowTransform& tf, int lane) {
+  TfLane t;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int i = lane + 32 * e;
+    const bool in_norm = tf.norm_dim > 0 && i >= tf.norm_offset && i < tf.norm_offset + tf.norm_dim;
+    const bool in_rope = tf.rope_dim > 0 && i >= tf.rope_offset && i < tf.rope_offset + tf.rope_dim;
+    t.g[e] = in_norm && tf.gamma ? __ldg(tf.gamma + (i - tf.norm_offset)) : 1.f;
+    t.b[e] = in_norm && tf.beta ? __ldg(tf.beta + (i - tf.norm_offset)) : 0.f;
+    t.f[e] = in_rope ? __ldg(tf.inv_freq + ((i - tf.rope_offset) >> 1) / tf.rope_sources) : 0.f;
+  }
+  return t;
+}
+
 // The two-branch latent's row transforms (LatentIndex summary, Sec. 3.1,
 // Sec. A.2, Sec. D.2) on one fp32 row held by a warp (lane holds elements
 // lane + 32 e): LayerNorm of the NoPE range (biased variance, correctly
@@ -115,7 +137,8 @@ __device__ __forceinline__ float warp_max(float x) {
 // pos * inv_freq[p / sources], the angle formed exactly and its cosine and
 // sine taken in double precision, then rounded to fp32.  Slot partners are
 // adjacent lanes (the range starts on an even element).
-__device__ __forceinline__ void transform_row(float (&v)[8], int lane, int64_t pos, const RowTransform& tf) {
+__device__ __forceinline__ void transform_row(float (&v)[8], int lane, int64_t pos, const RowTransform& tf,
+                                              const TfLane& c) {
   if (tf.norm_dim > 0) {
     const int a = tf.norm_offset, b = tf.norm_offset + tf.norm_dim;
     float s = 0.f;
@@ -138,12 +161,7 @@ __device__ __forceinline__ void transform_row(float (&v)[8], int lane, int64_t p
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = lane + 32 * e;
-      if (i >= a && i < b) {
-        float y = __fdiv_rn(v[e] - mean, sd);
-        if (tf.gamma) y *= __ldg(tf.gamma + (i - a));
-        if (tf.beta) y += __ldg(tf.beta + (i - a));
-        v[e] = y;
-      }
+      if (i >= a && i < b) v[e] = __fdiv_rn(v[e] - mean, sd) * c.g[e] + c.b[e];
     }
   }
   if (tf.rope_dim > 0) {
@@ -153,11 +171,10 @@ __device__ __forceinline__ void transform_row(float (&v)[8], int lane, int64_t p
       const int i = lane + 32 * e;
       const float partner = __shfl_xor_sync(0xffffffffu, v[e], 1);
       if (i >= a && i < b) {
-        const int f = ((i - a) >> 1) / tf.rope_sources;
         double sn, cs;
-        sincos(static_cast<double>(pos) * static_cast<double>(__ldg(tf.inv_freq + f)), &sn, &cs);
-        const float c = static_cast<float>(cs), sf = static_cast<float>(sn);
-        v[e] = ((i - a) & 1) == 0 ? v[e] * c - partner * sf : partner * sf + v[e] * c;
+        sincos(static_cast<double>(pos) * static_cast<double>(c.f[e]), &sn, &cs);
+        const float co = static_cast<float>(cs), si = static_cast<float>(sn);
+        v[e] = ((i - a) & 1) == 0 ? v[e] * co - partner * si : partner * si + v[e] * co;
       }
     }
   }
@@ -170,8 +187,9 @@ __device__ __forceinline__ void transform_row(float (&v)[8], int lane, int64_t p
 // [scale_split, dim), stored as scale[2 row] and scale[2 row + 1].
 template <bool TF>
 __device__ __forceinline__ void write_row(float (&v)[8], int lane, int64_t row, int64_t pos, int dim, int dtype,
-                                          int scale_split, const RowTransform& tf, void* data, float* scale) {
-  if constexpr (TF) transform_row(v, lane, pos, tf);
+                                          int scale_split, const RowTransform& tf, const TfLane& tc, void* data,
+                                          float* scale) {
+  if constexpr (TF) transform_row(v, lane, pos, tf, tc);
   if (dtype == LI_F32) {
     float* dst = reinterpret_cast<float*>(data) + row * dim;
 #pragma unroll
@@ -278,6 +296,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
   }
   __syncthreads();
   if (!last) return;
+  TfLane tc;
+  if constexpr (TF) tc = load_tf_lane(tf, threadIdx.x & 31);
   __threadfence();
   const int nx = n_tok * dim, np = splits * nx;   // np <= kStagePer * blockDim.x
   {
@@ -315,8 +335,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
       const int i = lane + 32 * e;
       v[e] = i < dim ? cs[m * dim + i] : 0.f;
     }
-    write_row<TF>(v, lane, static_cast<int64_t>(b) * capacity + len + t, len + t, dim, dtype, scale_split, tf, data,
-              scale);
+    write_row<TF>(v, lane, static_cast<int64_t>(b) * capacity + len + t, len + t, dim, dtype, scale_split, tf, tc,
+                  data, scale);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -342,6 +362,8 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
   pdl_begin();
   pdl_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  TfLane tc;
+  if constexpr (TF) tc = load_tf_lane(tf, lane);
   const int tok = blockIdx.x * 8 + warp;
   if (tok < batch * T_chunk) {
     const int b = tok / T_chunk, t = tok % T_chunk;
@@ -368,7 +390,7 @@ __global__ void __launch_bounds__(256) store_kernel(const float* __restrict__ c,
         }
         v[e] = x;
       }
-      write_row<TF>(v, lane, row, len + t0 + t, dim, dtype, scale_split, tf, data, scale);
+      write_row<TF>(v, lane, row, len + t0 + t, dim, dtype, scale_split, tf, tc, data, scale);
     }
   }
   if (!bump) return;
