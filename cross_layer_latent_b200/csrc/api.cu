@@ -546,14 +546,18 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   t.cand = at<uint2>(ws, L.cand);
   if (static_cast<int64_t>(t.rows) * t.n > static_cast<int64_t>((L.scores - L.cand) / 8))
     return fail(ctx, LI_ERR_WORKSPACE, "selection of %d x %d exceeds the workspace candidate buffer", t.rows, t.n);
-  // The cluster kernel minimises latency for a few rows; once its CTAs
-  // (rows x cluster size) exceed about one wave, the chunked path, which
-  // spreads every row over many small blocks, has the better throughput.
-  const int64_t cs = topk_cluster_size(t.n);
-  if (t.n <= kClusterMaxN && static_cast<int64_t>(t.rows) * cs <= 2 * static_cast<int64_t>(ctx->num_sms)) {
+  // Rows of up to kClusterMaxN positions take the single-launch cluster
+  // kernel: sized for latency while its CTAs (rows x cluster size) stay
+  // within about one wave, for throughput beyond (measured on 1024 x 65536:
+  // 467 us, against 566 us for the chunked multi-kernel path).
+  if (t.rows > 65535) return fail(ctx, LI_ERR_UNSUPPORTED, "more than 65535 selection rows");
+  if (t.n <= kClusterMaxN) {
+    const int64_t cs_lat = topk_cluster_size(t.n, kTopkKeysLatency);
+    const int kpt = static_cast<int64_t>(t.rows) * cs_lat <= 2 * static_cast<int64_t>(ctx->num_sms)
+                        ? kTopkKeysLatency : kTopkKeysThroughput;
     int cs = 0;
     Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);
-    const cudaError_t e = launch_topk_cluster(t, st, &cs);
+    const cudaError_t e = launch_topk_cluster(t, st, &cs, kpt);
     Lc.grid = cs * t.rows;
     Lc.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster");

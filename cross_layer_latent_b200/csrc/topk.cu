@@ -698,17 +698,20 @@ cudaError_t launch_radix_pt(const TopkArgs& a, int cs, cudaStream_t st) {
 
 }  // namespace
 
-int topk_cluster_size(int64_t n) {
-  // As many CTAs as keep 4 keys a thread, up to a cluster of 8: short rows
-  // (the 8192 candidates of hierarchical selection) are latency-bound, and
-  // spreading them over more CTAs shortens every pass.
-  int64_t cs = (n + kClusterThreads * 4 - 1) / (kClusterThreads * 4);
+int topk_cluster_size(int64_t n, int keys_per_thread) {
+  // As many CTAs as keep `keys_per_thread` keys a thread, up to a cluster of
+  // 8.  A few rows (decode) are latency-bound: 4 keys a thread spreads them
+  // over more CTAs and shortens every pass.  Many rows (a prefill chunk)
+  // fill the GPU many times over: 32 keys a thread means fewer CTAs, each
+  // paying the per-pass overhead once for more keys.
+  int64_t cs = (n + static_cast<int64_t>(kClusterThreads) * keys_per_thread - 1) /
+               (static_cast<int64_t>(kClusterThreads) * keys_per_thread);
   return static_cast<int>(cs < 1 ? 1 : (cs > kClusterMaxSize ? kClusterMaxSize : cs));
 }
 
-cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size) {
+cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size, int keys_per_thread) {
   const int64_t n = a.n;
-  const int cs = topk_cluster_size(n);
+  const int cs = topk_cluster_size(n, keys_per_thread);
   const int64_t per_thread = (n + static_cast<int64_t>(cs) * kClusterThreads - 1) / (static_cast<int64_t>(cs) * kClusterThreads);
   if (cluster_size) *cluster_size = cs;
   if (per_thread <= 4) return launch_radix_pt<4>(a, cs, st);
