@@ -28,6 +28,8 @@
 // CTA is persistent over a contiguous range of items; a segment is one
 // (sequence, query group) of the scan or one (sequence, query) of the gather.
 // Every wait is bounded; ring positions advance without integer division.
+#include <type_traits>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -233,7 +235,7 @@ __device__ __forceinline__ void drain_ring(uint64_t* bars, uint32_t n, uint32_t 
   }
 }
 
-template <int KIND, bool GATHER, bool SEG>
+template <int KIND, bool GATHER, bool SEG, bool MQ>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_constant__ ScanArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -701,7 +703,56 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       // a bias cs is factored out (cs > 0) and D0_h + (cs1 / cs) D1_h summed
       float rho = 0.f;
       if constexpr (SEG) rho = cs1 / cs;
-      for (int qi = 0; qi < k_Qg; ++qi) {
+      // One score: the head sums of query row qi from its HP columns at vq,
+      // in the same order as the per-query loop below (so results agree bit
+      // for bit whichever path runs), then the store.
+      auto finish = [&](int qi, const float* vq, auto hp) {
+        constexpr int HP = decltype(hp)::value;
+        const int t = g * k_Qg + qi;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* wq = ep_w + qi * k_H_pad;
+        const float* qs = ep_qs + qi * k_H_pad;
+        const float* be = ep_beta + qi * k_H_pad;
+#pragma unroll
+        for (int h0 = 0; h0 < HP; h0 += 16) {
+          if (!has_beta) relu_dot16(vq + h0, wq + h0, part);
+          else relu_dot16_beta(vq + h0, wq + h0, qs + h0, be + h0, cs, part);
+        }
+        float sc = (part[0] + part[1]) + (part[2] + part[3]);
+        if (!has_beta && e4) sc *= cs;
+        if (row_in_item && j < ep_len[qi]) {
+          if (GATHER && tok < 0) {
+            sc = -INFINITY;
+            record_status(k_status, kStatusIndex);
+          }
+          const int64_t row = static_cast<int64_t>(b) * k_T + t;
+          k_scores[row * k_score_stride + j] = sc;
+        }
+      };
+      // Several query rows per item (prefill, a stacked group): their columns
+      // come 64 at a time under one wait, since the epilogue is then bound by
+      // the latency of tensor-memory loads rather than by arithmetic.
+      // (MQ: Qg > 1, H_pad of 16, 32 or 64, N a multiple of 64, no segments)
+      if constexpr (MQ) {
+        {
+          for (int q0 = 0; q0 < k_Qg && g * k_Qg + q0 < k_T; q0 += 64 / k_H_pad) {
+            float v[64];
+            tmem_load64_sync(tbase + static_cast<uint32_t>(q0 * k_H_pad), v);
+            const int nq = min(64 / k_H_pad, k_T - (g * k_Qg + q0));
+            if (k_H_pad == 64) {
+              finish(q0, v, std::integral_constant<int, 64>{});
+            } else if (k_H_pad == 32) {
+              finish(q0, v, std::integral_constant<int, 32>{});
+              if (nq > 1) finish(q0 + 1, v + 32, std::integral_constant<int, 32>{});
+            } else {
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (u < nq) finish(q0 + u, v + 16 * u, std::integral_constant<int, 16>{});
+            }
+          }
+        }
+      }
+      for (int qi = 0; qi < k_Qg && !MQ; ++qi) {
         const int t = g * k_Qg + qi;
         if (t >= k_T) break;
         float part[4] = {0.f, 0.f, 0.f, 0.f};
@@ -774,7 +825,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
 
 template <int KIND, bool GATHER, bool SEG = false>
 cudaError_t launch_one(const ScanArgs& a, int grid, cudaStream_t st) {
-  auto k = scan_kernel<KIND, GATHER, SEG>;
+  // several query rows per item with head groups of 16, 32 or 64: the
+  // epilogue variant that reads 64 columns per tensor-memory wait
+  if constexpr (!GATHER && !SEG) {
+    if (a.Qg > 1 && (a.H_pad == 16 || a.H_pad == 32 || a.H_pad == 64) && a.N % 64 == 0) {
+      auto k = scan_kernel<KIND, false, false, true>;
+      const cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(k), a.smem_bytes);
+      if (e != cudaSuccess) return e;
+      return launch_pdl(k, dim3(grid), dim3(kScanThreads), a.smem_bytes, st, 1, a);
+    }
+  }
+  auto k = scan_kernel<KIND, GATHER, SEG, false>;
   const cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(k), a.smem_bytes);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, dim3(grid), dim3(kScanThreads), a.smem_bytes, st, 1, a);
