@@ -365,9 +365,9 @@ li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, boo
   // metadata ring never throttles the stage ring; then more query slots.
   const bool has_meta = gather || c->dtype == LI_E4M3;
   const int ep_stride = (q->beta ? 3 * N : N) + 16;
-  // barriers (2 x kMaxStages + 2 + 2 + 8 + 8 + 2 x kMetaSlots + 2) x 8 B,
+  // barriers (3 x kMaxStages + 2 + 2 + 8 + 8 + 2 x kMetaSlots + 2) x 8 B,
   // tensor-memory base, abort flag, prefix, epilogue parameters, gather limits
-  const size_t fixed_misc = static_cast<size_t>(2 * kMaxStages + 22 + 2 * kMetaSlots) * 8 + 16 +
+  const size_t fixed_misc = static_cast<size_t>(3 * kMaxStages + 22 + 2 * kMetaSlots) * 8 + 16 +
                             static_cast<size_t>(n_seg + 1) * 4 + 16 + static_cast<size_t>(kEpiWarps) * ep_stride * 4 +
                             (gather ? static_cast<size_t>(2 * n_seg) * 4 : 0) + 64;
   const size_t budget = static_cast<size_t>(ctx->max_smem_optin) - 1024;

@@ -12,9 +12,11 @@ namespace li {
 constexpr int kTileM = 128;          // cache rows per MMA tile (UMMA M)
 constexpr int kEpiWarps = 8;         // two epilogue warpgroups, alternating tiles
 // warp 0 loads, warps 1 and 2 + kEpiWarps issue the MMAs of the two M blocks,
-// warps 2 .. 1 + kEpiWarps run the epilogue
-constexpr int kScanThreads = 96 + 32 * kEpiWarps;
+// warps 2 .. 1 + kEpiWarps run the epilogue, warp 3 + kEpiWarps issues half
+// of the row gathers (gather variant; idle in the scan)
+constexpr int kScanThreads = 128 + 32 * kEpiWarps;
 constexpr int kMmaWarp2 = 2 + kEpiWarps;
+constexpr int kGatherWarp2 = 3 + kEpiWarps;
 constexpr int kMetaSlots = 8;        // ring of per-item row metadata (fp8 scales, gathered rows)
 constexpr int kMaxItemRows = 256;    // rows of one work item (two M=128 MMA blocks)
 constexpr int kMaxSegments = 1024;   // (sequence, query group) segments per scan launch

@@ -52,6 +52,7 @@ struct ScanSmem {
   uint64_t* mfull;
   uint64_t* mempty;
   uint64_t* drain;
+  uint64_t* ready;      // gather: [stage] the first loader has armed the stage and published its rows
   uint32_t* tmem_base;
   int* abort_flag;
   int* prefix;          // [n_segments + 1]
@@ -77,7 +78,8 @@ __device__ __forceinline__ ScanSmem carve(uint8_t* base, const ScanArgs& a) {
   s.mfull = s.accempty + 8;
   s.mempty = s.mfull + kMetaSlots;
   s.drain = s.mempty + kMetaSlots;        // one per MMA issuer
-  s.tmem_base = reinterpret_cast<uint32_t*>(s.drain + 2);
+  s.ready = s.drain + 2;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.ready + kMaxStages);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
   s.prefix = s.abort_flag + 2;
   // 16-byte aligned parameter arrays (read four at a time)
@@ -246,7 +248,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
 
   if (tid == 0) {
     // every MMA issuer (one per M block) releases stages and query slots
-    for (int i = 0; i < a.n_stages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], a.MB); }
+    for (int i = 0; i < a.n_stages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], a.MB);
+      mbar_init(&s.ready[i], 1);
+    }
     for (int i = 0; i < a.n_bslots; ++i) { mbar_init(&s.bfull[i], 1); mbar_init(&s.bempty[i], a.MB); }
     // accumulator (slot, M block): one issuer fills it, one warpgroup drains it
     for (int i = 0; i < 2 * a.n_acc; ++i) { mbar_init(&s.accfull[i], 1); mbar_init(&s.accempty[i], 4); }
@@ -499,15 +505,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       }
       cp_async_arrive_noinc(&s.mfull[ms.i]);
       mbar_arrive(&s.mfull[ms.i]);
+      __threadfence_block();                       // the token ids, for the second loader warp
       __syncwarp();
       ms.step(NM);
       bool ok = true;
       for (int sp = 0; sp < k_spi; ++sp) {
         if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
-        if (lane == 0) mbar_arrive_expect_tx(&s.full[st.i], stage_tx);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&s.full[st.i], stage_tx);   // both warps' copies land on it
+          mbar_arrive(&s.ready[st.i]);
+        }
         __syncwarp();
         const uint32_t stage = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
-        for (int u = lane; u < groups * k_KS; u += 32) {
+        // one TMA operation costs its issuing warp ~74 cycles: the second
+        // loader warp issues the upper half of the stage's gathers
+        for (int u = lane; u < (groups * k_KS + 1) / 2; u += 32) {
           const int c = u / groups, r0 = 4 * (u - c * groups);
           const int t0 = mtok[r0], t1 = mtok[r0 + 1], t2 = mtok[r0 + 2], t3 = mtok[r0 + 3];
           tma_gather4(stage + static_cast<uint32_t>(c) * chunk_region + static_cast<uint32_t>(r0 * k_swz), &a.map_a,
@@ -525,6 +537,39 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       if (lane == 0) {
         drain_ring(s.full, S, n_st);
         drain_ring(s.bfull, NB, n_bs);
+      }
+    }
+  } else if (warp == kGatherWarp2) {
+    // ------------------------------------------------------------ second gather loader, 32 lanes
+    // Follows the first loader item by item and stage by stage: once a stage
+    // is armed and the item's token ids are published (ready), it issues the
+    // upper half of the stage's row gathers onto the same barrier.
+    if constexpr (GATHER) {
+      Ring st, ms;
+      SegWalk w{s.prefix, n_groups};
+      const int groups = k_RI >> 2;
+      const int nops = groups * k_KS, half = (nops + 1) / 2;
+      for (int item = begin; item < end; ++item) {
+        if (*s.abort_flag) break;
+        w.to(item);
+        const int* mtok = reinterpret_cast<const int*>(
+            reinterpret_cast<const float*>(s.meta + static_cast<size_t>(ms.i) * k_meta_bytes) + k_R * k_nsc);
+        const int seq_row = w.b * k_capacity;
+        bool ok = true;
+        for (int sp = 0; sp < k_spi; ++sp) {
+          if (!bounded_wait(&s.ready[st.i], st.ph, wc)) { ok = false; break; }
+          const uint32_t stage = smem_addr(s.a_stages + static_cast<size_t>(st.i) * k_a_stage_bytes);
+          for (int u = half + lane; u < nops; u += 32) {
+            const int c = u / groups, r0 = 4 * (u - c * groups);
+            const int t0 = mtok[r0], t1 = mtok[r0 + 1], t2 = mtok[r0 + 2], t3 = mtok[r0 + 3];
+            tma_gather4(stage + static_cast<uint32_t>(c) * chunk_region + static_cast<uint32_t>(r0 * k_swz),
+                        &a.map_a, &s.full[st.i], (sp * k_KS + c) * elt_per_chunk, seq_row + (t0 >= 0 ? t0 : 0),
+                        seq_row + (t1 >= 0 ? t1 : 0), seq_row + (t2 >= 0 ? t2 : 0), seq_row + (t3 >= 0 ? t3 : 0));
+          }
+          st.step(S);
+        }
+        if (!ok) break;
+        ms.step(NM);
       }
     }
   } else if (warp == 1 || warp == kMmaWarp2) {
