@@ -335,6 +335,9 @@ class Step:
         self.w = [view(self.in_dev, f"w{l}") for l in range(wl.group)]
         self.out_dev = torch.full((2 * wl.group, b, T, wl.k), -1, dtype=torch.int32, device=dev)
         self.out_host = torch.empty(self.out_dev.shape, dtype=torch.int32).pin_memory()
+        # every layer's head weights are read where the step's inputs land
+        for l in range(wl.group):
+            g.w[l] = self.w[l]
         self.hs_idx = [self.out_dev[l] for l in range(wl.group)]
         self.dsa_idx = [self.out_dev[wl.group + l] for l in range(wl.group)]
         self.W_down = torch.from_numpy(Wd).to(dev, bf)
@@ -354,7 +357,6 @@ class Step:
         g.idx = self.hs_idx
         g.append(self.h_anchor, self.W_down)
         for l in range(wl.group):
-            g.w[l].copy_(self.w[l])
             li.li_absorb_query(self.ctx, self.q[l], self.W_K[l], wl.d_c, g.dtype, g.q_abs[l], g.q_abs_scale[l])
         g.hs_anchor(0)
         for l in range(1, wl.group):
@@ -641,29 +643,38 @@ def recall_leg(step, dev):
 
 
 def fused_leg(step, args, flush, stream, dist, dev, world):
-    """Scoring + selection of all G layers over the full prefix: G per-layer
-    scans of the shared latent, against one scan with the G layers' absorbed
-    queries stacked (G * H MMA columns; queries from the anchor's hidden state
-    in the training-aware instantiation).  Both from captured graphs, L2
-    flushed before each, CUDA events on the stream."""
-    g, wl = step.g, step.wl
+    """Query absorption, scoring and selection of all G layers over the full
+    prefix, for the training-aware instantiation (every layer's query from
+    the anchor's hidden state): G per-layer absorbs and scans of the shared
+    latent, against one group absorb and one scan with the G layers' queries
+    stacked (G * H MMA columns).  Both from captured graphs, L2 flushed
+    before each, CUDA events on the stream."""
+    li, g, wl = step.li, step.g, step.wl
     step.reset()
-    step.hs_path()                       # absorbed queries of every layer
     torch.cuda.synchronize()
+    # the group's queries and weights as the anchor's projection yields them:
+    # stacked [batch, G, H, .] (set up once, outside the timing)
+    q_stack = torch.stack([step.q[l][:, 0] for l in range(wl.group)], dim=1).contiguous()
+    w_stack = torch.stack([step.w[l][:, 0] for l in range(wl.group)], dim=1).contiguous()
 
     def per_layer():
         for l in range(wl.group):
+            li.li_absorb_query(step.ctx, step.q[l], step.W_K[l], wl.d_c, g.dtype, g.q_abs[l], g.q_abs_scale[l])
             g.score_topk(l)
 
-    times = graph_times([per_layer, g.fused_group_score_topk], args, flush, stream, dist, dev)
+    def fused():
+        g.set_group_queries(q_stack, step.W_K, w_stack)
+        g.fused_group_score_topk()
+
+    times = graph_times([per_layer, fused], args, flush, stream, dist, dev)
     keys = wl.group * int(sum(int(n) for n in step.inp.lengths))
     lat_bytes = int(sum(int(n) for n in step.inp.lengths)) * row_bytes(wl, wl.d_c)
     return {"per_layer_ms": times[0], "fused_ms": times[1], "fused_speedup": times[0] / times[1],
             "keys_per_step": keys, "per_layer_keys_per_s": world * keys / (times[0] / 1e3),
             "fused_keys_per_s": world * keys / (times[1] / 1e3),
             "fused_latent_gb_per_s": lat_bytes / (times[1] / 1e3) / 1e9,
-            "mode": f"{wl.group} layers x (scan + top-{wl.k}) of {wl.batch} sequences; fused: one scan, "
-                    f"{wl.group} x {wl.heads} MMA columns"}
+            "mode": f"{wl.group} layers x (absorb + scan + top-{wl.k}) of {wl.batch} sequences; fused: one group "
+                    f"absorb, one scan with {wl.group} x {wl.heads} MMA columns"}
 
 
 def max_over_ranks(x, dist, dev):

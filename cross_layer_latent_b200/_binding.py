@@ -8,7 +8,7 @@ there is no fallback path.
 import ctypes
 import os
 from dataclasses import dataclass
-from typing import Optional
+from typing import List, Optional
 
 import torch
 
@@ -75,6 +75,7 @@ _sigs = {
     "li_append_latent": (_I, [_P, ctypes.POINTER(c_li_cache), _P, _I, _I, _P, _I, _P, _SZ, _P]),
     "li_append_latent_ex": (_I, [_P, ctypes.POINTER(c_li_cache), _P, _I, _I, _P, _I,
                                  ctypes.POINTER(c_li_latent_transform), _P, _SZ, _P]),
+    "li_absorb_query_group": (_I, [_P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(_P), _I, _I, _P, _P, _P]),
     "li_absorb_query": (_I, [_P, _P, _I, _I, _I, _I, _P, _I64, _P, _I64, _I, _I, _P, _P, _P, _P]),
     "li_score_topk": (_I, [_P, ctypes.POINTER(c_li_cache), ctypes.POINTER(c_li_query), _I, _P, _P, _P, _P,
                            _SZ, _P]),
@@ -311,6 +312,16 @@ def li_hs_follower_refine(ctx: Context, cache: Cache, query: Query, cand: torch.
     ctx.check(_lib.li_hs_follower_refine(ctx.handle, ctypes.byref(cc), ctypes.byref(qq), _ptr(cand),
                                          _ptr(cand_n), int(B), int(k), _ptr(out_idx), _ptr(out_score),
                                          _ptr(scores_dump), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def li_absorb_query_group(ctx: Context, q: torch.Tensor, W_K: List[torch.Tensor], d_c: int, out_dtype: int,
+                          q_abs: torch.Tensor, q_abs_scale: Optional[torch.Tensor] = None, stream=None):
+    """q [batch, G, H, d_k] (f32 or bf16), W_K: G decoders [d_k, d_c] of q's
+    dtype -> q_abs [batch, G, H, d_c] (and q_abs_scale [batch, G, H] for e4m3)."""
+    batch, G, H, d_k = q.shape
+    ptrs = (_P * G)(*[W.data_ptr() for W in W_K])
+    ctx.check(_lib.li_absorb_query_group(ctx.handle, _ptr(q), _dtype(q), batch, G, H, d_k, ptrs, int(d_c),
+                                         int(out_dtype), _ptr(q_abs), _ptr(q_abs_scale), _stream(stream)))
 
 
 def li_topk(ctx: Context, scores: torch.Tensor, k: int, out_idx: torch.Tensor, out_score: Optional[torch.Tensor],

@@ -826,6 +826,35 @@ li_status li_append_latent_ex(li_ctx* c, const li_cache* cache, const void* h, l
   return LI_OK;
 }
 
+li_status li_absorb_query_group(li_ctx* c, const void* q, li_dtype q_dtype, int batch, int G, int H, int d_k,
+                                const void* const* W_K, int d_c, li_dtype out_dtype, void* q_abs, float* q_abs_scale,
+                                void* stream) {
+  const char* what = "li_absorb_query_group";
+  if (!c) return LI_ERR_ARG;
+  if (!q || !q_abs || !W_K) return fail(c, LI_ERR_ARG, "%s: q, q_abs and W_K must be non-NULL", what);
+  if (q_dtype != LI_F32 && q_dtype != LI_BF16) return fail(c, LI_ERR_DTYPE, "%s: q must be F32 or BF16", what);
+  if (out_dtype != LI_F32 && out_dtype != LI_BF16 && out_dtype != LI_E4M3)
+    return fail(c, LI_ERR_DTYPE, "%s: unknown out dtype", what);
+  if (out_dtype == LI_E4M3 && !q_abs_scale) return fail(c, LI_ERR_ARG, "%s: E4M3 output needs q_abs_scale", what);
+  if (G < 1 || G > kMaxAbsorbLayers) return fail(c, LI_ERR_SHAPE, "%s: G = %d must be in [1, %d]", what, G,
+                                                 kMaxAbsorbLayers);
+  if (batch < 1 || H < 1 || d_k < 1 || d_k > 256 || d_c < 2 || d_c > 256 || (d_c & 1))
+    return fail(c, LI_ERR_SHAPE, "%s: need batch, H >= 1, d_k in [1, 256] and an even d_c in [2, 256]", what);
+  if (static_cast<int64_t>(batch) * H > 2 * 65535)
+    return fail(c, LI_ERR_SHAPE, "%s: batch * H must be <= %d", what, 2 * 65535);
+  const size_t elt = q_dtype == LI_BF16 ? 2 : 4;
+  if ((static_cast<size_t>(d_k) * d_c * elt) % 16)
+    return fail(c, LI_ERR_SHAPE, "%s: d_k * d_c * element size must be a multiple of 16", what);
+  for (int l = 0; l < G; ++l)
+    if (!W_K[l] || !aligned(W_K[l], 16)) return fail(c, LI_ERR_ALIGN, "%s: W_K[%d] NULL or not 16-byte aligned", what, l);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Launch L(c, st, "absorb", 0, 256, 0);
+  const cudaError_t e = launch_absorb_group(q, q_dtype, batch, G, H, d_k, W_K, d_c, out_dtype, q_abs, q_abs_scale, st);
+  L.done();
+  if (e != cudaSuccess) return cuda_fail(c, e, "group absorb launch");
+  return LI_OK;
+}
+
 li_status li_absorb_query(li_ctx* c, const void* q, li_dtype q_dtype, int n_tok, int H, int d_k, const void* W_K,
                           int64_t W_K_head_stride, const float* b_K, int64_t b_K_head_stride, int d_c,
                           li_dtype out_dtype, void* q_abs, float* q_abs_scale, float* beta, void* stream) {

@@ -518,20 +518,35 @@ __device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
 }
 __device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
 
+// Decoders of the layers one absorb launch serves (one, or a group's layers).
+struct AbsorbLayers {
+  const void* W[kMaxAbsorbLayers];
+  int G, H;
+};
+
 // Shared decoder (one W_K for every head): rows (token, head) are taken R at a
 // time per block. The decoder is staged once in shared memory with 16-byte
 // loads, the R query rows as fp32; each thread then owns column pairs of a row
 // and accumulates j = 0..d_k-1 in order with fp32 fma (the same order as the
 // per-head kernel above, so both give identical results). A warp per row
 // finally converts the fp32 row to the output dtype.
+// With several layers (grid y = layer l, decoder L.W[l]), the rows of
+// token b and head h of layer l sit at row (b * G + l) * H + h of q and of
+// the outputs (the layers of a token stacked), and M counts the rows of one
+// layer; with one layer, row m is m.
 template <typename T>
-__global__ void __launch_bounds__(256) absorb_shared_kernel(const T* __restrict__ q, int M, int d_k,
-                                                            const T* __restrict__ W,
+__global__ void __launch_bounds__(256) absorb_shared_kernel(const T* __restrict__ q, int M, int d_k, AbsorbLayers L,
                                                             const float* __restrict__ bK, int d_c, int R,
                                                             int out_dtype, void* q_abs, float* q_abs_scale,
                                                             float* beta) {
   pdl_begin();
   pdl_release();
+  const int layer = blockIdx.y;
+  const T* __restrict__ W = static_cast<const T*>(L.W[layer]);
+  auto grow = [&](int m) -> int64_t {
+    return L.G == 1 ? static_cast<int64_t>(m)
+                    : (static_cast<int64_t>(m / L.H) * L.G + layer) * L.H + (m % L.H);
+  };
   extern __shared__ __align__(16) unsigned char absorb_smem[];
   T* Ws = reinterpret_cast<T*>(absorb_smem);                                   // [d_k][d_c]
   float* qs = reinterpret_cast<float*>(absorb_smem + (static_cast<size_t>(d_k) * d_c * sizeof(T) + 15) / 16 * 16);
@@ -547,8 +562,15 @@ __global__ void __launch_bounds__(256) absorb_shared_kernel(const T* __restrict_
     for (int x = threadIdx.x; x < n16; x += blockDim.x) cp_async_16(dst + 16u * x, src + x);
     cp_async_commit();
     const int nq = nr * d_k;
-    for (int x = threadIdx.x; x < R * d_k; x += blockDim.x)
-      qs[x] = x < nq ? to_f(q[static_cast<int64_t>(r0) * d_k + x]) : 0.f;
+    if (L.G == 1) {
+      for (int x = threadIdx.x; x < R * d_k; x += blockDim.x)
+        qs[x] = x < nq ? to_f(q[static_cast<int64_t>(r0) * d_k + x]) : 0.f;
+    } else {
+      for (int x = threadIdx.x; x < R * d_k; x += blockDim.x) {
+        const int rr = x / d_k;
+        qs[x] = x < nq ? to_f(q[grow(r0 + rr) * d_k + (x - rr * d_k)]) : 0.f;
+      }
+    }
     cp_async_wait_all();
   }
   __syncthreads();
@@ -571,7 +593,7 @@ __global__ void __launch_bounds__(256) absorb_shared_kernel(const T* __restrict_
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int rr = warp; rr < nr; rr += blockDim.x >> 5) {
-    const int64_t row = r0 + rr;
+    const int64_t row = grow(r0 + rr);
     const float* orow = os + rr * d_c;
     if (beta) {
       float bsum = 0.f;
@@ -689,6 +711,44 @@ cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t sp
                     capacity, dim, dtype, scale_split, tf, done_counter, status);
 }
 
+static cudaError_t launch_absorb_shared(const void* q, int q_dtype, int M, int d_k, const AbsorbLayers& L, int layers,
+                                 const float* b, int d_c, int R, size_t smem, int out_dtype, void* q_abs,
+                                 float* q_abs_scale, float* beta, cudaStream_t st) {
+  const dim3 grid((M + R - 1) / R, layers);
+  cudaError_t e;
+  if (q_dtype == LI_BF16) {
+    auto k = absorb_shared_kernel<__nv_bfloat16>;
+    e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k, grid, dim3(256), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(q), M, d_k, L, b, d_c,
+                      R, out_dtype, q_abs, q_abs_scale, beta);
+  }
+  auto k = absorb_shared_kernel<float>;
+  e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, grid, dim3(256), smem, st, 1, reinterpret_cast<const float*>(q), M, d_k, L, b, d_c, R,
+                    out_dtype, q_abs, q_abs_scale, beta);
+}
+
+cudaError_t launch_absorb_group(const void* q, int q_dtype, int batch, int G, int H, int d_k, const void* const* W,
+                                int d_c, int out_dtype, void* q_abs, float* q_abs_scale, cudaStream_t st) {
+  const size_t elt = q_dtype == LI_BF16 ? 2 : 4;
+  const int M = batch * H;                       // rows of one layer
+  const int R = M <= 4096 ? 2 : 32;
+  const size_t smem = absorb_shared_smem(d_k, d_c, R, elt);
+  if (G < 1 || G > kMaxAbsorbLayers || (d_c & 1) || smem > 200 * 1024 || (static_cast<size_t>(d_k) * d_c * elt) % 16)
+    return cudaErrorInvalidValue;
+  AbsorbLayers L{};
+  for (int l = 0; l < G; ++l) {
+    if (!W[l] || (reinterpret_cast<uintptr_t>(W[l]) & 15)) return cudaErrorInvalidValue;
+    L.W[l] = W[l];
+  }
+  L.G = G;
+  L.H = H;
+  return launch_absorb_shared(q, q_dtype, M, d_k, L, G, nullptr, d_c, R, smem, out_dtype, q_abs, q_abs_scale,
+                              nullptr, st);
+}
+
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
                           int out_dtype, void* q_abs, float* q_abs_scale, float* beta, cudaStream_t st) {
@@ -702,21 +762,11 @@ cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k,
   const bool aligned = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (static_cast<size_t>(d_k) * d_c * elt) % 16 == 0;
   if (W != nullptr && W_head_stride == 0 && b_head_stride == 0 && (d_c & 1) == 0 && aligned &&
       smem <= 200 * 1024) {
-    const int grid = (M + R - 1) / R;
-    cudaError_t e;
-    if (q_dtype == LI_BF16) {
-      auto k = absorb_shared_kernel<__nv_bfloat16>;
-      e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      return launch_pdl(k, dim3(grid), dim3(256), smem, st, 1, reinterpret_cast<const __nv_bfloat16*>(q), M, d_k,
-                        reinterpret_cast<const __nv_bfloat16*>(W), b, d_c, R, out_dtype, q_abs, q_abs_scale, beta);
-    } else {
-      auto k = absorb_shared_kernel<float>;
-      e = raise_smem_limit(reinterpret_cast<const void*>(k), static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      return launch_pdl(k, dim3(grid), dim3(256), smem, st, 1, reinterpret_cast<const float*>(q), M, d_k,
-                        reinterpret_cast<const float*>(W), b, d_c, R, out_dtype, q_abs, q_abs_scale, beta);
-    }
+    AbsorbLayers L{};
+    L.W[0] = W;
+    L.G = 1;
+    L.H = H;
+    return launch_absorb_shared(q, q_dtype, M, d_k, L, 1, b, d_c, R, smem, out_dtype, q_abs, q_abs_scale, beta, st);
   }
   const dim3 grid((H + kAbsorbHeads - 1) / kAbsorbHeads, n_tok);
   if (q_dtype == LI_BF16)

@@ -185,6 +185,11 @@ cudaError_t launch_append_store(const float* c, int64_t c_tok_stride, int64_t sp
                                 int batch, int T_chunk, int t0, int T_total, bool bump, void* data,
                                 float* scale, int32_t* lengths, int capacity, int dim, int dtype, int scale_split,
                                 const RowTransform& tf, unsigned int* done_counter, int* status, cudaStream_t st);
+// G layers' decoders (G <= kMaxAbsorbLayers, 16-byte aligned, shared by the
+// heads) absorbed into queries stacked [batch][G][H][.] in one launch.
+constexpr int kMaxAbsorbLayers = 8;
+cudaError_t launch_absorb_group(const void* q, int q_dtype, int batch, int G, int H, int d_k, const void* const* W,
+                                int d_c, int out_dtype, void* q_abs, float* q_abs_scale, cudaStream_t st);
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
                           int out_dtype, void* q_abs, float* q_abs_scale, float* beta,

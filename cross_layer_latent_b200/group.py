@@ -15,8 +15,8 @@ from typing import List, Optional
 import torch
 
 from ._binding import (LI_BF16, LI_E4M3, LI_F32, Cache, Context, LatentTransform, Query, li_absorb_query,
-                       li_append_latent, li_append_latent_ex, li_dsa_score_topk, li_hs_anchor_candidates, li_hs_follower_refine, li_score_topk,
-                       workspace)
+                       li_absorb_query_group, li_append_latent, li_append_latent_ex, li_dsa_score_topk,
+                       li_hs_anchor_candidates, li_hs_follower_refine, li_score_topk, workspace)
 
 TORCH_DTYPE = {LI_F32: torch.float32, LI_BF16: torch.bfloat16, LI_E4M3: torch.uint8}
 
@@ -51,8 +51,7 @@ class GroupIndexer:
         dev, tdt = self.device, TORCH_DTYPE[dtype]
         self.latent = _cache(batch, capacity, d_c, dtype, dev, scale_split)
         self.keys: List[Cache] = [_cache(batch, capacity, d_k, dtype, dev) for _ in range(G)] if dsa else []
-        # layer-major storage: layer l's queries are the contiguous slice [l],
-        # and the fused group scan restacks all layers with one copy each
+        # per-layer queries, layer-major: layer l's are the contiguous slice [l]
         e4 = dtype == LI_E4M3
         self.q_abs_all = torch.zeros(G, batch, T, H, d_c, dtype=tdt, device=dev)
         self.q_abs_scale_all = torch.ones(G, batch, T, H, device=dev) if e4 else None
@@ -149,31 +148,34 @@ class GroupIndexer:
                       self.ws, stream)
         return self.idx[layer]
 
-    def fused_group_score_topk(self, dump: Optional[torch.Tensor] = None, stream=None):
-        """Full LatentIndex for all G layers of a decode token with one pass
-        over the shared latent: the layers' absorbed queries are stacked as G
-        query rows of each sequence (training-aware instantiation, Sec. D.2:
-        every layer's query comes from the anchor's hidden state, so all exist
-        at once).  The scan takes up to 256 // H of them per MMA (G * H columns
-        at G = 4, H = 64: one read of the latent for the whole group).
-        Selections land in idx_group [batch, G, k]; dump, if given, is
-        [batch, G, capacity]."""
+    def set_group_queries(self, q: torch.Tensor, W_K: List[torch.Tensor], w: torch.Tensor, stream=None):
+        """Training-aware instantiation (Sec. D.2): every layer's query and
+        head weights come from the anchor's hidden state, so the group's
+        queries arrive together.  q [batch, G, H, d_k] (f32 or bf16) is
+        absorbed with the G decoders W_K[l] [d_k, d_c] (q's dtype) in one
+        launch, stacked as q_group [batch, G, H, d_c]; w [batch, G, H] f32 is
+        kept as the group's head weights (not copied)."""
         if self.T != 1:
             raise ValueError("the fused group scan stacks decode queries (T = 1)")
         if not hasattr(self, "q_group"):
             dev, G, b = self.device, self.G, self.batch
-            self.q_group = torch.empty_like(self.q_abs_all[:, :, 0].transpose(0, 1).contiguous())
-            self.q_group_scale = (torch.empty(b, G, self.H, device=dev)
-                                  if self.q_abs_scale_all is not None else None)
-            self.w_group = torch.empty(b, G, self.H, device=dev)
+            self.q_group = torch.empty(b, G, self.H, self.d_c, dtype=TORCH_DTYPE[self.dtype], device=dev)
+            self.q_group_scale = torch.empty(b, G, self.H, device=dev) if self.dtype == LI_E4M3 else None
             self.idx_group = torch.full((b, G, self.k), -1, dtype=torch.int32, device=dev)
             self.score_group = torch.zeros(b, G, self.k, device=dev)
             self.ws_group = workspace(self.ctx, b, G, self.capacity, self.H, self.k, 0, device=dev)
-        # layer-major [G, b, H, ...] to sequence-major [b, G, H, ...]: one copy per array
-        self.q_group.copy_(self.q_abs_all[:, :, 0].transpose(0, 1))
-        self.w_group.copy_(self.w_all[:, :, 0].transpose(0, 1))
-        if self.q_group_scale is not None:
-            self.q_group_scale.copy_(self.q_abs_scale_all[:, :, 0].transpose(0, 1))
+        li_absorb_query_group(self.ctx, q, W_K, self.d_c, self.dtype, self.q_group, self.q_group_scale, stream)
+        self.w_group = w
+
+    def fused_group_score_topk(self, dump: Optional[torch.Tensor] = None, stream=None):
+        """Full LatentIndex for all G layers of a decode token with one pass
+        over the shared latent: the queries set by set_group_queries are the
+        G query rows of each sequence, and the scan takes up to 256 // H of
+        them per MMA (G * H columns at G = 4, H = 64: one read of the latent
+        for the whole group).  Selections land in idx_group [batch, G, k];
+        dump, if given, is [batch, G, capacity]."""
+        if not hasattr(self, "w_group"):
+            raise RuntimeError("set_group_queries must come first")
         q = Query(q=self.q_group, w=self.w_group, q_scale=self.q_group_scale, beta=None, q_pos=None, dtype=self.dtype)
         li_score_topk(self.ctx, self.latent, q, self.k, self.idx_group, self.score_group, dump, self.ws_group, stream)
         return self.idx_group

@@ -242,6 +242,24 @@ LI_API li_status li_absorb_query(li_ctx* ctx, const void* q, li_dtype q_dtype, i
                           int64_t b_K_head_stride, int d_c, li_dtype out_dtype, void* q_abs,
                           float* q_abs_scale, float* beta, void* stream);
 
+/* Absorption for a whole group at once (training-aware instantiation,
+ * Sec. D.2: every layer's query comes from the anchor's hidden state, so the
+ * G layers' queries exist together).  For sequence b, layer l < G and head
+ * h: q_abs[b][l][h] = W_K[l]^T q[b][l][h], with the arithmetic and rounding
+ * of li_absorb_query with a shared decoder, written stacked so that the G
+ * layers are the T = G query rows of one li_score_topk call (one pass over
+ * the latent for the group).  One launch for all layers.
+ * q       [batch][G][H][d_k] of q_dtype (F32 or BF16).
+ * W_K     host array of G device pointers, each a decoder [d_k][d_c] of
+ *         q_dtype, 16-byte aligned (d_k * d_c * element size a multiple of
+ *         16); shared by the heads of its layer; no decoder bias.
+ * q_abs   [batch][G][H][d_c] of out_dtype; q_abs_scale [batch][G][H] fp32
+ *         for E4M3 output (as li_absorb_query).
+ * Needs 1 <= G <= 8, d_c even, batch * H <= 65535 * 2.                      */
+LI_API li_status li_absorb_query_group(li_ctx* ctx, const void* q, li_dtype q_dtype, int batch, int G, int H,
+                                int d_k, const void* const* W_K, int d_c, li_dtype out_dtype,
+                                void* q_abs, float* q_abs_scale, void* stream);
+
 /* ------------------------------------------------ a3 + a4: scan and select */
 
 /* Full-prefix LatentIndex scoring and per-layer selection (Sec. 3.1): scores

@@ -47,8 +47,18 @@ def test_fused_group_scan_equals_per_layer_scans(ctx, name):
         g.score_topk(l, dump=dump)
         torch.cuda.synchronize()
         per_layer.append((dump.cpu().numpy()[:, 0], g.idx[l].cpu().numpy()[:, 0]))
+    # the group's queries stacked [batch, G, H, d_k], absorbed in one launch
+    q_stack = torch.from_numpy(np.ascontiguousarray(np.stack([inp.q[l][:, 0] for l in range(wl.group)], axis=1)))
+    w_stack = torch.from_numpy(np.ascontiguousarray(np.stack([inp.w[l][:, 0] for l in range(wl.group)], axis=1)))
+    W_K = [torch.from_numpy(inp.W_K[l]).to(DEV).contiguous() for l in range(wl.group)]
+    g.set_group_queries(q_stack.to(DEV), W_K, w_stack.to(DEV))
     gdump = torch.full((wl.batch, wl.group, wl.capacity), float("nan"), device=DEV)
     g.fused_group_score_topk(dump=gdump)
+    # the group absorb writes the per-layer absorb's values, stacked
+    for l in range(wl.group):
+        assert torch.equal(g.q_group[:, l], g.q_abs[l][:, 0]), f"{name} layer {l}: absorbed queries differ"
+        if g.q_group_scale is not None:
+            assert torch.equal(g.q_group_scale[:, l], g.q_abs_scale[l][:, 0])
     torch.cuda.synchronize()
     assert li.li_device_status(ctx, g.ws_group) == "LI_OK"
     gd, gidx = gdump.cpu().numpy(), g.idx_group.cpu().numpy()
