@@ -785,7 +785,8 @@ li_status li_append_latent_ex(li_ctx* c, const li_cache* cache, const void* h, l
   {
     const int n_tok = cache->batch * T;
     const int splits = append_fused_splits(d_model, dim);
-    if (append_fusable(n_tok, dim, splits)) {
+    if (append_fusable(n_tok, dim, splits) &&
+        append_fused_smem(n_tok, dim, splits, d_model, static_cast<size_t>(eb)) <= 96 * 1024) {
       Launch Lg(c, st, "append", 0, 256, 0);
       const cudaError_t e = launch_append_fused(h, h_dtype, W_down, d_model, dim, cache->batch, T, splits, tmp,
                                                 cache->data, cache->scale, cache->lengths, cache->capacity,

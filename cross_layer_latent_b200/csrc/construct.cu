@@ -260,27 +260,58 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
   // its warps share one slice of the hidden states (read once, then from L1)
   const int sp = static_cast<int>(blockIdx.x) % splits;
   const int j = (static_cast<int>(blockIdx.x) / splits) * kAppendWarps + warp;
-  if (j < dim) {
-    const int len = d_model / splits;
-    const int i0 = sp * len, i1 = i0 + len;
-    float acc[kGemvTok];
+  const int len = d_model / splits;   // a multiple of 256 (append_fused_splits)
+  const int i0 = sp * len;
+  // The block's slice of every token's hidden state goes to shared memory
+  // once (all 16-byte pieces in flight), while each warp requests all of its
+  // decoder row slice at once: the GEMV waits one memory round trip, not one
+  // per 256-element step.  (The last block reuses this memory for the
+  // partial sums afterwards.)
+  T* hs = reinterpret_cast<T*>(ps);   // [n_tok][len]
+  {
+    const int per_tok = len * static_cast<int>(sizeof(T)) / 16;
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(hs));
+    for (int x = threadIdx.x; x < n_tok * per_tok; x += blockDim.x) {
+      const int t = x / per_tok, c = x - t * per_tok;
+      cp_async_16(dst + 16u * x, h + static_cast<int64_t>(t) * d_model + i0 + c * (16 / static_cast<int>(sizeof(T))));
+    }
+    cp_async_commit();
+  }
+  float acc[kGemvTok];
 #pragma unroll
-    for (int t = 0; t < kGemvTok; ++t) acc[t] = 0.f;
-    const T* wrow = W + static_cast<int64_t>(j) * d_model;
-#pragma unroll 4
-    for (int i = i0 + lane * 8; i < i1; i += 256) {
-      float wv[8];
-      load8<T>(wrow + i, wv);
+  for (int t = 0; t < kGemvTok; ++t) acc[t] = 0.f;
+  constexpr int kSteps = 4;           // 256-element steps held in registers at once
+  for (int ib = 0; ib < len; ib += kSteps * 256) {
+    float wv[kSteps][8];
+    if (j < dim) {
+      const T* wrow = W + static_cast<int64_t>(j) * d_model + i0;
 #pragma unroll
-      for (int t = 0; t < kGemvTok; ++t) {
-        if (t < n_tok) {
-          float hv[8];
-          load8<T>(h + static_cast<int64_t>(t) * d_model + i, hv);
+      for (int u = 0; u < kSteps; ++u)
+        if (ib + u * 256 < len) load8<T>(wrow + ib + u * 256 + lane * 8, wv[u]);
+    }
+    if (ib == 0) {
+      cp_async_wait_all();
+      __syncthreads();
+    }
+    if (j < dim) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[t] = fmaf(wv[e], hv[e], acc[t]);
+      for (int u = 0; u < kSteps; ++u) {
+        const int i = ib + u * 256 + lane * 8;
+        if (ib + u * 256 < len) {
+#pragma unroll
+          for (int t = 0; t < kGemvTok; ++t) {
+            if (t < n_tok) {
+              float hv[8];
+              load8<T>(hs + t * len + i, hv);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[t] = fmaf(wv[u][e], hv[e], acc[t]);
+            }
+          }
         }
       }
     }
+  }
+  if (j < dim) {
 #pragma unroll
     for (int t = 0; t < kGemvTok; ++t) {
 #pragma unroll
@@ -659,6 +690,14 @@ int append_fused_splits(int d_model, int dim) {
   return 1;
 }
 
+// Shared memory of the one-launch append: the hidden-state slices during the
+// GEMV, then (last block) the partial sums.
+size_t append_fused_smem(int n_tok, int dim, int splits, int d_model, size_t h_elt) {
+  const size_t partials = static_cast<size_t>(splits + 1) * n_tok * dim * sizeof(float);
+  const size_t slices = static_cast<size_t>(n_tok) * (d_model / splits) * h_elt;
+  return partials > slices ? partials : slices;
+}
+
 bool append_fusable(int n_tok, int dim, int splits) {
   return splits >= 1 && n_tok <= kGemvTok && dim <= 256 && (splits + 1) * n_tok * dim <= kFuseMaxPartials;
 }
@@ -670,7 +709,7 @@ cudaError_t launch_append_fused_tf(const void* h, int h_dtype, const void* W, in
                                    int* status, cudaStream_t st) {
   const int n_tok = batch * T;
   const int grid = splits * ((dim + kAppendWarps - 1) / kAppendWarps);
-  const size_t smem = static_cast<size_t>(splits + 1) * n_tok * dim * sizeof(float);
+  const size_t smem = append_fused_smem(n_tok, dim, splits, d_model, h_dtype == LI_BF16 ? 2 : 4);
   cudaError_t e;
   if (h_dtype == LI_BF16) {
     auto k = gemv_append_kernel<__nv_bfloat16, TF>;

@@ -177,6 +177,7 @@ cudaError_t launch_append_gemv(const void* h, int h_dtype, const void* W, int d_
 // reduces the splits in order and stores the rows.
 int append_fused_splits(int d_model, int dim);
 bool append_fusable(int n_tok, int dim, int splits);
+size_t append_fused_smem(int n_tok, int dim, int splits, int d_model, size_t h_elt);
 cudaError_t launch_append_fused(const void* h, int h_dtype, const void* W, int d_model, int dim, int batch, int T,
                                 int splits, float* part, void* data, float* scale, int32_t* lengths, int capacity,
                                 int dtype, int scale_split, const RowTransform& tf, unsigned int* done, int* status,
