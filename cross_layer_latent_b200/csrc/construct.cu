@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
   float acc[kGemvTok];
 #pragma unroll
   for (int t = 0; t < kGemvTok; ++t) acc[t] = 0.f;
-  constexpr int kSteps = 4;           // 256-element steps held in registers at once
+  constexpr int kSteps = 8;           // 256-element steps held in registers at once
   for (int ib = 0; ib < len; ib += kSteps * 256) {
     float wv[kSteps][8];
     if (j < dim) {
