@@ -415,7 +415,7 @@ __device__ __forceinline__ void push_group_counts(cg::cluster_group& cluster, in
 // bins: res[i] = {bin, above}.  The boundary group comes from the gathered
 // group counts ga[CS][NG] (local), its 32 bins from every CTA's histogram
 // (distributed shared memory).  The block synchronises afterwards.
-template <int NG, bool CL>
+template <int NG, bool CL, int CMAX>
 __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, unsigned* hist, const unsigned* ga,
                                           int nn, const int* need, int (*res)[2]) {
   if (threadIdx.x >= 32) return;
@@ -427,9 +427,9 @@ __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, un
   for (int e = 0; e < GPL; ++e) gc[e] = 0;
   {
     const int g_lo = NG - GPL * (lane + 1);          // lowest group of this lane
-    unsigned v[kClusterMaxSize][GPL];
+    unsigned v[CMAX][GPL];
 #pragma unroll
-    for (int rk = 0; rk < kClusterMaxSize; ++rk) {
+    for (int rk = 0; rk < CMAX; ++rk) {
       if (rk < CS) {
         const unsigned* src = ga + rk * NG + g_lo;
         if (GPL == 2) {
@@ -442,7 +442,7 @@ __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, un
       }
     }
 #pragma unroll
-    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+    for (int rk = 0; rk < CMAX; ++rk)
       if (rk < CS) {
 #pragma unroll
         for (int e = 0; e < GPL; ++e) gc[e] += v[rk][e];
@@ -479,13 +479,13 @@ __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, un
     above = __shfl_sync(0xffffffffu, above, src_lane);
     // the group's 32 bins, descending: lane l takes bin 32 g + 31 - l
     const int bin = grp_sel * 32 + 31 - lane;
-    unsigned bv[kClusterMaxSize];
+    unsigned bv[CMAX];
 #pragma unroll
-    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+    for (int rk = 0; rk < CMAX; ++rk)
       if (rk < CS) bv[rk] = rank_ptr<CL>(cluster, hist, rk)[bin];
     unsigned bc = 0;
 #pragma unroll
-    for (int rk = 0; rk < kClusterMaxSize; ++rk)
+    for (int rk = 0; rk < CMAX; ++rk)
       if (rk < CS) bc += bv[rk];
     unsigned bincl = bc;
 #pragma unroll
@@ -502,7 +502,9 @@ __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, un
   }
 }
 
-template <int PT, bool CL>
+// CMAX: the largest cluster this instantiation serves (8, portable; 16 for
+// the longest decode rows, non-portable).
+template <int PT, bool CL, int CMAX = 8>
 __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const TopkArgs a) {
   pdl_begin();
   constexpr int NW = kClusterThreads / 32;
@@ -510,12 +512,12 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   __shared__ __align__(16) unsigned H1[2048];                       // top 11 bits
   __shared__ __align__(16) unsigned H2[2048];                       // next 11 bits (boundary bin)
   __shared__ __align__(16) unsigned H3[1024];                       // last 10 bits (boundary prefix)
-  __shared__ __align__(16) unsigned G1[kClusterMaxSize * 64];       // group counts of every CTA
-  __shared__ __align__(16) unsigned G2[kClusterMaxSize * 64];
-  __shared__ __align__(16) unsigned G3[kClusterMaxSize * 32];
+  __shared__ __align__(16) unsigned G1[CMAX * 64];                  // group counts of every CTA
+  __shared__ __align__(16) unsigned G2[CMAX * 64];
+  __shared__ __align__(16) unsigned G3[CMAX * 32];
   __shared__ int res[1][2];
   __shared__ int wtot[NW];                                          // packed (gt, eq) per warp
-  __shared__ int cin[kClusterMaxSize][2];                           // (gt, eq) totals of earlier CTAs
+  __shared__ int cin[CMAX][2];                                      // (gt, eq) totals of earlier CTAs
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = CL ? static_cast<int>(cluster.num_blocks()) : 1;
   const int c = CL ? static_cast<int>(cluster.block_rank()) : 0;
@@ -580,7 +582,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   __syncthreads();
   push_group_counts<64, CL>(cluster, CS, c, H1, G1);
   sync_row<CL>(cluster);
-  find_bins<64, CL>(cluster, CS, H1, G1, 1, &keff, res);
+  find_bins<64, CL, CMAX>(cluster, CS, H1, G1, 1, &keff, res);
   __syncthreads();
   unsigned pre = static_cast<unsigned>(res[0][0]);
   int above = res[0][1];
@@ -593,7 +595,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   __syncthreads();
   push_group_counts<64, CL>(cluster, CS, c, H2, G2);
   sync_row<CL>(cluster);
-  find_bins<64, CL>(cluster, CS, H2, G2, 1, &need, res);
+  find_bins<64, CL, CMAX>(cluster, CS, H2, G2, 1, &need, res);
   __syncthreads();
   pre = (pre << 11) | static_cast<unsigned>(res[0][0]);
   above += res[0][1];
@@ -606,7 +608,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   __syncthreads();
   push_group_counts<32, CL>(cluster, CS, c, H3, G3);
   sync_row<CL>(cluster);
-  find_bins<32, CL>(cluster, CS, H3, G3, 1, &need, res);
+  find_bins<32, CL, CMAX>(cluster, CS, H3, G3, 1, &need, res);
   __syncthreads();
   const unsigned T = (pre << 10) | static_cast<unsigned>(res[0][0]);
   above += res[0][1];
@@ -693,12 +695,30 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
 template <int PT>
 cudaError_t launch_radix_pt(const TopkArgs& a, int cs, cudaStream_t st) {
   if (cs == 1) return launch_pdl(topk_radix_kernel<PT, false>, dim3(1, a.rows, 1), dim3(kClusterThreads), 0, st, 1, a);
+  if constexpr (PT == 16) {
+    if (cs > 8) {
+      // a 16-CTA cluster is non-portable: allowed once per process
+      static cudaError_t allowed = cudaFuncSetAttribute(topk_radix_kernel<16, true, 16>,
+                                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (allowed != cudaSuccess) return allowed;
+      return launch_pdl(topk_radix_kernel<16, true, 16>, dim3(cs, a.rows, 1), dim3(kClusterThreads), 0, st, cs, a);
+    }
+  }
+  if (cs > kClusterMaxSize) return cudaErrorInvalidValue;   // only 16 keys a thread comes in clusters past 8
   return launch_pdl(topk_radix_kernel<PT, true>, dim3(cs, a.rows, 1), dim3(kClusterThreads), 0, st, cs, a);
 }
 
 }  // namespace
 
 int topk_cluster_size(int64_t n, int keys_per_thread) {
+  // Rows past 65536 positions at the latency target (decode's full-prefix
+  // selections) take clusters of up to 16 CTAs (16 keys a thread at
+  // 131072), measured faster than 8 CTAs at 32 keys a thread; everything
+  // else stays within portable clusters of 8.
+  if (keys_per_thread == kTopkKeysLatency && n > 65536) {
+    const int64_t cs16 = (n + static_cast<int64_t>(kClusterThreads) * 16 - 1) / (static_cast<int64_t>(kClusterThreads) * 16);
+    return static_cast<int>(cs16 > 16 ? 16 : cs16);
+  }
   // As many CTAs as keep `keys_per_thread` keys a thread, up to a cluster of
   // 8.  A few rows (decode) are latency-bound: 4 keys a thread spreads them
   // over more CTAs and shortens every pass.  Many rows (a prefill chunk)
