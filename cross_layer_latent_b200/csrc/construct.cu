@@ -322,14 +322,17 @@ __global__ void __launch_bounds__(kAppendWarps * 32) gemv_append_kernel(const T*
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    last = atomicAdd(done, 1u) == gridDim.x - 1 ? 1u : 0u;
+    // acquire-release at GPU scope: publishes this block's partial sums
+    // (ordered before it by the barrier) and, in the last block, makes
+    // every other block's visible to the reads below
+    unsigned prev;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(done) : "memory");
+    last = prev == gridDim.x - 1 ? 1u : 0u;
   }
   __syncthreads();
   if (!last) return;
   TfLane tc;
   if constexpr (TF) tc = load_tf_lane(tf, threadIdx.x & 31);
-  __threadfence();
   const int nx = n_tok * dim, np = splits * nx;   // np <= kStagePer * blockDim.x
   {
     // every partial sum in flight at once
