@@ -552,7 +552,7 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   // 467 us, against 566 us for the chunked multi-kernel path).
   if (t.rows > 65535) return fail(ctx, LI_ERR_UNSUPPORTED, "more than 65535 selection rows");
   if (t.n <= kClusterMaxN) {
-    const int64_t cs_lat = topk_cluster_size(t.n, kTopkKeysLatency);
+    const int64_t cs_lat = topk_cluster_size(t.n, kTopkKeysLatency, t.rows);
     const int kpt = static_cast<int64_t>(t.rows) * cs_lat <= 2 * static_cast<int64_t>(ctx->num_sms)
                         ? kTopkKeysLatency : kTopkKeysThroughput;
     int cs = 0;

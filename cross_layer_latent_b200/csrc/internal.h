@@ -141,7 +141,7 @@ constexpr int kClusterMaxN = kClusterThreads * 32 * kClusterMaxSize;   // 131072
 // CTAs per row of the single-launch selection at a target of keys per thread
 // (kTopkKeysLatency for a few rows, kTopkKeysThroughput for many).
 constexpr int kTopkKeysLatency = 4, kTopkKeysThroughput = 32;
-int topk_cluster_size(int64_t n, int keys_per_thread);
+int topk_cluster_size(int64_t n, int keys_per_thread, int rows);
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size,
                                 int keys_per_thread = kTopkKeysLatency);
 

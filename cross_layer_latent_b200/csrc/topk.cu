@@ -710,12 +710,13 @@ cudaError_t launch_radix_pt(const TopkArgs& a, int cs, cudaStream_t st) {
 
 }  // namespace
 
-int topk_cluster_size(int64_t n, int keys_per_thread) {
-  // Rows past 65536 positions at the latency target (decode's full-prefix
-  // selections) take clusters of up to 16 CTAs (16 keys a thread at
-  // 131072), measured faster than 8 CTAs at 32 keys a thread; everything
-  // else stays within portable clusters of 8.
-  if (keys_per_thread == kTopkKeysLatency && n > 65536) {
+int topk_cluster_size(int64_t n, int keys_per_thread, int rows) {
+  // A few rows (at most 4) past 65536 positions at the latency target
+  // (decode's full-prefix selections) take clusters of up to 16 CTAs (16
+  // keys a thread at 131072), measured faster than 8 CTAs at 32 keys a
+  // thread.  A 16-CTA cluster needs most of a GPC, so more rows would not
+  // run in one wave; everything else stays within portable clusters of 8.
+  if (keys_per_thread == kTopkKeysLatency && n > 65536 && rows <= 4) {
     const int64_t cs16 = (n + static_cast<int64_t>(kClusterThreads) * 16 - 1) / (static_cast<int64_t>(kClusterThreads) * 16);
     return static_cast<int>(cs16 > 16 ? 16 : cs16);
   }
@@ -731,7 +732,7 @@ int topk_cluster_size(int64_t n, int keys_per_thread) {
 
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size, int keys_per_thread) {
   const int64_t n = a.n;
-  const int cs = topk_cluster_size(n, keys_per_thread);
+  const int cs = topk_cluster_size(n, keys_per_thread, a.rows);
   const int64_t per_thread = (n + static_cast<int64_t>(cs) * kClusterThreads - 1) / (static_cast<int64_t>(cs) * kClusterThreads);
   if (cluster_size) *cluster_size = cs;
   if (per_thread <= 4) return launch_radix_pt<4>(a, cs, st);
