@@ -72,3 +72,20 @@ def test_fused_group_scan_equals_per_layer_scans(ctx, name):
             assert np.array_equal(gidx[b, l], e)
             ref = Reference(inp, c64, l, b)
             assert_scores_close(gd[b, l, :n], ref.scores, ref.M, RTOL[wl.cache_dtype], f"{name} fused layer {l}")
+
+
+def test_group_absorb_rejects_bad_arguments(ctx):
+    q = torch.zeros(2, 9, 16, 32, device=DEV)
+    W = [torch.zeros(32, 64, device=DEV) for _ in range(9)]
+    out = torch.zeros(2, 9, 16, 64, device=DEV)
+    with pytest.raises(li.LiError):                      # more than 8 layers
+        li.li_absorb_query_group(ctx, q, W, 64, li.LI_F32, out)
+    q4 = q[:, :4].contiguous()
+    out4 = out[:, :4].contiguous()
+    with pytest.raises(li.LiError):                      # a decoder off 16-byte alignment
+        li.li_absorb_query_group(ctx, q4, [W[0], W[1], W[2], W[3].view(-1)[1:].view(-1)[:32 * 64 - 1]], 64,
+                                 li.LI_F32, out4)
+    with pytest.raises(li.LiError):                      # e4m3 output without scales
+        li.li_absorb_query_group(ctx, q4, W[:4], 64, li.LI_E4M3, out4.to(torch.uint8))
+    torch.cuda.synchronize()
+    assert not out4.any()

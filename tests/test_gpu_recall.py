@@ -103,3 +103,16 @@ def test_recall_of_the_library_selections(ctx):
                 assert np.all((rec[b] >= 0) & (rec[b] <= 1 + 1e-5))
             means[m].append(float(rec.mean()))
     np.testing.assert_allclose(means["full"], means["dsa"], rtol=2e-3)
+
+
+def test_recall_rejects_bad_arguments(ctx):
+    p = torch.zeros(2, 4, 100, device=DEV)
+    sel = torch.zeros(2, 8, dtype=torch.int32, device=DEV)
+    with pytest.raises(li.LiError):                      # K below 1
+        li.li_attention_recall(ctx, p, sel, 0)
+    small = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(li.LiError):                      # workspace too small
+        rec = torch.empty(2, 4, device=DEV)
+        ctx.check(li._binding._lib.li_attention_recall(ctx.handle, li._binding._ptr(p), 2, 4, 100, None,
+                                                       li._binding._ptr(sel), 8, 8, li._binding._ptr(rec), None,
+                                                       li._binding._ptr(small), small.numel(), None))
