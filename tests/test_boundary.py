@@ -25,10 +25,11 @@ def lib():
     return ctypes.CDLL(LIB)
 
 
-def test_header_declares_the_north_star_entry_points():
+def test_header_declares_the_decode_path_entry_points():
     syms = declared_symbols()
-    for name in ("li_append_latent", "li_absorb_query", "li_score_topk", "li_hs_anchor_candidates",
-                 "li_hs_follower_refine", "li_dsa_score_topk", "li_topk", "li_device_status"):
+    for name in ("li_append_latent", "li_append_latent_ex", "li_absorb_query", "li_absorb_query_group",
+                 "li_score_topk", "li_hs_anchor_candidates", "li_hs_follower_refine", "li_dsa_score_topk", "li_topk",
+                 "li_device_status", "li_attention_recall"):
         assert name in syms
 
 
