@@ -544,6 +544,8 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   t.chunk_gt = at<int>(ws, L.chunk_gt);
   t.chunk_off = at<int>(ws, L.chunk_off);
   t.cand = at<uint2>(ws, L.cand);
+  t.status = at<int>(ws, L.status);
+  t.wait_ns = ctx->wait_ns;
   if (static_cast<int64_t>(t.rows) * t.n > static_cast<int64_t>((L.scores - L.cand) / 8))
     return fail(ctx, LI_ERR_WORKSPACE, "selection of %d x %d exceeds the workspace candidate buffer", t.rows, t.n);
   // Rows of up to kClusterMaxN positions take the single-launch cluster
@@ -578,6 +580,7 @@ TopkArgs topk_args(const float* scores, int64_t stride, int rows, int n, int k) 
   t.n = n;
   t.k = k;
   t.len_div = 1;
+  t.wait_ns = 2000000000ull;
   return t;
 }
 
@@ -1192,6 +1195,8 @@ extern "C" li_status li_score_topk_static(li_ctx* c, const li_cache* cache, cons
   t.q_pos = q->q_pos;
   t.out_idx = out_idx;
   t.out_score = out_score;
+  t.status = status;
+  t.wait_ns = c->wait_ns;
   {
     int cs = 0;
     Launch Lc(c, st, "topk_cluster", 0, kClusterThreads, 0);

@@ -130,6 +130,10 @@ struct TopkArgs {
   uint2* cand;                // [rows][n]
   int n_chunks;
   bool hist_ready;            // first-digit histogram already accumulated (fused)
+  // bounded waits of the cluster kernel's exchanges: a wait that runs out
+  // records LI_ERR_DEVICE_TIMEOUT in *status (may be null)
+  int* status;
+  uint64_t wait_ns;
 };
 
 // Single-launch selection for rows of up to kClusterMaxN positions: one

@@ -152,6 +152,38 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
+// ------------------------------------------------------------------ cluster exchange
+
+// The shared::cluster address of the object at shared address `p` in the
+// cluster's CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+
+// One-way stores into a CTA's shared memory (shared::cluster addresses).  The
+// bytes count against the transaction count of that CTA's mbarrier `bar`,
+// whose phase completes once every expected byte has landed; the sender
+// does not wait.
+__device__ __forceinline__ void st_async_v2(uint32_t addr, uint32_t x, uint32_t y, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.u32 [%0], {%1, %2}, [%3];"
+               ::"r"(addr), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.u32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar) : "memory");
+}
+
+// Split cluster barrier: every thread of every CTA of the cluster arrives,
+// then waits.  The relaxed arrive orders nothing by itself (a preceding
+// fence_barrier_init publishes mbarrier initialisation).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 // ------------------------------------------------------------------ dependent launch
 
 // Every kernel of the library is launched with programmatic stream

@@ -358,24 +358,29 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
 // ============================================================================
 // Single-launch selection for rows of up to 131072 positions.
 //
-// A row is taken by CS <= 8 CTAs of 512 threads (a thread-block cluster when
+// A row is taken by CS <= 16 CTAs of 512 threads (a thread-block cluster when
 // CS > 1).  Warp w of CTA c owns the contiguous run of 32 * PT positions
 // starting at (c * 16 + w) * 32 * PT; in slab j of the run, lane l holds the
 // four positions j * 128 + 4 l + {0..3} (one coalesced 16-byte load per lane
 // and slab) as order-preserving uint32 keys in registers for the whole
 // kernel.  The exact k-th key T is found digit by digit (11 + 11 + 10 bits):
 // each pass histograms, in its own shared-memory array, the keys matching the
-// digits found so far, and reduces it to group counts (32 bins a group); the
-// CTAs meet at one barrier; then one warp per CTA sums the group counts of
-// every CTA through distributed shared memory, finds the boundary group, sums
-// that group's 32 bins the same way and finds the boundary bin.  Arrays are
-// never reused, so a pass needs one barrier, and only ~100 counters per CTA
-// cross the cluster per pass.  The output rank of a selected element is
-// #greater before it +
-// min(#equal before it, #equal taken), from warp scans within slabs, warp
-// totals within the CTA and per-CTA totals pushed into the shared memory of
-// the later CTAs before a last barrier; after it no CTA touches another's
-// shared memory, so none has to wait for the others to exit.
+// digits found so far.  The CTAs then exchange counts by one-way pushes: each
+// sends its group counts (32 bins a group) into a slot of every other CTA's
+// shared memory; every CTA sums the same slots, so all find the same
+// boundary group, and each then sends that group's 32 bins the same way and
+// finds the boundary bin.  A push lands against an mbarrier of the receiving
+// CTA that expects exactly the bytes its peers send (one mbarrier per
+// exchange, each completed once), so a CTA waits only for its own data: there
+// is no cluster-wide barrier or remote read on the way to T.  The output rank
+// of a selected element is #greater before it + min(#equal before it, #equal
+// taken), from warp scans within slabs, warp totals within the CTA and
+// per-CTA totals pushed to the later CTAs.  One relaxed cluster barrier opens
+// the exchanges (every CTA's mbarriers are initialised) and one closes the
+// kernel (no CTA exits while a peer may still push to it).  Every wait is
+// bounded; a CTA whose wait ran out records the timeout, keeps sending what
+// its peers expect, writes no output, and waits for what is still in flight
+// to it before exiting.
 // ============================================================================
 #include <cooperative_groups.h>
 
@@ -384,69 +389,60 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-template <bool CL>
-__device__ __forceinline__ void sync_row(cg::cluster_group& cluster) {
-  if (CL) cluster.sync();
-  else __syncthreads();
-}
+// Exchanges of one selection, each an mbarrier completed once (parity 0).
+enum { kXGroups1 = 0, kXBins1, kXGroups2, kXBins2, kXGroups3, kXBins3, kXTotals, kNumExchanges };
 
-template <bool CL, typename T>
-__device__ __forceinline__ T* rank_ptr(cg::cluster_group& cluster, T* p, int rk) {
-  if (CL) return cluster.map_shared_rank(p, rk);
-  return p;
-}
-
-// After this CTA's histogram hist[NG * 32] is complete (and the block has
-// synchronised): the group counts (sum of bins [32 g, 32 g + 32)) are written
-// into slot c of ga[CS][NG] in the shared memory of every CTA of the row.
-template <int NG, bool CL>
-__device__ __forceinline__ void push_group_counts(cg::cluster_group& cluster, int CS, int c, const unsigned* hist,
-                                                  unsigned* ga) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int g = warp; g < NG; g += kClusterThreads / 32) {
-    const unsigned v = __reduce_add_sync(0xffffffffu, hist[g * 32 + lane]);
-    if (lane < CS) rank_ptr<CL>(cluster, ga, lane)[c * NG + g] = v;
-  }
-}
-
-// Warp 0: find, for each of nn counts need[i] (1 <= need[i] <= total), the bin
-// (counting from the top) that holds the need[i]-th element of the row's
-// histogram summed over the CS CTAs, and how many elements lie in higher
-// bins: res[i] = {bin, above}.  The boundary group comes from the gathered
-// group counts ga[CS][NG] (local), its 32 bins from every CTA's histogram
-// (distributed shared memory).  The block synchronises afterwards.
+// One radix digit.  hist[NG * 32] is this CTA's complete histogram (the block
+// has synchronised).  Group counts go into slot c of gcnt[CS][NG] of every CTA
+// (bars[0] of the receiver), the boundary group's bins into slot c of
+// gbins[CS][32] (bars[1]).  Warp 0 finds the bin holding the need-th element
+// counted from the top (1 <= need <= the row's total) and the elements in
+// higher bins: res = {bin, above}.  The caller synchronises the block
+// afterwards.
 template <int NG, bool CL, int CMAX>
-__device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, unsigned* hist, const unsigned* ga,
-                                          int nn, const int* need, int (*res)[2]) {
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
-  // lane l owns groups (descending) NG-1-(NG/32)l ... : 2 groups when NG = 64, 1 when 32
+__device__ __forceinline__ void select_digit(int CS, int c, const unsigned* hist, unsigned* gcnt, unsigned* gbins,
+                                             uint64_t* bars, int need, int (*res)[2], const WaitCtl& w) {
+  constexpr int GPW = NG / (kClusterThreads / 32);    // groups per warp: 4 (NG 64) or 2 (NG 32)
+  static_assert(GPW == 2 || GPW == 4, "one 8- or 16-byte push per warp and receiver");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  {
+    unsigned v[GPW];
+#pragma unroll
+    for (int e = 0; e < GPW; ++e) v[e] = __reduce_add_sync(0xffffffffu, hist[(warp * GPW + e) * 32 + lane]);
+    unsigned* mine = gcnt + c * NG + warp * GPW;
+    if (lane == c) {
+#pragma unroll
+      for (int e = 0; e < GPW; ++e) mine[e] = v[e];
+    } else if (CL && lane < CS) {
+      const uint32_t dst = cluster_addr(mine, lane), bar = cluster_addr(&bars[0], lane);
+      if constexpr (GPW == 4) st_async_v4(dst, make_uint4(v[0], v[1], v[2], v[3]), bar);
+      else st_async_v2(dst, v[0], v[1], bar);
+    }
+  }
+  __syncthreads();                                     // own slot visible to warp 0
+  if (warp != 0) return;
+  if (CL) bounded_wait(&bars[0], 0, w);
+
+  // boundary group: lane l owns groups (descending) NG-1-GPL*l ...
   constexpr int GPL = NG / 32;
   unsigned gc[GPL];
 #pragma unroll
   for (int e = 0; e < GPL; ++e) gc[e] = 0;
   {
-    const int g_lo = NG - GPL * (lane + 1);          // lowest group of this lane
-    unsigned v[CMAX][GPL];
+    const int g_lo = NG - GPL * (lane + 1);            // lowest group of this lane
 #pragma unroll
     for (int rk = 0; rk < CMAX; ++rk) {
       if (rk < CS) {
-        const unsigned* src = ga + rk * NG + g_lo;
-        if (GPL == 2) {
+        const unsigned* src = gcnt + rk * NG + g_lo;
+        if constexpr (GPL == 2) {
           const uint2 u = *reinterpret_cast<const uint2*>(src);
-          v[rk][0] = u.y;                              // higher group first
-          v[rk][GPL - 1] = u.x;
+          gc[0] += u.y;                                // higher group first
+          gc[1] += u.x;
         } else {
-          v[rk][0] = src[0];
+          gc[0] += src[0];
         }
       }
     }
-#pragma unroll
-    for (int rk = 0; rk < CMAX; ++rk)
-      if (rk < CS) {
-#pragma unroll
-        for (int e = 0; e < GPL; ++e) gc[e] += v[rk][e];
-      }
   }
   unsigned tot = 0;
 #pragma unroll
@@ -457,48 +453,52 @@ __device__ __forceinline__ void find_bins(cg::cluster_group& cluster, int CS, un
     const unsigned u = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += u;
   }
-  const unsigned excl = incl - tot;
-  for (int i = 0; i < nn; ++i) {
-    const unsigned nd = static_cast<unsigned>(need[i]);
-    // boundary group and elements above it
-    const unsigned hit = __ballot_sync(0xffffffffu, excl < nd && nd <= incl);
-    const int src_lane = __ffs(hit) - 1;
-    int grp_sel = 0;
-    unsigned above = 0;
-    if (lane == src_lane) {
-      unsigned cum = excl;
-      grp_sel = NG - 1 - GPL * lane;
+  const unsigned nd = static_cast<unsigned>(need);
+  const unsigned hit = __ballot_sync(0xffffffffu, incl - tot < nd && nd <= incl);
+  const int src_lane = hit ? __ffs(hit) - 1 : 0;
+  int grp_sel = 0;
+  unsigned above = 0;
+  if (lane == src_lane) {
+    unsigned cum = incl - tot;
+    grp_sel = NG - 1 - GPL * lane;
 #pragma unroll
-      for (int e = 0; e < GPL; ++e) {
-        if (cum + gc[e] >= nd) { grp_sel = NG - 1 - GPL * lane - e; break; }
-        cum += gc[e];
-      }
-      above = cum;
+    for (int e = 0; e < GPL; ++e) {
+      if (cum + gc[e] >= nd) { grp_sel = NG - 1 - GPL * lane - e; break; }
+      cum += gc[e];
     }
-    grp_sel = __shfl_sync(0xffffffffu, grp_sel, src_lane);
-    above = __shfl_sync(0xffffffffu, above, src_lane);
-    // the group's 32 bins, descending: lane l takes bin 32 g + 31 - l
-    const int bin = grp_sel * 32 + 31 - lane;
-    unsigned bv[CMAX];
+    above = cum;
+  }
+  grp_sel = __shfl_sync(0xffffffffu, grp_sel, src_lane);
+  above = __shfl_sync(0xffffffffu, above, src_lane);
+
+  // this CTA's bins of the boundary group to every other CTA (8 x 16 B each)
+  if (CL) {
+    const uint4* src = reinterpret_cast<const uint4*>(hist + grp_sel * 32);
+    for (int o = lane; o < 8 * CS; o += 32) {
+      const int rk = o >> 3, ch = o & 7;
+      if (rk != c) st_async_v4(cluster_addr(gbins + c * 32 + ch * 4, rk), src[ch], cluster_addr(&bars[1], rk));
+    }
+    bounded_wait(&bars[1], 0, w);
+  }
+  // the group's 32 bins summed over the CTAs, descending: lane l takes bin 32 g + 31 - l
+  const int bin = grp_sel * 32 + 31 - lane;
+  unsigned bc = hist[bin];
+  if (CL) {
 #pragma unroll
     for (int rk = 0; rk < CMAX; ++rk)
-      if (rk < CS) bv[rk] = rank_ptr<CL>(cluster, hist, rk)[bin];
-    unsigned bc = 0;
+      if (rk < CS && rk != c) bc += gbins[rk * 32 + 31 - lane];
+  }
+  unsigned bincl = bc;
 #pragma unroll
-    for (int rk = 0; rk < CMAX; ++rk)
-      if (rk < CS) bc += bv[rk];
-    unsigned bincl = bc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned u = __shfl_up_sync(0xffffffffu, bincl, o);
-      if (lane >= o) bincl += u;
-    }
-    const unsigned nd2 = nd - above;
-    const unsigned bexcl = bincl - bc;
-    if (bexcl < nd2 && nd2 <= bincl) {
-      res[i][0] = bin;
-      res[i][1] = static_cast<int>(above + bexcl);
-    }
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned u = __shfl_up_sync(0xffffffffu, bincl, o);
+    if (lane >= o) bincl += u;
+  }
+  const unsigned nd2 = nd - above;
+  const unsigned bexcl = bincl - bc;
+  if (bexcl < nd2 && nd2 <= bincl) {
+    res[0][0] = bin;
+    res[0][1] = static_cast<int>(above + bexcl);
   }
 }
 
@@ -515,9 +515,14 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   __shared__ __align__(16) unsigned G1[CMAX * 64];                  // group counts of every CTA
   __shared__ __align__(16) unsigned G2[CMAX * 64];
   __shared__ __align__(16) unsigned G3[CMAX * 32];
+  __shared__ __align__(16) unsigned B1[CL ? CMAX * 32 : 1];         // boundary-group bins of every CTA
+  __shared__ __align__(16) unsigned B2[CL ? CMAX * 32 : 1];
+  __shared__ __align__(16) unsigned B3[CL ? CMAX * 32 : 1];
+  __shared__ __align__(8) uint64_t xbar[kNumExchanges];
+  __shared__ __align__(8) int cin[CMAX][2];                         // (gt, eq) totals of earlier CTAs
   __shared__ int res[1][2];
   __shared__ int wtot[NW];                                          // packed (gt, eq) per warp
-  __shared__ int cin[CMAX][2];                                      // (gt, eq) totals of earlier CTAs
+  __shared__ int abort_flag;
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = CL ? static_cast<int>(cluster.num_blocks()) : 1;
   const int c = CL ? static_cast<int>(cluster.block_rank()) : 0;
@@ -536,6 +541,25 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   }
   if (keff <= 0) return;   // the same for every CTA of the row
 
+  const WaitCtl wctl{&abort_flag, a.status, a.wait_ns};
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    if (CL) {
+      for (int i = 0; i < kNumExchanges; ++i) mbar_init(&xbar[i], 1);
+      // the bytes every other CTA pushes: group counts (NG x 4 B), boundary
+      // bins (128 B), and the totals of the earlier CTAs (8 B each)
+      const uint32_t peers = static_cast<uint32_t>(CS - 1);
+      mbar_arrive_expect_tx(&xbar[kXGroups1], peers * 64 * 4);
+      mbar_arrive_expect_tx(&xbar[kXBins1], peers * 128);
+      mbar_arrive_expect_tx(&xbar[kXGroups2], peers * 64 * 4);
+      mbar_arrive_expect_tx(&xbar[kXBins2], peers * 128);
+      mbar_arrive_expect_tx(&xbar[kXGroups3], peers * 32 * 4);
+      mbar_arrive_expect_tx(&xbar[kXBins3], peers * 128);
+      mbar_arrive_expect_tx(&xbar[kXTotals], static_cast<uint32_t>(c) * 8);
+      fence_barrier_init();
+    }
+  }
+  if (CL) cluster_arrive_relaxed();
   {
     uint4* z = reinterpret_cast<uint4*>(H1);
     for (int i = threadIdx.x; i < 512; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
@@ -580,9 +604,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   for (int j = 0; j < PT; ++j)
     if ((vmask >> j) & 1u) atomicAdd(&H1[key[j] >> 21], 1u);
   __syncthreads();
-  push_group_counts<64, CL>(cluster, CS, c, H1, G1);
-  sync_row<CL>(cluster);
-  find_bins<64, CL, CMAX>(cluster, CS, H1, G1, 1, &keff, res);
+  if (CL) cluster_wait();                              // every CTA's mbarriers are initialised
+  select_digit<64, CL, CMAX>(CS, c, H1, G1, B1, &xbar[kXGroups1], keff, res, wctl);
   __syncthreads();
   unsigned pre = static_cast<unsigned>(res[0][0]);
   int above = res[0][1];
@@ -593,9 +616,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   for (int j = 0; j < PT; ++j)
     if (((vmask >> j) & 1u) && (key[j] >> 21) == pre) atomicAdd(&H2[(key[j] >> 10) & 2047u], 1u);
   __syncthreads();
-  push_group_counts<64, CL>(cluster, CS, c, H2, G2);
-  sync_row<CL>(cluster);
-  find_bins<64, CL, CMAX>(cluster, CS, H2, G2, 1, &need, res);
+  select_digit<64, CL, CMAX>(CS, c, H2, G2, B2, &xbar[kXGroups2], need, res, wctl);
   __syncthreads();
   pre = (pre << 11) | static_cast<unsigned>(res[0][0]);
   above += res[0][1];
@@ -606,9 +627,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   for (int j = 0; j < PT; ++j)
     if (((vmask >> j) & 1u) && (key[j] >> 10) == pre) atomicAdd(&H3[key[j] & 1023u], 1u);
   __syncthreads();
-  push_group_counts<32, CL>(cluster, CS, c, H3, G3);
-  sync_row<CL>(cluster);
-  find_bins<32, CL, CMAX>(cluster, CS, H3, G3, 1, &need, res);
+  select_digit<32, CL, CMAX>(CS, c, H3, G3, B3, &xbar[kXGroups3], need, res, wctl);
   __syncthreads();
   const unsigned T = (pre << 10) | static_cast<unsigned>(res[0][0]);
   above += res[0][1];
@@ -638,57 +657,66 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
     }
     gb = before & 0xFFFF;
     eb = before >> 16;
-    if (CL && threadIdx.x < CS && static_cast<int>(threadIdx.x) > c) {
-      int* dst = cluster.map_shared_rank(&cin[0][0], static_cast<int>(threadIdx.x));
-      dst[2 * c] = total & 0xFFFF;        // per-CTA totals <= 16384
-      dst[2 * c + 1] = total >> 16;
-    }
+    // per-CTA totals (<= 16384 each) to every later CTA
+    if (CL && threadIdx.x < CS && static_cast<int>(threadIdx.x) > c)
+      st_async_v2(cluster_addr(&cin[c][0], threadIdx.x), static_cast<uint32_t>(total & 0xFFFF),
+                  static_cast<uint32_t>(total >> 16), cluster_addr(&xbar[kXTotals], threadIdx.x));
   }
   if (CL) {
-    cluster.sync();
+    cluster_arrive_relaxed();           // this CTA has sent everything it sends
+    if (warp == 0) bounded_wait(&xbar[kXTotals], 0, wctl);
+    __syncthreads();
     for (int rk = 0; rk < c; ++rk) {
       gb += cin[rk][0];
       eb += cin[rk][1];
     }
   }
-  const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
-  const unsigned lt = (1u << lane) - 1u;
+  const bool aborted = abort_flag != 0;   // uniform: set before the last block barrier
+  if (!aborted) {
+    const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
+    const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int j = 0; j < NSLAB; ++j) {
-    unsigned bg[4], be[4];
+    for (int j = 0; j < NSLAB; ++j) {
+      unsigned bg[4], be[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const bool v = (vmask >> (4 * j + e)) & 1u;
-      bg[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] > T);
-      be[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] == T);
-    }
-    // elements of lower lanes in this slab come first
-    int g = gb, q = eb;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      g += __popc(bg[e] & lt);
-      q += __popc(be[e] & lt);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const bool gt = (bg[e] >> lane) & 1u;
-      const bool eq = (be[e] >> lane) & 1u;
-      if (gt || (eq && q < need_eq)) {
-        const int rank = g + min(q, need_eq);
-        if (rank < a.k) {
-          const int64_t pos = run + j * 128 + 4 * lane + e;
-          oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
-          if (osv) osv[rank] = radix_value(key[4 * j + e]);   // no reload: the key is the score
-        }
+      for (int e = 0; e < 4; ++e) {
+        const bool v = (vmask >> (4 * j + e)) & 1u;
+        bg[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] > T);
+        be[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] == T);
       }
-      g += gt ? 1 : 0;
-      q += eq ? 1 : 0;
-    }
+      // elements of lower lanes in this slab come first
+      int g = gb, q = eb;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      gb += __popc(bg[e]);
-      eb += __popc(be[e]);
+      for (int e = 0; e < 4; ++e) {
+        g += __popc(bg[e] & lt);
+        q += __popc(be[e] & lt);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool gt = (bg[e] >> lane) & 1u;
+        const bool eq = (be[e] >> lane) & 1u;
+        if (gt || (eq && q < need_eq)) {
+          const int rank = g + min(q, need_eq);
+          if (rank < a.k) {
+            const int64_t pos = run + j * 128 + 4 * lane + e;
+            oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
+            if (osv) osv[rank] = radix_value(key[4 * j + e]);   // no reload: the key is the score
+          }
+        }
+        g += gt ? 1 : 0;
+        q += eq ? 1 : 0;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        gb += __popc(bg[e]);
+        eb += __popc(be[e]);
+      }
     }
+  }
+  if (CL) {
+    cluster_wait();                     // every CTA has sent everything it sends
+    if (aborted && warp == 0)           // let what is still in flight to this CTA land
+      for (int i = 0; i < kNumExchanges; ++i) drain_wait(&xbar[i], 0, 1000000);
   }
 }
 
