@@ -360,10 +360,9 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
 //
 // A row is taken by CS <= 16 CTAs of 512 threads (a thread-block cluster when
 // CS > 1).  Warp w of CTA c owns the contiguous run of 32 * PT positions
-// starting at (c * 16 + w) * 32 * PT; in slab j of the run, lane l holds the
-// four positions j * 128 + 4 l + {0..3} (one coalesced 16-byte load per lane
-// and slab) as order-preserving uint32 keys in registers for the whole
-// kernel.  The exact k-th key T is found digit by digit (11 + 11 + 10 bits):
+// starting at (c * 16 + w) * 32 * PT, and lane l the PT positions from
+// l * PT on within it (PT / 4 16-byte loads), held as order-preserving
+// uint32 keys in registers for the whole kernel.  The exact k-th key T is found digit by digit (11 + 11 + 10 bits):
 // each pass histograms, in its own shared-memory array, the keys matching the
 // digits found so far.  The CTAs then exchange counts by one-way pushes: each
 // sends its group counts (32 bins a group) into a slot of every other CTA's
@@ -374,8 +373,9 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
 // exchange, each completed once), so a CTA waits only for its own data: there
 // is no cluster-wide barrier or remote read on the way to T.  The output rank
 // of a selected element is #greater before it + min(#equal before it, #equal
-// taken), from warp scans within slabs, warp totals within the CTA and
-// per-CTA totals pushed to the later CTAs.  One relaxed cluster barrier opens
+// taken), from a scan over the lanes, warp totals within the CTA and
+// per-CTA totals pushed to the later CTAs; each lane then writes its own
+// selected keys in position order.  One relaxed cluster barrier opens
 // the exchanges (every CTA's mbarriers are initialised) and one closes the
 // kernel (no CTA exits while a peer may still push to it).  Every wait is
 // bounded; a CTA whose wait ran out records the timeout, keeps sending what
@@ -570,13 +570,14 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   }
 
   const int64_t run = (static_cast<int64_t>(c) * NW + warp) * 32 * PT;   // first position of this warp
+  const int64_t first = run + static_cast<int64_t>(lane) * PT;          // first position of this lane
   const float* row = a.scores + static_cast<int64_t>(r) * a.row_stride;
   unsigned key[PT];
   unsigned vmask = 0;
   if ((a.row_stride & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0 && run + 32 * PT <= n) {
 #pragma unroll
     for (int j = 0; j < NSLAB; ++j) {
-      const float4 f = *reinterpret_cast<const float4*>(row + run + j * 128 + 4 * lane);
+      const float4 f = *reinterpret_cast<const float4*>(row + first + 4 * j);
       key[4 * j] = radix_key(f.x);
       key[4 * j + 1] = radix_key(f.y);
       key[4 * j + 2] = radix_key(f.z);
@@ -585,15 +586,11 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
     vmask = PT == 32 ? 0xffffffffu : ((1u << PT) - 1u);
   } else {
 #pragma unroll
-    for (int j = 0; j < NSLAB; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int64_t pos = run + j * 128 + 4 * lane + e;
-        key[4 * j + e] = 0;
-        if (pos < n) {
-          key[4 * j + e] = radix_key(row[pos]);
-          vmask |= 1u << (4 * j + e);
-        }
+    for (int i = 0; i < PT; ++i) {
+      key[i] = 0;
+      if (first + i < n) {
+        key[i] = radix_key(row[first + i]);
+        vmask |= 1u << i;
       }
     }
   }
@@ -633,7 +630,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   above += res[0][1];
   const int need_eq = keff - above;     // elements equal to T that are taken
 
-  // ---- ordered output: warp totals, CTA totals, then per-slab ballots
+  // ---- ordered output: lane scan, warp totals, CTA totals, then each lane's keys
+  int lane_before = 0;                  // packed (gt, eq) of the lower lanes of this warp
   {
     int x = 0;
 #pragma unroll
@@ -642,20 +640,26 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
       x += (v && key[j] > T) ? 1 : 0;
       x += (v && key[j] == T) ? 0x10000 : 0;
     }
-    x = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(x)));   // <= 32 * PT each field
-    if (lane == 0) wtot[warp] = x;
+    int incl = x;                       // <= 32 * PT each field
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    lane_before = incl - x;
+    if (lane == 31) wtot[warp] = incl;
   }
   __syncthreads();
-  int gb = 0, eb = 0;                   // elements before this warp's run
+  int gb = 0, eb = 0;                   // elements before this lane's positions
   {
-    int before = 0, total = 0;
+    int before = lane_before, total = 0;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const int v = wtot[w];
       before += w < warp ? v : 0;
       total += v;
     }
-    gb = before & 0xFFFF;
+    gb = before & 0xFFFF;               // <= 16384 each field within a CTA
     eb = before >> 16;
     // per-CTA totals (<= 16384 each) to every later CTA
     if (CL && threadIdx.x < CS && static_cast<int>(threadIdx.x) > c)
@@ -674,43 +678,22 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   const bool aborted = abort_flag != 0;   // uniform: set before the last block barrier
   if (!aborted) {
     const int* map = a.idx_map ? a.idx_map + static_cast<int64_t>(r) * a.map_stride : nullptr;
-    const unsigned lt = (1u << lane) - 1u;
+    int g = gb, q = eb;
 #pragma unroll
-    for (int j = 0; j < NSLAB; ++j) {
-      unsigned bg[4], be[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool v = (vmask >> (4 * j + e)) & 1u;
-        bg[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] > T);
-        be[e] = __ballot_sync(0xffffffffu, v && key[4 * j + e] == T);
-      }
-      // elements of lower lanes in this slab come first
-      int g = gb, q = eb;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        g += __popc(bg[e] & lt);
-        q += __popc(be[e] & lt);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool gt = (bg[e] >> lane) & 1u;
-        const bool eq = (be[e] >> lane) & 1u;
-        if (gt || (eq && q < need_eq)) {
-          const int rank = g + min(q, need_eq);
-          if (rank < a.k) {
-            const int64_t pos = run + j * 128 + 4 * lane + e;
-            oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
-            if (osv) osv[rank] = radix_value(key[4 * j + e]);   // no reload: the key is the score
-          }
+    for (int i = 0; i < PT; ++i) {
+      const bool v = (vmask >> i) & 1u;
+      const bool gt = v && key[i] > T;
+      const bool eq = v && key[i] == T;
+      if (gt || (eq && q < need_eq)) {
+        const int rank = g + min(q, need_eq);
+        if (rank < a.k) {
+          const int64_t pos = first + i;
+          oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
+          if (osv) osv[rank] = radix_value(key[i]);   // no reload: the key is the score
         }
-        g += gt ? 1 : 0;
-        q += eq ? 1 : 0;
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        gb += __popc(bg[e]);
-        eb += __popc(be[e]);
-      }
+      g += gt ? 1 : 0;
+      q += eq ? 1 : 0;
     }
   }
   if (CL) {
