@@ -78,3 +78,13 @@ def test_topk_ragged_lengths_and_short_rows(ctx):
     lengths = np.array([0, 1, 5, 63, 64, 65, 4096, 12345, 20000])
     _check(ctx, x, 64, lengths)
     _check(ctx, x, 2048, lengths)
+
+
+@pytest.mark.parametrize("kind", ["gauss", "ties", "const"])
+def test_topk_ragged_rows_in_the_widest_clusters(ctx, kind):
+    """Rows of 131072 positions take 16-CTA clusters; valid prefixes that end
+    inside one CTA, leave 15 CTAs of the cluster empty, or are empty."""
+    rng = np.random.default_rng(7)
+    x = _rows(kind, 4, 131072, rng)
+    _check(ctx, x, 2048, np.array([70001, 131072, 3, 0]))
+    _check(ctx, x, 2048, np.array([8191, 8192, 8193, 131071]))
