@@ -359,7 +359,12 @@ LI_API li_status li_score_topk_static(li_ctx* ctx, const li_cache* cache, const 
 
 /* Top-k of `rows` fp32 rows: row r is scores[r * row_stride + 0 .. n_r),
  * n_r = lengths ? lengths[r] : n (lengths[r] is clamped to [0, n]).
- * out_idx [rows][k] int32, out_score [rows][k] fp32 or NULL. */
+ * out_idx [rows][k] int32, out_score [rows][k] fp32 or NULL.
+ * Rows of up to 131072 positions are selected by one cluster of CTAs per
+ * row that exchange digit counts through each other's shared memory; those
+ * waits are bounded like every other.  A row whose wait ran out records
+ * LI_ERR_DEVICE_TIMEOUT in the status word and leaves slots 0..k_eff-1
+ * unwritten (the padding after them is written first). */
 LI_API li_status li_topk(li_ctx* ctx, const float* scores, int rows, int n, int64_t row_stride,
                   const int32_t* lengths, int k, int32_t* out_idx, float* out_score, void* ws,
                   size_t ws_bytes, void* stream);
