@@ -51,6 +51,7 @@ def parse():
     p.add_argument("--no-other-contexts", action="store_true")
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-fused", action="store_true")
+    p.add_argument("--no-score-only", action="store_true")
     p.add_argument("--no-two-branch", action="store_true")
     p.add_argument("--no-recall", action="store_true")
     return p.parse_args()
@@ -128,7 +129,7 @@ def run_reference(args):
     return 0
 
 
-def cpu_baseline(inp, hnew, Wd, Wk, budget_s=10.0):
+def _oracle_rate(inp, hnew, Wd, Wk, budget_s):
     keys, t0 = 0, time.perf_counter()
     reps = 0
     while True:
@@ -137,9 +138,25 @@ def cpu_baseline(inp, hnew, Wd, Wk, budget_s=10.0):
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": keys / dt, "unit": "keys/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"{reps} sequence-steps (HS + DSA-style group step of one sequence, cycling over the "
-                      f"{inp.wl.batch} sequences), fp64 NumPy, {dt:.1f} s"}
+    return keys / dt, reps, dt
+
+
+def cpu_baseline(inp, hnew, Wd, Wk, budget_s=10.0, one_thread_s=3.0):
+    """The oracle on the host: all cores (BLAS threads as NumPy starts them),
+    then a shorter sample with BLAS held to one thread."""
+    value, reps, dt = _oracle_rate(inp, hnew, Wd, Wk, budget_s)
+    out = {"value": value, "unit": "keys/s", "cores": cpu_cores(), "kind": "oracle",
+           "sample": f"{reps} sequence-steps (HS + DSA-style group step of one sequence, cycling over the "
+                     f"{inp.wl.batch} sequences), fp64 NumPy, {dt:.1f} s"}
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return out
+    with threadpool_limits(limits=1):
+        v1, reps1, dt1 = _oracle_rate(inp, hnew, Wd, Wk, one_thread_s)
+    out["one_thread"] = {"value": v1, "unit": "keys/s", "cores": 1,
+                         "sample": f"{reps1} sequence-steps, BLAS limited to one thread, {dt1:.1f} s"}
+    return out
 
 
 # ------------------------------------------------------------------ clocks
@@ -675,6 +692,54 @@ def recall_leg(step, dev):
     return res
 
 
+def score_only_leg(step, args, flush, stream, dist, dev, world):
+    """The step's two paths without construction -- no append, and no query
+    absorption or conversion (the queries absorbed and converted by the last
+    full step are reused): the HS anchor scan with its two selections and the
+    3 followers' gathers and selections, against the 4 DSA-style key scans and
+    selections.  Both from captured graphs, L2 flushed before each replay,
+    CUDA events on the stream.  Then the whole step with construction (both
+    step graphs) replayed with no flush in between, so that the next step
+    finds in L2 whatever of the caches the previous one left there."""
+    g, wl = step.g, step.wl
+    step.reset()
+    step.hs_path()
+    step.dsa_path()
+    torch.cuda.synchronize()
+
+    def hs_only():
+        g.idx = step.hs_idx
+        g.hs_anchor(0)
+        for l in range(1, wl.group):
+            g.hs_follower(l)
+
+    def dsa_only():
+        g.idx = step.dsa_idx
+        for l in range(wl.group):
+            g.dsa_score_topk(l)
+
+    t_hs, t_dsa = graph_times([hs_only, dsa_only], args, flush, stream, dist, dev)
+    warm = []
+    for i in range(args.warmup + args.steps):
+        step.reset()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step.graphs[0].replay()
+        step.graphs[1].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            warm.append(e0.elapsed_time(e1))
+    t_warm = max_over_ranks(statistics.mean(warm), dist, dev)
+    keys = step.hs_keys + step.dsa_keys
+    return {"hs_ms": t_hs, "dsa_ms": t_dsa, "hs_speedup_over_dsa": t_dsa / t_hs,
+            "hs_keys_per_s": world * step.hs_keys / (t_hs / 1e3),
+            "dsa_keys_per_s": world * step.dsa_keys / (t_dsa / 1e3),
+            "warm_l2_step_ms": t_warm, "warm_l2_keys_per_s": world * keys / (t_warm / 1e3),
+            "mode": "score + top-k only (queries absorbed beforehand), L2 flushed before each replay; "
+                    "warm_l2: the whole step with construction, replays back to back without a flush"}
+
+
 def fused_leg(step, args, flush, stream, dist, dev, world):
     """Query absorption, scoring and selection of all G layers over the full
     prefix, for the training-aware instantiation (every layer's query from
@@ -934,6 +999,13 @@ def main():
                       "eager_value": whole_job_rate(world, keys, args.steps, te_eager),
                       "eager_ms_per_step": te_eager / args.steps,
                       "eager_mode": "serial, with every library call issued eagerly"}
+
+    # ---- both paths without construction, and the whole step with a warm L2
+    if not args.no_score_only:
+        try:
+            out["paths"]["score_only"] = score_only_leg(step, args, flush, stream, dist, dev, world)
+        except Exception as e:      # reported in the line; the measured figures above stand
+            out["paths"]["score_only"] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     # ---- full LatentIndex for the whole group: 4 per-layer scans of the shared
     #      latent against one fused scan with the 4 layers' queries stacked
