@@ -357,9 +357,14 @@ LI_API li_status li_score_topk_static(li_ctx* ctx, const li_cache* cache, const 
 
 /* ----------------------------------------------------- a4: plain selection */
 
-/* Top-k of `rows` fp32 rows: row r is scores[r * row_stride + 0 .. n_r),
- * n_r = lengths ? lengths[r] : n (lengths[r] is clamped to [0, n]).
+/* Top-k of `rows` fp32 rows (LatentIndex summary, Sec. 3.1: every layer
+ * keeps its own top-k tokens; Sec. C.4: the budget is capped by the valid
+ * prefix), by the rule under "Selections" above: row r is
+ * scores[r * row_stride + 0 .. n_r), n_r = lengths ? lengths[r] : n
+ * (lengths[r] is clamped to [0, n]; lengths is [rows] int32 or NULL).
  * out_idx [rows][k] int32, out_score [rows][k] fp32 or NULL.
+ * ws: li_workspace_bytes(ctx, rows, 1, n, 1, k, 0) bytes.  Needs
+ * rows <= 65535; rows longer than 131072 positions take a multi-kernel path.
  * Rows of up to 131072 positions are selected by one cluster of CTAs per
  * row that exchange digit counts through each other's shared memory; those
  * waits are bounded like every other.  A row whose wait ran out records
