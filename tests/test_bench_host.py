@@ -56,3 +56,36 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     assert r["kind"] == "oracle" and r["unit"] == "keys/s" and r["value"] > 0
     assert r["cores"] == bench.cpu_cores() >= 1
     assert r["one_thread"]["cores"] == 1 and r["one_thread"]["value"] > 0
+
+
+def _reference_line(extra_env=None, workload_idx=1):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **(extra_env or {}))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", str(workload_idx),
+                        "--steps", "1", "--warmup", "0"], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    return [json.loads(x) for x in lines]
+
+
+def test_reference_arm_prints_one_oracle_line_with_its_own_figures():
+    """The reference arm times the oracle on the host: its cpu_baseline and
+    e2e figures are the line's own value, with nothing crossing PCIe."""
+    lines = _reference_line()
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["impl"] == "reference" and d["unit"] == "keys/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["dtype"] == "f64" and d["data"] == "synthetic"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"].startswith("v32-decode-bf16-n8k")
+
+
+def test_reference_arm_prints_nothing_on_other_ranks():
+    assert _reference_line({"RANK": "1", "WORLD_SIZE": "2"}) == []
