@@ -362,9 +362,9 @@ cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st) {
 // CS > 1).  Warp w of CTA c owns the contiguous run of 32 * PT positions
 // starting at (c * 16 + w) * 32 * PT, and lane l the PT positions from
 // l * PT on within it (PT / 4 16-byte loads), held as order-preserving
-// uint32 keys in registers for the whole kernel.  The exact k-th key T is found digit by digit (11 + 11 + 10 bits):
-// each pass histograms, in its own shared-memory array, the keys matching the
-// digits found so far.  The CTAs then exchange counts by one-way pushes: each
+// uint32 keys in registers for the whole kernel.  The exact k-th key T is
+// found digit by digit (11 + 11 + 10 bits): each pass histograms, in its own
+// shared-memory array, the keys matching the digits found so far.  The CTAs then exchange counts by one-way pushes: each
 // sends its group counts (32 bins a group) into a slot of every other CTA's
 // shared memory; every CTA sums the same slots, so all find the same
 // boundary group, and each then sends that group's 32 bins the same way and
