@@ -89,3 +89,14 @@ def test_reference_arm_prints_one_oracle_line_with_its_own_figures():
 
 def test_reference_arm_prints_nothing_on_other_ranks():
     assert _reference_line({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_prefill_oracle_sample_counts_the_causal_prefixes():
+    """Queries at positions 64512..65535 of a 65536-token prefix see
+    p + 1 tokens each: 1024 * (64513 + 65536) / 2 pairs a layer.  A sample
+    of two rows is the first and the last query, in each of the 4 layers."""
+    r = bench.prefill_cpu_baseline(rows=2)
+    assert r["keys_per_layer"] == 1024 * (64513 + 65536) // 2 == 66_585_088
+    assert r["keys_sampled"] == 4 * (64513 + 65536)
+    assert r["kind"] == "oracle" and r["unit"] == "keys/s" and r["value"] > 0
+    assert r["extrapolated_layer_s"] == pytest.approx(r["keys_per_layer"] / r["value"])
