@@ -42,7 +42,7 @@ METRIC = "decode indexer keys scored/s and % HBM roofline at 8K-128K ctx; HS vs 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=64)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", type=int, default=3)
