@@ -38,6 +38,40 @@ def test_hand_example_scores_and_selection():
                              np.array(a["w"])).tolist() == a["scores"]
 
 
+def test_hand_example_kth_score():
+    """The selection boundary used by the tolerance rule: the k_eff-th best
+    score, worked by hand on the example's scores (ties and k past n)."""
+    a = _golden("hand_example.json")["anchor"]
+    s = np.array(a["scores"])
+    for k, v in a["kth"].items():
+        assert indexer.kth_score(s, int(k)) == v
+    for k, v in a["kth_n2"].items():
+        assert indexer.kth_score(s, int(k), n=2) == v
+    assert indexer.kth_score(s, 3, n=0) == np.inf
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_kth_score_counts(seed):
+    """Pure-Python characterisation without sorting: v is the k_eff-th best
+    score iff v is one of the scores, fewer than k_eff scores exceed it and
+    at least k_eff reach it; it is also the lowest score the top-k keeps."""
+    rng = np.random.default_rng(40 + seed)
+    for row in _adversarial_rows(rng):
+        vals = row.astype(float).tolist()
+        for k in (1, 2, 7, len(vals), len(vals) + 3):
+            for n in (len(vals), len(vals) // 2):
+                v = indexer.kth_score(row, k, n)
+                pre = vals[:n]
+                keff = min(k, n)
+                if keff == 0:
+                    assert v == np.inf
+                    continue
+                assert v in pre
+                assert sum(1 for x in pre if x > v) < keff <= sum(1 for x in pre if x >= v)
+                idx, kept = indexer.topk(row, k, n)
+                assert kept[idx >= 0].min() == v
+
+
 def test_hand_example_bias():
     g = _golden("hand_example.json")
     c = np.array(g["latent"], float)

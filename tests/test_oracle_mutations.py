@@ -55,8 +55,24 @@ def _topk_unsorted_output(scores, k, n=None):
     return idx, vals
 
 
+def _kth_off_by_one(scores, k, n=None):
+    s = np.asarray(scores, float)[: (len(scores) if n is None else n)]
+    keff = min(int(k), len(s))
+    if keff == 0:
+        return np.inf
+    return float(np.sort(s)[::-1][min(keff, len(s) - 1)])
+
+
+def _kth_distinct_values(scores, k, n=None):
+    # a slip: the k-th best distinct value (ties counted once)
+    s = np.asarray(scores, float)[: (len(scores) if n is None else n)]
+    u = np.unique(s)[::-1]
+    return np.inf if len(s) == 0 else float(u[min(int(k), len(u)) - 1])
+
+
 PIN_SETS = [pins.test_hand_example_scores_and_selection, pins.test_hand_example_hs,
-            pins.test_hand_example_bias,
+            pins.test_hand_example_bias, pins.test_hand_example_kth_score,
+            lambda: pins.test_kth_score_counts(0),
             lambda: pins.test_absorbed_scoring_equals_explicit_keys(0),
             lambda: pins.test_topk_matches_sorted(5)]
 
@@ -67,6 +83,8 @@ PIN_SETS = [pins.test_hand_example_scores_and_selection, pins.test_hand_example_
     ("wrong absorbed operand", "absorb", _absorb_wrong_operand),
     ("ties to the higher index", "topk", _topk_high_index_ties),
     ("selection not in position order", "topk", _topk_unsorted_output),
+    ("k-th score off by one", "kth_score", _kth_off_by_one),
+    ("k-th score over distinct values", "kth_score", _kth_distinct_values),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, attr, bad):
     monkeypatch.setattr(ix, attr, bad)
