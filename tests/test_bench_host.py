@@ -100,3 +100,16 @@ def test_prefill_oracle_sample_counts_the_causal_prefixes():
     assert r["keys_sampled"] == 4 * (64513 + 65536)
     assert r["kind"] == "oracle" and r["unit"] == "keys/s" and r["value"] > 0
     assert r["extrapolated_layer_s"] == pytest.approx(r["keys_per_layer"] / r["value"])
+
+
+def test_cpu_baseline_configs_time_whole_group_steps():
+    """The oracle timed on the smaller decode workloads: every sequence of a
+    step (tiny-f32 builds its latent from the hidden states first)."""
+    r = bench.cpu_baseline_configs(indices=(0, 1), budget_s=0.05)
+    for i in (0, 1):
+        wl = workload(i)
+        d = r[wl.name]
+        hs, dsa = bench.keys_per_step(wl, generate(wl).lengths)
+        assert d["keys_per_step"] == hs + dsa
+        assert d["kind"] == "oracle" and d["unit"] == "keys/s" and d["value"] > 0
+        assert d["cores"] == bench.cpu_cores()
