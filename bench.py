@@ -54,6 +54,7 @@ def parse():
     p.add_argument("--no-score-only", action="store_true")
     p.add_argument("--no-two-branch", action="store_true")
     p.add_argument("--no-recall", action="store_true")
+    p.add_argument("--no-gate", action="store_true")
     return p.parse_args()
 
 
@@ -73,13 +74,14 @@ def config_of(wl, paths="HS + DSA-style, with construction"):
 
 # ------------------------------------------------------------------ CPU oracle leg
 
-def oracle_sample_step(inp, b, hnew, Wd, Wk):
+def oracle_sample_step(inp, b, hnew, Wd, Wk, latent=None):
     """The oracle's version of one sequence's group step (HS + DSA-style, with
-    construction of the new token's latent and keys)."""
+    construction of the new token's latent and keys).  latent: the cached
+    latent rows when the workload gives hidden states instead (tiny-f32)."""
     from oracle import indexer
     wl = inp.wl
     n = int(inp.lengths[b])
-    c = inp.latent[b, :n].astype(np.float64)
+    c = (inp.latent if latent is None else latent)[b, :n].astype(np.float64)
     indexer.latent(hnew[b], Wd)                          # anchor latent of the new token
     qt0, _ = indexer.absorb(inp.q[0][b, 0], inp.W_K[0])
     s0 = indexer.score(c, qt0, inp.w[0][b, 0])
@@ -139,6 +141,31 @@ def _oracle_rate(inp, hnew, Wd, Wk, budget_s):
             break
     dt = time.perf_counter() - t0
     return keys / dt, reps, dt
+
+
+def cpu_baseline_configs(indices=(0, 1, 2), budget_s=3.0):
+    """The oracle timed on whole group steps (every sequence of the batch) of
+    the smaller decode workloads, each for about budget_s of host time."""
+    from oracle import indexer
+    out = {}
+    for i in indices:
+        wl = workload(i)
+        inp = generate(wl)
+        hnew, Wd, Wk = construction_inputs(wl)
+        lat = indexer.latent(inp.hidden, inp.W_down) if inp.latent is None else None
+        keys, steps, t0 = 0, 0, time.perf_counter()
+        while True:
+            for b in range(wl.batch):
+                keys += oracle_sample_step(inp, b, hnew, Wd, Wk, lat)
+            steps += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        out[wl.name] = {"value": keys / dt, "unit": "keys/s", "cores": cpu_cores(), "kind": "oracle",
+                        "ms_per_step": 1e3 * dt / steps, "keys_per_step": keys // steps,
+                        "sample": f"{steps} whole group steps (HS + DSA-style, all {wl.batch} sequences, with "
+                                  f"construction), fp64 NumPy, {dt:.1f} s"}
+    return out
 
 
 def cpu_baseline(inp, hnew, Wd, Wk, budget_s=10.0, one_thread_s=3.0):
@@ -534,7 +561,10 @@ def prefill_leg(li, ctx, args, rank, dev):
             peaks = json.load(f)
     except Exception:
         pass
-    peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    # the scan is timed alone (an event pair around one launch): the burst
+    # GEMM figure is its denominator; the sustained one is given beside it
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", 1400.0))
     scan_tflops = flop / (statistics.mean(scan_ms) / 1e3) / 1e12 if scan_ms else None
     return {"workload": f"{wl.name}: {wl.queries} queries at positions {int(inp.q_pos.min())}..{int(inp.q_pos.max())}"
                         f" of a {wl.capacity}-position bf16 prefix, H {wl.heads}, d_c {wl.d_c}, k {wl.k}",
@@ -543,7 +573,9 @@ def prefill_leg(li, ctx, args, rank, dev):
             "select_ms": sum(sel_ms) / max(len(call_ms), 1),
             "roofline": {"bound": "tensor", "achieved": scan_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": (scan_tflops / peak) if scan_tflops else None,
-                         "peak_source": "measured cuBLAS bf16 GEMM, sustained (MEASURED_PEAKS.json)"},
+                         "peak_source": "measured cuBLAS bf16 GEMM, burst (MEASURED_PEAKS.json bf16_tflops): "
+                                        "the scan kernel is timed alone",
+                         "frac_of_sustained": (scan_tflops / peak_sus) if scan_tflops else None},
             "keys_per_s": wl.group * pairs / (sum(call_ms) / 1e3)}
 
 
@@ -808,6 +840,53 @@ def fused_leg(step, args, flush, stream, dist, dev, world):
                     f"absorb, one scan with {wl.group} x {wl.heads} MMA columns"}
 
 
+def gate_leg(step, args, flush, stream, dist, dev, world, lead_ms=4.0):
+    """Full LatentIndex for one layer of the step's workload, the decode
+    latent scan plus its top-k: li_score_topk over every sequence's whole
+    prefix, timed from a captured graph (L2 flushed before each replay, CUDA
+    events on the stream).  Algorithmic bytes are the cache rows read plus
+    the k selected indices a sequence writes; the roofline denominator is
+    the measured HBM copy bandwidth.  The scan and the selection are also
+    timed one by one (eager, an event pair around each launch, the GPU kept
+    ahead of the host)."""
+    li, g, wl, ctx = step.li, step.g, step.wl, step.ctx
+    step.reset()
+    torch.cuda.synchronize()
+
+    def one():
+        g.idx = step.hs_idx
+        g.score_topk(0)
+
+    (t_ms,) = graph_times([one], args, flush, stream, dist, dev)
+    n_tok = int(sum(int(n) for n in step.inp.lengths))
+    alg = n_tok * row_bytes(wl, wl.d_c) + wl.batch * wl.queries * wl.k * 4
+    peak, peak_kind = measured_peaks()
+    cycles = int(lead_ms * 1e-3 * 2.0e9)
+    li.li_profile_reset(ctx)
+    recs = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        torch.cuda._sleep(cycles)
+        li.li_profile_enable(ctx, True)
+        one()
+        li.li_profile_enable(ctx, False)
+        torch.cuda.synchronize()
+        recs += li.li_profile_read(ctx)
+        li.li_profile_reset(ctx)
+    step.status("after the scan + top-k leg")
+    per = {}
+    for r in recs:
+        per.setdefault(r["kernel"], []).append(r["ms"] * 1e3)
+    achieved = alg / (t_ms / 1e3) / 1e9
+    return {"call_us": t_ms * 1e3, "alg_bytes": alg, "achieved_gbs": achieved, "peak_gbs": peak,
+            "frac": achieved / peak, "keys_per_s": world * n_tok / (t_ms / 1e3),
+            "kernel_us": {k: statistics.median(v) for k, v in per.items()},
+            "target_us_at_0.70": alg / (0.70 * peak * 1e9) * 1e6,
+            "mode": f"li_score_topk (full LatentIndex, one layer: scan of {wl.batch} x {wl.length_range[1]} "
+                    f"{wl.cache_dtype} latent rows plus each sequence's top-{wl.k}), graph replay, L2 flushed "
+                    f"before each; peak: {peak_kind} HBM copy bandwidth"}
+
+
 def max_over_ranks(x, dist, dev):
     """The slowest rank's value (every rank gets it)."""
     t = torch.tensor([x], device=dev, dtype=torch.float64)
@@ -925,8 +1004,8 @@ def main():
            "paths": {"hs_ms": hs_mean, "dsa_ms": dsa_mean,
                      "hs_ms_median": statistics.median(hs_ms), "dsa_ms_median": statistics.median(dsa_ms),
                      "hs_keys_per_step": step.hs_keys, "dsa_keys_per_step": step.dsa_keys,
-                     "hs_keys_per_s": step.hs_keys / (hs_mean / 1e3),
-                     "dsa_keys_per_s": step.dsa_keys / (dsa_mean / 1e3),
+                     "hs_keys_per_s": world * step.hs_keys / (hs_mean / 1e3),
+                     "dsa_keys_per_s": world * step.dsa_keys / (dsa_mean / 1e3),
                      "hs_speedup_over_dsa": dsa_mean / hs_mean,
                      "profiled_hs_ms": statistics.mean(p_hs), "profiled_dsa_ms": statistics.mean(p_dsa)},
            "kernels": by_kernel,
@@ -1053,6 +1132,10 @@ def main():
     if not args.no_recall:
         out["paths"]["recall"] = recall_leg(step, dev)
 
+    # ---- the decode latent scan plus its top-k (full LatentIndex, one layer)
+    if not args.no_gate:
+        out["scan_topk"] = gate_leg(step, args, flush, stream, dist, dev, world)
+
     # ---- HS against DSA-style at the shorter contexts (same library, same protocol)
     if not args.no_other_contexts:
         other = {}
@@ -1090,6 +1173,19 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, step.hnew, step.Wd, step.Wk)
+        out["cpu_baseline"]["configs"] = cpu_baseline_configs()
+
+    # ---- flat summary: HS against DSA-style keys/s at each context length
+    ctxs = {wl.name: out["paths"]}
+    ctxs.update(out["paths"].get("other_contexts", {}))
+    for name, d in ctxs.items():
+        tag = {"v32-decode-bf16-n8k": "8k", "batched-ragged-bf16-n32k": "32k",
+               "long-e4m3-n128k": "128k"}.get(name, name)
+        out[f"hs_keys_per_s_{tag}"] = d["hs_keys_per_s"]
+        out[f"dsa_keys_per_s_{tag}"] = d["dsa_keys_per_s"]
+        out[f"hs_speedup_over_dsa_{tag}"] = d["hs_speedup_over_dsa"]
+    if "scan_topk" in out:
+        out["scan_topk_frac_hbm"] = out["scan_topk"]["frac"]
     if rank == 0:
         print(json.dumps(out))
     step.graphs = None
