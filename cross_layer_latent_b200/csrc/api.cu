@@ -523,7 +523,7 @@ li_status run_topk_chunked(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L
     return fail(ctx, LI_ERR_UNSUPPORTED, "selection rows longer than %d", kMaxTopkChunks * kTopkChunk);
   if (t.rows > 65535) return fail(ctx, LI_ERR_UNSUPPORTED, "more than 65535 selection rows");
   static const char* names[4] = {"topk_hist", "topk_filter", "topk_select", "topk_emit"};
-  for (int stage = t.hist_ready ? 1 : 0; stage < 4; ++stage) {
+  for (int stage = 0; stage < 4; ++stage) {
     const int grid = stage == 2 ? t.rows : t.rows * t.n_chunks;
     Launch Lc(ctx, st, names[stage], grid, stage == 2 ? 1024 : kTopkThreads, 0);
     const cudaError_t e = launch_topk_stage(stage, t, st);
@@ -554,9 +554,7 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   // 467 us, against 566 us for the chunked multi-kernel path).
   if (t.rows > 65535) return fail(ctx, LI_ERR_UNSUPPORTED, "more than 65535 selection rows");
   if (t.n <= kClusterMaxN) {
-    const int64_t cs_lat = topk_cluster_size(t.n, kTopkKeysLatency, t.rows);
-    const int kpt = static_cast<int64_t>(t.rows) * cs_lat <= 2 * static_cast<int64_t>(ctx->num_sms)
-                        ? kTopkKeysLatency : kTopkKeysThroughput;
+    const int kpt = topk_keys_per_thread(t.n, t.rows, ctx->num_sms);
     int cs = 0;
     Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);
     const cudaError_t e = launch_topk_cluster(t, st, &cs, kpt);
@@ -567,7 +565,6 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   }
   li_status s = clear_select_state(ctx, ws, L, t.rows, st);
   if (s != LI_OK) return s;
-  t.hist_ready = false;
   return run_topk_chunked(ctx, t, ws, L, st);
 }
 
@@ -1128,10 +1125,15 @@ __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 constexpr int kStaticMaxDevices = 64;
 std::mutex g_static_mu;
+// Per device: the scratch's device address and the CUDA context it was
+// looked up in (a device reset replaces the context and unmaps the old one).
 void* g_static_addr[kStaticMaxDevices] = {};
+CUcontext g_static_cuctx[kStaticMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 
 // Device address of the scratch on the current device, looked up once per
-// device (the lookup is the only setup this entry point needs).
+// device and context (the lookup is the only setup this entry point needs).
 li_status static_scratch(li_ctx* c, void** out, const char* what) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1141,8 +1143,22 @@ li_status static_scratch(li_ctx* c, void** out, const char* what) {
                 dev);
   if (dev < 0 || dev >= kStaticMaxDevices)
     return fail(c, LI_ERR_UNSUPPORTED, "%s: device ordinal %d above %d", what, dev, kStaticMaxDevices - 1);
+  static CtxGetCurrentFn ctx_current = [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    const cudaError_t r = cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q);
+    return (r == cudaSuccess && q == cudaDriverEntryPointSuccess) ? reinterpret_cast<CtxGetCurrentFn>(fn) : nullptr;
+  }();
+  if (!ctx_current) return fail(c, LI_ERR_CUDA, "%s: cuCtxGetCurrent is unavailable", what);
+  CUcontext cur = nullptr;
+  if (ctx_current(&cur) == CUDA_SUCCESS && !cur) {
+    // nothing has made the primary context current in this thread yet
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(c, e, what);
+    (void)ctx_current(&cur);
+  }
+  if (!cur) return fail(c, LI_ERR_CUDA, "%s: no current CUDA context", what);
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_addr[dev]) {
+  if (!g_static_addr[dev] || g_static_cuctx[dev] != cur) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess || !p) {
@@ -1150,6 +1166,7 @@ li_status static_scratch(li_ctx* c, void** out, const char* what) {
       return cuda_fail(c, e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress (static scratch)");
     }
     g_static_addr[dev] = p;
+    g_static_cuctx[dev] = cur;
   }
   *out = g_static_addr[dev];
   return LI_OK;
@@ -1200,7 +1217,7 @@ extern "C" li_status li_score_topk_static(li_ctx* c, const li_cache* cache, cons
   {
     int cs = 0;
     Launch Lc(c, st, "topk_cluster", 0, kClusterThreads, 0);
-    e = launch_topk_cluster(t, st, &cs);
+    e = launch_topk_cluster(t, st, &cs, topk_keys_per_thread(t.n, t.rows, c->num_sms));
     Lc.grid = cs * t.rows;
     Lc.done();
     if (e != cudaSuccess) return cuda_fail(c, e, "topk_cluster");

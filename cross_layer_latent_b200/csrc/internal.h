@@ -129,7 +129,6 @@ struct TopkArgs {
   int* chunk_off;             // [rows][n_chunks]
   uint2* cand;                // [rows][n]
   int n_chunks;
-  bool hist_ready;            // first-digit histogram already accumulated (fused)
   // bounded waits of the cluster kernel's exchanges: a wait that runs out
   // records LI_ERR_DEVICE_TIMEOUT in *status (may be null)
   int* status;
@@ -146,6 +145,10 @@ constexpr int kClusterMaxN = kClusterThreads * 32 * kClusterMaxSize;   // 131072
 // (kTopkKeysLatency for a few rows, kTopkKeysThroughput for many).
 constexpr int kTopkKeysLatency = 4, kTopkKeysThroughput = 32;
 int topk_cluster_size(int64_t n, int keys_per_thread, int rows);
+// The keys-per-thread target of a selection of `rows` rows of n positions:
+// latency-sized while its CTAs stay within about one wave of the GPU's SMs,
+// throughput-sized beyond.
+int topk_keys_per_thread(int64_t n, int rows, int num_sms);
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size,
                                 int keys_per_thread = kTopkKeysLatency);
 
@@ -154,7 +157,7 @@ constexpr int kTopkThreads = 256;
 constexpr int kMaxTopkChunks = 8192;
 
 // The four stages of a selection, launched in order on one stream:
-// 0 first-digit histogram (skipped when hist_ready), 1 filter (boundary
+// 0 first-digit histogram, 1 filter (boundary
 // bucket candidates and per-chunk counts), 2 select (exact threshold, tie
 // cut and output offsets, one CTA per row), 3 emit (ordered output).
 cudaError_t launch_topk_stage(int stage, const TopkArgs& a, cudaStream_t st);

@@ -273,11 +273,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     tmem_alloc(s.tmem_base, a.tmem_cols);
     tmem_relinquish();
   }
-  if (!GATHER && warp == 2 && lane == 0 && a.q_pos == nullptr) {
+  if (!GATHER && warp == kGatherWarp2 && lane == 0 && a.q_pos == nullptr) {
     // Until the lengths are visible the CTA cannot know its first items; it
     // guesses them from full-capacity segments (exact when every sequence
     // is full) and prefetches their rows and scales into L2, so that the
-    // first tile loads after the prologue hit L2 instead of HBM.
+    // first tile loads after the prologue hit L2 instead of HBM.  The warp
+    // that issues them has no other role in the scan and stays out of the
+    // prologue's barriers (issuing the prefetches takes about a microsecond).
     const int ips = (a.capacity + a.R - 1) / a.R;
     const int64_t total = static_cast<int64_t>(a.n_segments) * ips;
     const int64_t b0 = total * blockIdx.x / gridDim.x, b1 = total * (blockIdx.x + 1) / gridDim.x;
@@ -293,8 +295,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   // everything above touches only this CTA's own resources; the lengths,
   // queries and cache rows below may come from the previous kernel
   pdl_begin();
-  // Items per segment, then an exclusive prefix over segments.
-  for (int i = tid; i < a.n_segments; i += blockDim.x) {
+  // Items per segment, then an exclusive prefix over segments (the scan:
+  // every warp but the prefetching one; the gather: all of them).
+  constexpr int kPrologueThreads = GATHER ? kScanThreads : kScanThreads - 32;
+  const bool in_prologue = GATHER || warp != kGatherWarp2;
+  auto prologue_sync = [in_prologue] {
+    if constexpr (GATHER) {
+      __syncthreads();
+    } else {
+      if (in_prologue) named_bar_sync(1, kPrologueThreads);   // the prefetching warp does not take part
+    }
+  };
+  for (int i = tid; i < a.n_segments && tid < kPrologueThreads; i += kPrologueThreads) {
     s.prefix[i + 1] = segment_items<GATHER>(a, i);
     if (GATHER) {
       int n = a.cand_n[i];
@@ -303,7 +315,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       s.seg_len[i] = len < 0 ? 0 : (len > a.capacity ? a.capacity : len);
     }
   }
-  __syncthreads();
+  prologue_sync();
   if (warp == 0) {
     int carry = 0;
     for (int c = 0; c < a.n_segments; c += 32) {
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     if (lane == 0) s.prefix[0] = 0;
   }
   tc_fence_before();
-  __syncthreads();
+  prologue_sync();
   tc_fence_after();
 
   // Every scalar argument is copied into registers once: the argument block
@@ -744,10 +756,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              (acc.i * static_cast<uint32_t>(k_MB) + static_cast<uint32_t>(mb)) *
                                  static_cast<uint32_t>(k_N * k_nsc);
-      // segmented scales: head h's product is cs * D0_h + cs1 * D1_h; without
-      // a bias cs is factored out (cs > 0) and D0_h + (cs1 / cs) D1_h summed
-      float rho = 0.f;
-      if constexpr (SEG) rho = cs1 / cs;
+      // segmented scales: head h's product is cs * D0_h + cs1 * D1_h, formed
+      // per head before the ReLU (no division: a zero scale stays finite);
+      // with one scale per row it is taken outside the head sum instead
+      const bool scale_after = !has_beta && e4 && !SEG;
       // One score: the head sums of query row qi from its HP columns at vq,
       // in the same order as the per-query loop below (so results agree bit
       // for bit whichever path runs), then the store.
@@ -764,7 +776,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           else relu_dot16_beta(vq + h0, wq + h0, qs + h0, be + h0, cs, part);
         }
         float sc = (part[0] + part[1]) + (part[2] + part[3]);
-        if (!has_beta && e4) sc *= cs;
+        if (scale_after) sc *= cs;
         if (row_in_item && j < ep_len[qi]) {
           if (GATHER && tok < 0) {
             sc = -INFINITY;
@@ -812,7 +824,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
                                tbase + static_cast<uint32_t>(k_N + qi * k_H_pad + h0), v, v1);
             if (!has_beta) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = fmaf(rho, v1[e], v[e]);
+              for (int e = 0; e < 16; ++e) v[e] = fmaf(cs1, v1[e], cs * v[e]);
               relu_dot16(v, wq + h0, part);
             } else {
 #pragma unroll
@@ -840,7 +852,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         }
         if (qi == 0 && lane == 0 && (ew & 3) == 0) trace_event(k_trace, lt, 7);
         float sc = (part[0] + part[1]) + (part[2] + part[3]);
-        if (!has_beta && e4) sc *= cs;
+        if (scale_after) sc *= cs;
         if (row_in_item && j < ep_len[qi]) {
           if (GATHER && tok < 0) {
             sc = -INFINITY;

@@ -89,6 +89,9 @@ typedef struct li_ctx li_ctx;
  *         be a multiple of 16 bytes and `data` 16-byte aligned.
  * scale   [batch][capacity] fp32 per-token dequantisation scale (LI_E4M3
  *         only, NULL otherwise): element value = scale[b][s] * e4m3 code.
+ *         Every scale of a valid row must be finite and >= 0: the scan takes
+ *         it outside the ReLU (max(0, a x) = a max(0, x) only for a >= 0).
+ *         The library's own appends write amax / 448, or 1 for a zero row.
  * lengths [batch] int32 valid rows per sequence (read and advanced on the
  *         device by li_append_latent).
  * dim: multiple of 8 (F32), 16 (BF16) or 32 (E4M3), at most 256.  Scanning
@@ -117,7 +120,8 @@ typedef struct {
  *         must match the cache: F32 with F32 (tf32 tensor cores), BF16 with
  *         BF16, E4M3 with E4M3.  16-byte aligned.
  * q_scale [batch][T][H] fp32 per-(token, head) dequantisation scale of an
- *         E4M3 query; NULL otherwise.
+ *         E4M3 query; NULL otherwise.  Finite and >= 0 (without beta it is
+ *         folded into the head weight, outside the ReLU).
  * beta    [batch][T][H] fp32 decoder-bias term added before the ReLU, or NULL.
  * w       [batch][T][H] fp32 head weights.
  * T       query tokens per sequence (1 = decode).  H heads, 1..256.
@@ -157,7 +161,9 @@ LI_API li_status li_device_status(li_ctx* ctx, const void* ws, void* stream, li_
  * (default 2e9 = 2 s).  When a wait runs out the kernel records
  * LI_ERR_DEVICE_TIMEOUT, drains its own copies in flight, frees its tensor
  * memory and returns.  0 makes every wait that is not already satisfied
- * when it starts give up at once (a way to exercise that path). */
+ * when it starts give up at once (a way to exercise that path).  The
+ * outputs of a call whose wait ran out are undefined; read the status with
+ * li_device_status before the workspace's next use. */
 LI_API li_status li_set_wait_limit(li_ctx* ctx, uint64_t ns);
 
 /* ------------------------------------------------------------- a1: append */
@@ -343,6 +349,9 @@ LI_API li_status li_dsa_score_topk(li_ctx* ctx, const li_cache* key_cache, const
  * Setup: the first call on a device looks up the scratch's device address
  *   (once per device, with the context's device current; a failure returns
  *   LI_ERR_CUDA).  Make that first call before any stream capture begins.
+ *   The address belongs to the device's current CUDA context: when that
+ *   context changes (after cudaDeviceReset, say), the next call looks it up
+ *   again, and that call too must come before any capture.
  * Zeroing: the scratch starts zeroed when the library is loaded; the status
  *   word is cleared by every call itself; the scores need no clearing.
  * Status: device-detected errors (a bounded wait that ran out) are written to

@@ -10,7 +10,7 @@ import torch
 import cross_layer_latent_b200 as li
 from oracle import indexer
 from tests.gpu_setup import build_group
-from tests.helpers import RTOL, assert_scores_close
+from tests.helpers import RTOL, assert_scores_close, assert_selection_close
 from workloads import generate, workload
 
 pytestmark = pytest.mark.gpu
@@ -98,3 +98,52 @@ def test_full_size_hs_and_dsa(ctx, index):
         ref = indexer.dsa_score_keys(keys, inp.q[0][b, 0], inp.w[0][b, 0])
         M = indexer.error_scale(keys, inp.q[0][b, 0], inp.w[0][b, 0])
         assert_scores_close(d[b, 0, pos], ref, M, rtol, f"{wl.name} DSA seq {b}")
+
+
+def test_full_size_prefill_chunk(ctx):
+    """The whole prefill chunk: 1024 queries at positions 64512..65535 against
+    their causal prefixes of the 65536-row bf16 latent (H 32, d_c 256, k 2048;
+    each layer keeps its own top-k, up to 2048 per query: LatentIndex summary,
+    Sec. 3.1 and Sec. 4.1), through li_score_topk in the configuration the
+    benchmark times.  A seeded sample of 32 query rows (the first and the last
+    among them) in two layers is compared with the oracle element by element;
+    every selection of those rows is bit-exact against the oracle's top-k of
+    the dumped row and within the selection rule of the oracle's own scores.
+    The launch must take the many-rows selection (32 keys a thread)."""
+    wl = workload(4)
+    inp = generate(wl)
+    g = build_group(ctx, inp, dsa=False)
+    rtol = RTOL[wl.cache_dtype]
+    rng = np.random.default_rng(404)
+    rows = np.unique(np.concatenate([[0, wl.queries - 1], rng.choice(wl.queries, 30, replace=False)]))
+    dump = torch.full((1, wl.queries, wl.capacity), float("nan"), device=DEV)
+    c64 = inp.latent[0].astype(np.float64)
+    for l in range(2):
+        li.li_profile_enable(ctx, True)
+        li.li_profile_reset(ctx)
+        g.score_topk(l, dump=dump)
+        torch.cuda.synchronize()
+        recs = li.li_profile_read(ctx)
+        li.li_profile_enable(ctx, False)
+        li.li_profile_reset(ctx)
+        assert li.li_device_status(ctx, g.ws) == "LI_OK"
+        sel = [r for r in recs if r["kernel"].startswith("topk")]
+        assert len(sel) == 1 and sel[0]["kernel"] == "topk_cluster", [r["kernel"] for r in recs]
+        cs = sel[0]["grid"] // wl.queries
+        assert -(-wl.capacity // (cs * 512)) == 32, f"selection took {cs} CTAs a row, not 32 keys a thread"
+        d, idx, sc = _np(dump), _np(g.idx[l]), _np(g.score[l])
+        qt_all, _ = indexer.absorb(inp.q[l][0], inp.W_K[l])
+        for t in rows:
+            n = indexer.valid_length(inp.lengths[0], inp.q_pos[0, t])
+            assert n == int(inp.q_pos[0, t]) + 1
+            assert np.all(np.isnan(d[0, t, n:])), f"layer {l} query {t}: scores past its causal prefix"
+            ref = indexer.score(c64[:n], qt_all[t], inp.w[l][0, t])
+            M = indexer.error_scale(c64[:n], qt_all[t], inp.w[l][0, t])
+            assert_scores_close(d[0, t, :n], ref, M, rtol, f"prefill layer {l} query {t}")
+            e, ev = indexer.topk(d[0, t, :n], wl.k, n)
+            assert np.array_equal(idx[0, t], e), f"prefill layer {l} query {t}: selection"
+            keep = e >= 0
+            got = np.where(sc[0, t][keep] == 0, np.float32(0), sc[0, t][keep])
+            want = np.where(ev[keep] == 0, 0.0, ev[keep]).astype(np.float32)
+            assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+            assert_selection_close(idx[0, t], ref, M, wl.k, n, rtol, f"prefill layer {l} query {t}")

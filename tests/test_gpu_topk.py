@@ -1,4 +1,6 @@
 """li_topk on identical fp32 arrays must match the oracle's sort bit for bit."""
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -18,6 +20,11 @@ def ctx():
     c = li.Context(0)
     yield c
     c.close()
+
+
+def _seed(*parts):
+    """A seed that is the same in every process (str hashes are salted)."""
+    return zlib.crc32(repr(parts).encode())
 
 
 def _rows(kind, rows, n, rng):
@@ -68,7 +75,7 @@ def _check(ctx, x, k, lengths=None):
 @pytest.mark.parametrize("rows,n,k", [(1, 8192, 2048), (4, 131072, 2048), (3, 1000, 64), (5, 4097, 4097),
                                       (64, 5000, 100)])
 def test_topk_bit_exact(ctx, kind, rows, n, k):
-    rng = np.random.default_rng(hash((kind, rows, n, k)) % 2 ** 32)
+    rng = np.random.default_rng(_seed(kind, rows, n, k))
     _check(ctx, _rows(kind, rows, n, rng), k)
 
 
@@ -88,3 +95,48 @@ def test_topk_ragged_rows_in_the_widest_clusters(ctx, kind):
     x = _rows(kind, 4, 131072, rng)
     _check(ctx, x, 2048, np.array([70001, 131072, 3, 0]))
     _check(ctx, x, 2048, np.array([8191, 8192, 8193, 131071]))
+
+
+def _launched_keys_per_thread(ctx, fn, rows, n):
+    """Run fn with the launch profile on; the keys a thread of the one
+    cluster selection it launched holds (4, 8, 16 or 32)."""
+    li.li_profile_enable(ctx, True)
+    li.li_profile_reset(ctx)
+    fn()
+    torch.cuda.synchronize()
+    recs = li.li_profile_read(ctx)
+    li.li_profile_enable(ctx, False)
+    li.li_profile_reset(ctx)
+    sel = [r for r in recs if r["kernel"].startswith("topk")]
+    assert len(sel) == 1 and sel[0]["kernel"] == "topk_cluster", [r["kernel"] for r in recs]
+    cs = sel[0]["grid"] // rows
+    per = -(-n // (cs * 512))
+    return next(p for p in (4, 8, 16, 32) if per <= p)
+
+
+@pytest.mark.parametrize("kind", ["gauss", "ties", "zeros"])
+@pytest.mark.parametrize("rows,n", [(1024, 65536), (400, 20000)])
+def test_topk_many_rows_take_the_throughput_selection(ctx, kind, rows, n):
+    """Many rows (a prefill chunk's queries) fill the GPU many times over and
+    take the selection sized for throughput, 32 keys a thread; it must stay
+    bit-exact, with ragged valid prefixes (empty, ending inside a CTA, full)."""
+    rng = np.random.default_rng(_seed(kind, rows, n, 32))
+    x = _rows(kind, rows, n, rng)
+    lengths = rng.integers(0, n + 1, rows)
+    lengths[:4] = [0, 1, n, n - 1]
+    k = 2048
+    xd = torch.from_numpy(x).to(DEV)
+    ld = torch.from_numpy(lengths.astype(np.int32)).to(DEV)
+    idx = torch.full((rows, k), -7, dtype=torch.int32, device=DEV)
+    val = torch.zeros(rows, k, device=DEV)
+    ws = li.workspace(ctx, rows, 1, n, 1, k)
+    pt = _launched_keys_per_thread(ctx, lambda: li.li_topk(ctx, xd, k, idx, val, ws, lengths=ld), rows, n)
+    assert pt == 32, f"launched the {pt}-keys-a-thread selection"
+    gi, gv = idx.cpu().numpy(), val.cpu().numpy()
+    for r in range(rows):
+        ei, _ = indexer.topk(x[r], k, int(lengths[r]))
+        assert np.array_equal(gi[r], ei), f"row {r} (length {lengths[r]}): first difference at {np.argmax(gi[r] != ei)}"
+        keep = ei >= 0
+        want = np.where(x[r][ei[keep]] == 0, np.float32(0), x[r][ei[keep]])
+        got = np.where(gv[r][keep] == 0, np.float32(0), gv[r][keep])
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32))

@@ -16,6 +16,8 @@ DEV = "cuda:0"
 CASES = {
     "v32-bf16-n3000": lambda: shrunk(workload(1), capacity=3000, queries=1),
     "long-e4m3-n5000": lambda: shrunk(workload(3), capacity=5000, batch=2),
+    # 64 query rows of a prefill chunk: enough rows for the many-rows selection
+    "prefill-bf16-64x20000": lambda: shrunk(workload(4), capacity=20000, queries=64),
 }
 
 
@@ -31,7 +33,7 @@ def test_static_scratch_matches_workspace_entry_point(ctx, name):
     wl = CASES[name]()
     inp = generate(wl)
     g = build_group(ctx, inp, dsa=False)
-    rows = (wl.batch, 1, wl.k)
+    rows = (wl.batch, wl.queries, wl.k)
     ref_idx = torch.empty(rows, dtype=torch.int32, device=DEV)
     ref_score = torch.empty(rows, device=DEV)
     li.li_score_topk(ctx, g.latent, g.query(0), wl.k, ref_idx, ref_score, None, g.ws)
@@ -42,8 +44,9 @@ def test_static_scratch_matches_workspace_entry_point(ctx, name):
         status = torch.full((1,), -1, dtype=torch.int32, device=DEV)
         li.li_score_topk_static(ctx, g.latent, g.query(0), wl.k, idx, score, status)
         torch.cuda.synchronize()
+        # the same kernels on the same inputs: identical bits
         assert torch.equal(idx, ref_idx), f"{name}: call {call} selected different tokens"
-        torch.testing.assert_close(score, ref_score, rtol=2e-3, atol=0.0)
+        assert torch.equal(score.view(torch.int32), ref_score.view(torch.int32)), f"{name}: call {call} scores"
         assert int(status.item()) == 0, f"{name}: call {call} device status {int(status.item())}"
 
 
