@@ -554,15 +554,18 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   // 467 us, against 566 us for the chunked multi-kernel path).
   if (t.rows > 65535) return fail(ctx, LI_ERR_UNSUPPORTED, "more than 65535 selection rows");
   if (t.n <= kClusterMaxN) {
-    const int kpt = topk_keys_per_thread(t.n, t.rows, ctx->num_sms);
+    const int rows_all = t.rows * (t.k2 > 0 ? 2 : 1);   // a second budget doubles the clusters
+    const int kpt = topk_keys_per_thread(t.n, rows_all, ctx->num_sms);
     int cs = 0;
     Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);
     const cudaError_t e = launch_topk_cluster(t, st, &cs, kpt);
-    Lc.grid = cs * t.rows;
+    Lc.grid = cs * rows_all;
     Lc.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster");
     return LI_OK;
   }
+  if (t.k2 > 0) return fail(ctx, LI_ERR_UNSUPPORTED, "two budgets in one selection need rows of at most %d",
+                            kClusterMaxN);
   li_status s = clear_select_state(ctx, ws, L, t.rows, st);
   if (s != LI_OK) return s;
   return run_topk_chunked(ctx, t, ws, L, st);
@@ -874,7 +877,7 @@ li_status li_absorb_query(li_ctx* c, const void* q, li_dtype q_dtype, int n_tok,
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   Launch L(c, st, "absorb", 0, 256, 0);
   const cudaError_t e = launch_absorb(q, q_dtype, n_tok, H, d_k, W_K, W_K_head_stride, b_K, b_K_head_stride, d_c,
-                                      out_dtype, q_abs, q_abs_scale, beta, st);
+                                      out_dtype, q_abs, q_abs_scale, beta, c->num_sms, st);
   L.done();
   if (e != cudaSuccess) return cuda_fail(c, e, "absorb launch");
   return LI_OK;
@@ -923,6 +926,16 @@ li_status li_hs_anchor_candidates(li_ctx* c, const li_cache* cache, const li_que
   t.out_idx = cand;
   t.out_score = cand_scores;
   t.out_count = cand_n;
+  if (cache->capacity <= kClusterMaxN) {
+    // the anchor's own top-k is the top-k of the full prefix: it is selected
+    // from the same scores by clusters of their own in the same launch as
+    // the candidates, rather than after them from the candidates' scores
+    t.out_score = nullptr;
+    t.k2 = k;
+    t.out_idx2 = anchor_idx;
+    t.out_score2 = anchor_score;
+    return run_topk(c, t, ws, L, st);
+  }
   if ((s = run_topk(c, t, ws, L, st)) != LI_OK) return s;
   // the anchor's own top-k: under the same order (score desc, position asc)
   // the top-k of the prefix is the top-k of its top-B, whose positions are

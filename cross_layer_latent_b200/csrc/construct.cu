@@ -658,6 +658,88 @@ size_t absorb_shared_smem(int d_k, int d_c, int R, size_t elt) {
   return (static_cast<size_t>(d_k) * d_c * elt + 15) / 16 * 16 + static_cast<size_t>(R) * (d_k + d_c) * 4;
 }
 
+// Shared decoder at decode sizes, split by output columns, for fp32 and bf16
+// output: CTA (s, g) computes the columns [s kSplitCols, (s + 1) kSplitCols)
+// of the U * 4 rows (token, head) of row group g, from its slice of the
+// decoder (d_k x kSplitCols) staged in shared memory; thread t takes column
+// t % kSplitCols of rows t / kSplitCols + 4 u.  The slice is a weight, not
+// a result of the step, so it is requested before the kernel waits for the
+// previous one in the stream; only the query rows wait.  Each output
+// accumulates j = 0..d_k-1 in order with fp32 fma, as the other absorb
+// kernels do (identical results).
+constexpr int kSplitCols = 64;   // 4 rows x kSplitCols columns per pass of 256 threads
+
+template <typename T, int U>
+__global__ void __launch_bounds__(256) absorb_split_kernel(const T* __restrict__ q, int M, int d_k,
+                                                           const T* __restrict__ W, int d_c, int out_dtype,
+                                                           void* q_abs) {
+  constexpr int kRows = 4 * U;
+  const int r0 = blockIdx.y * kRows;
+  const int c0 = blockIdx.x * kSplitCols;
+  extern __shared__ __align__(16) unsigned char split_smem[];
+  T* Ws = reinterpret_cast<T*>(split_smem);                                        // [d_k][kSplitCols]
+  float* qs = reinterpret_cast<float*>(split_smem + static_cast<size_t>(d_k) * kSplitCols * sizeof(T));  // [kRows][d_k]
+  {
+    // the decoder slice, every 16-byte piece in flight at once
+    constexpr int kPieces = kSplitCols * static_cast<int>(sizeof(T)) / 16;   // per decoder row
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(Ws));
+    for (int x = threadIdx.x; x < d_k * kPieces; x += blockDim.x) {
+      const int j = x / kPieces, pc = x - j * kPieces;
+      cp_async_16(dst + 16u * x, reinterpret_cast<const uint4*>(W + static_cast<int64_t>(j) * d_c + c0) + pc);
+    }
+    cp_async_commit();
+  }
+  pdl_begin();
+  pdl_release();
+  for (int x = threadIdx.x; x < kRows * d_k; x += blockDim.x) {
+    const int rr = x / d_k;
+    qs[x] = r0 + rr < M ? to_f(q[static_cast<int64_t>(r0) * d_k + x]) : 0.f;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int rs = threadIdx.x / kSplitCols, cc = threadIdx.x - rs * kSplitCols;
+  const T* wc = Ws + cc;
+  float acc[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) acc[u] = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < d_k; ++j) {
+    const float w = to_f(wc[j * kSplitCols]);
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc[u] = fmaf(w, qs[(rs + 4 * u) * d_k + j], acc[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int row = r0 + rs + 4 * u;
+    if (row >= M) continue;
+    const int64_t o = static_cast<int64_t>(row) * d_c + c0 + cc;
+    if (out_dtype == LI_F32) reinterpret_cast<float*>(q_abs)[o] = acc[u];
+    else reinterpret_cast<__nv_bfloat16*>(q_abs)[o] = __float2bfloat16_rn(acc[u]);
+  }
+}
+
+template <typename T>
+cudaError_t launch_absorb_split(const T* q, int M, int d_k, const T* W, int d_c, int out_dtype, void* q_abs,
+                                int num_sms, cudaStream_t st) {
+  // rows a thread takes: enough CTAs to cover about the SMs once, no more
+  const int S = d_c / kSplitCols;
+  int U = 1;
+  while (U < 8 && static_cast<int64_t>((M + 8 * U - 1) / (8 * U)) * S >= num_sms) U *= 2;
+  const size_t smem = static_cast<size_t>(d_k) * kSplitCols * sizeof(T) + static_cast<size_t>(4 * U) * d_k * 4;
+  const dim3 grid(S, (M + 4 * U - 1) / (4 * U));
+  auto go = [&](auto kernel) -> cudaError_t {
+    const cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(kernel), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kernel, grid, dim3(256), smem, st, 1, q, M, d_k, W, d_c, out_dtype, q_abs);
+  };
+  switch (U) {
+    case 1: return go(absorb_split_kernel<T, 1>);
+    case 2: return go(absorb_split_kernel<T, 2>);
+    case 4: return go(absorb_split_kernel<T, 4>);
+    default: return go(absorb_split_kernel<T, 8>);
+  }
+}
+
 }  // namespace
 
 int gemv_splits(int d_model, int n_tok) {
@@ -793,7 +875,8 @@ cudaError_t launch_absorb_group(const void* q, int q_dtype, int batch, int G, in
 
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
-                          int out_dtype, void* q_abs, float* q_abs_scale, float* beta, cudaStream_t st) {
+                          int out_dtype, void* q_abs, float* q_abs_scale, float* beta, int num_sms,
+                          cudaStream_t st) {
   const size_t elt = q_dtype == LI_BF16 ? 2 : 4;
   const int M = n_tok * H;
   // shared decoder: rows of R (token, head) pairs; two rows per block at
@@ -802,6 +885,17 @@ cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k,
   const int R = M <= 4096 ? 2 : 32;
   const size_t smem = absorb_shared_smem(d_k, d_c, R, elt);
   const bool aligned = (reinterpret_cast<uintptr_t>(W) & 15) == 0 && (static_cast<size_t>(d_k) * d_c * elt) % 16 == 0;
+  if (W != nullptr && W_head_stride == 0 && b == nullptr && beta == nullptr && M <= 4096 && aligned &&
+      d_c % kSplitCols == 0 && out_dtype != LI_E4M3) {
+    // decode, fp32 or bf16 output: the column-split kernel (its decoder
+    // slices stage before the wait).  E4M3 output needs each row's amax over
+    // all columns and stays with the whole-row kernel below.
+    if (q_dtype == LI_BF16)
+      return launch_absorb_split(reinterpret_cast<const __nv_bfloat16*>(q), M, d_k,
+                                 reinterpret_cast<const __nv_bfloat16*>(W), d_c, out_dtype, q_abs, num_sms, st);
+    return launch_absorb_split(reinterpret_cast<const float*>(q), M, d_k, reinterpret_cast<const float*>(W), d_c,
+                               out_dtype, q_abs, num_sms, st);
+  }
   if (W != nullptr && W_head_stride == 0 && b_head_stride == 0 && (d_c & 1) == 0 && aligned &&
       smem <= 200 * 1024) {
     AbsorbLayers L{};

@@ -122,6 +122,13 @@ struct TopkArgs {
   int32_t* out_idx;
   float* out_score;
   int32_t* out_count;         // k_eff per row, or null
+  // A second budget over the same rows in the same launch (cluster kernel
+  // only): with k2 > 0 the grid holds 2 x rows rows of clusters, and row
+  // rows + r selects the top-k2 of score row r into out_idx2 / out_score2
+  // (same lengths and index map, no count), independently of row r.
+  int k2;
+  int32_t* out_idx2;
+  float* out_score2;
   // workspace
   unsigned int* hist;         // [rows][2048]
   int* rowinfo;               // [rows][16]
@@ -200,7 +207,7 @@ cudaError_t launch_absorb_group(const void* q, int q_dtype, int batch, int G, in
                                 int d_c, int out_dtype, void* q_abs, float* q_abs_scale, cudaStream_t st);
 cudaError_t launch_absorb(const void* q, int q_dtype, int n_tok, int H, int d_k, const void* W,
                           int64_t W_head_stride, const float* b, int64_t b_head_stride, int d_c,
-                          int out_dtype, void* q_abs, float* q_abs_scale, float* beta,
+                          int out_dtype, void* q_abs, float* q_abs_scale, float* beta, int num_sms,
                           cudaStream_t st);
 
 // ---- selection quality

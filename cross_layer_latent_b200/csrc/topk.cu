@@ -525,18 +525,22 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = CL ? static_cast<int>(cluster.num_blocks()) : 1;
   const int c = CL ? static_cast<int>(cluster.block_rank()) : 0;
-  const int r = blockIdx.y;
+  // rows past a.rows select the second budget of the same score rows
+  const bool second = a.k2 > 0 && static_cast<int>(blockIdx.y) >= a.rows;
+  const int r = second ? static_cast<int>(blockIdx.y) - a.rows : static_cast<int>(blockIdx.y);
+  const int kk = second ? a.k2 : a.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = row_len(a, r);
-  const int keff = min(a.k, n);
-  int32_t* oi = a.out_idx + static_cast<int64_t>(r) * a.k;
-  float* osv = a.out_score ? a.out_score + static_cast<int64_t>(r) * a.k : nullptr;
+  const int keff = min(kk, n);
+  int32_t* oi = (second ? a.out_idx2 : a.out_idx) + static_cast<int64_t>(r) * kk;
+  float* const os_base = second ? a.out_score2 : a.out_score;
+  float* osv = os_base ? os_base + static_cast<int64_t>(r) * kk : nullptr;
   if (c == 0) {
-    for (int j = max(keff, 0) + threadIdx.x; j < a.k; j += blockDim.x) {
+    for (int j = max(keff, 0) + threadIdx.x; j < kk; j += blockDim.x) {
       oi[j] = -1;
       if (osv) osv[j] = -INFINITY;
     }
-    if (a.out_count && threadIdx.x == 0) a.out_count[r] = max(keff, 0);
+    if (!second && a.out_count && threadIdx.x == 0) a.out_count[r] = max(keff, 0);
   }
   if (keff <= 0) return;   // the same for every CTA of the row
 
@@ -685,7 +689,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
       const bool eq = v && key[i] == T;
       if (gt || (eq && q < need_eq)) {
         const int rank = g + min(q, need_eq);
-        if (rank < a.k) {
+        if (rank < kk) {
           const int64_t pos = first + i;
           oi[rank] = map ? map[pos] : static_cast<int32_t>(pos);
           if (osv) osv[rank] = radix_value(key[i]);   // no reload: the key is the score
@@ -704,18 +708,19 @@ __global__ void __launch_bounds__(kClusterThreads, 1) topk_radix_kernel(const To
 
 template <int PT>
 cudaError_t launch_radix_pt(const TopkArgs& a, int cs, cudaStream_t st) {
-  if (cs == 1) return launch_pdl(topk_radix_kernel<PT, false>, dim3(1, a.rows, 1), dim3(kClusterThreads), 0, st, 1, a);
+  const unsigned rows = static_cast<unsigned>(a.rows) * (a.k2 > 0 ? 2u : 1u);
+  if (cs == 1) return launch_pdl(topk_radix_kernel<PT, false>, dim3(1, rows, 1), dim3(kClusterThreads), 0, st, 1, a);
   if constexpr (PT == 16) {
     if (cs > 8) {
       // a 16-CTA cluster is non-portable: allowed once per process
       static cudaError_t allowed = cudaFuncSetAttribute(topk_radix_kernel<16, true, 16>,
                                                          cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (allowed != cudaSuccess) return allowed;
-      return launch_pdl(topk_radix_kernel<16, true, 16>, dim3(cs, a.rows, 1), dim3(kClusterThreads), 0, st, cs, a);
+      return launch_pdl(topk_radix_kernel<16, true, 16>, dim3(cs, rows, 1), dim3(kClusterThreads), 0, st, cs, a);
     }
   }
   if (cs > kClusterMaxSize) return cudaErrorInvalidValue;   // only 16 keys a thread comes in clusters past 8
-  return launch_pdl(topk_radix_kernel<PT, true>, dim3(cs, a.rows, 1), dim3(kClusterThreads), 0, st, cs, a);
+  return launch_pdl(topk_radix_kernel<PT, true>, dim3(cs, rows, 1), dim3(kClusterThreads), 0, st, cs, a);
 }
 
 }  // namespace
@@ -749,7 +754,7 @@ int topk_keys_per_thread(int64_t n, int rows, int num_sms) {
 
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size, int keys_per_thread) {
   const int64_t n = a.n;
-  const int cs = topk_cluster_size(n, keys_per_thread, a.rows);
+  const int cs = topk_cluster_size(n, keys_per_thread, a.rows * (a.k2 > 0 ? 2 : 1));
   const int64_t per_thread = (n + static_cast<int64_t>(cs) * kClusterThreads - 1) / (static_cast<int64_t>(cs) * kClusterThreads);
   if (cluster_size) *cluster_size = cs;
   if (per_thread <= 4) return launch_radix_pt<4>(a, cs, st);

@@ -154,9 +154,11 @@ CASES = {
     "v32-bf16-n3000": lambda: shrunk(workload(1), capacity=3000, queries=1),
     "ragged-bf16": lambda: shrunk(workload(2), capacity=2500, batch=3, length_range=(700, 2500)),
     "long-e4m3-n5000": lambda: shrunk(workload(3), capacity=5000, batch=2),
-    # past 65536 positions the anchor selects its candidates and its own top-k
-    # in two launches (the second from the candidates' scores)
     "long-e4m3-n70k": lambda: shrunk(workload(3), capacity=70000, batch=2, length_range=(66000, 70000)),
+    # past 131072 positions the selections take the chunked multi-kernel path,
+    # and the anchor selects its candidates and then its own top-k from the
+    # candidates' scores in a second selection
+    "long-e4m3-n140k": lambda: shrunk(workload(3), capacity=140000, batch=1),
 }
 
 
