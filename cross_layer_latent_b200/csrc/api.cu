@@ -319,13 +319,18 @@ li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, boo
   const int64_t row_bytes = static_cast<int64_t>(c->dim) * eb;
   int swz = row_bytes % 128 == 0 ? 128 : (row_bytes % 64 == 0 ? 64 : 32);
   int n_kchunks = static_cast<int>(row_bytes / swz);
+  bool tail64 = false;
   if (gather && swz < 128 && row_bytes > 128) {
     // Row gathers are bound by the number of TMA operations, so gather whole
     // 128-byte chunks: K is padded to a multiple of 128 bytes, and the bytes
     // past the row's end lie outside both tensor maps and arrive as zeros
     // (cache and queries alike), which adds exact zeros to every product.
+    // A row of 128 m + 64 bytes (the e4m3 latent: 192) gathers its last 64
+    // bytes by a second map with a 64-byte box, into a 64-byte-swizzled tile:
+    // as many operations, and no bytes read past the row.
     swz = 128;
     n_kchunks = static_cast<int>((row_bytes + 127) / 128);
+    tail64 = row_bytes % 128 == 64;
   }
   // segmented fp8: two scales per row and two accumulators per item, so at
   // most 128 MMA columns per accumulator
@@ -439,6 +444,12 @@ li_status plan_scan_build(li_ctx* ctx, const li_cache* c, const li_query* q, boo
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(swz / eb), 1};
     li_status s = encode_map(ctx, &a.map_a, c->dtype, 2, c->data, dims, strides, box, swz, false);
     if (s != LI_OK) return s;
+    if (tail64) {
+      const cuuint32_t box2[2] = {static_cast<cuuint32_t>(64 / eb), 1};
+      s = encode_map(ctx, &a.map_a2, c->dtype, 2, c->data, dims, strides, box2, 64, false);
+      if (s != LI_OK) return s;
+      a.tail64 = 1;
+    }
   } else {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(swz / eb), static_cast<cuuint64_t>(c->batch) * c->capacity,
                                 static_cast<cuuint64_t>(a.n_kchunks)};

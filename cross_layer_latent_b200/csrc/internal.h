@@ -29,6 +29,7 @@ struct alignas(64) ScanArgs {
   CUtensorMap map_a;          // cache rows: dims {swz/elt, batch*capacity, n_kchunks}, box {swz/elt, R, KS};
                               // gather: dims {dim, batch*capacity}, box {swz/elt, 1}
   CUtensorMap map_b;          // queries: dims {dim, H, batch*T}, box {swz/elt, H_pad, Qg}
+  CUtensorMap map_a2;         // gather with tail64: dims {dim, batch*capacity}, box {64 B / elt, 1}, 64-B swizzle
   const uint8_t* cache_data;  // [batch*capacity][row_bytes] (the rows the cache map covers)
   const float* cache_scale;   // [batch*capacity] (segmented: [batch*capacity][2]) or null
   const int* lengths;         // [batch]
@@ -48,6 +49,7 @@ struct alignas(64) ScanArgs {
   int swz, n_kchunks, elt_bytes;
   int R, MB;                  // rows per work item (128 or 256) and M=128 blocks per item
   int RI;                     // gather: candidate rows gathered per item (32, 64 or 128 <= R)
+  int tail64;                 // gather: rows of 128 m + 64 bytes; the last 64-byte chunk comes by map_a2
   int KS, stages_per_item;    // K-chunks per stage, stages per item
   int n_stages, n_bslots, n_acc, n_meta;
   int ep_stride;              // floats of epilogue parameters per epilogue warp

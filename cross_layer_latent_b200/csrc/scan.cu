@@ -193,14 +193,14 @@ __device__ __forceinline__ void relu_dot16_beta(const float* v, const float* w, 
 // issuing thread is a single dependency chain, so loop control and address
 // arithmetic per MMA would otherwise cost as much as the MMA itself.
 template <int KIND, int KSTEPS, int MB>
-__device__ __forceinline__ void issue_chunk(uint32_t d0, uint32_t a_c, uint32_t b_c, uint64_t desc_hi,
+__device__ __forceinline__ void issue_chunk(uint32_t d0, uint32_t a_c, uint32_t b_c, uint64_t adesc_hi, uint64_t desc_hi,
                                             uint32_t m_stride, uint32_t n_cols, uint32_t idesc, bool first_chunk) {
 #pragma unroll
   for (int ks = 0; ks < KSTEPS; ++ks) {
     const uint64_t bdesc = desc_hi | ((b_c + ks * 32u) >> 4);
 #pragma unroll
     for (int mb = 0; mb < MB; ++mb) {
-      const uint64_t adesc = desc_hi | ((a_c + mb * m_stride + ks * 32u) >> 4);
+      const uint64_t adesc = adesc_hi | ((a_c + mb * m_stride + ks * 32u) >> 4);
       umma<KIND>(d0 + mb * n_cols, adesc, bdesc, idesc, (first_chunk && ks == 0) ? 0u : 1u);
     }
   }
@@ -208,17 +208,18 @@ __device__ __forceinline__ void issue_chunk(uint32_t d0, uint32_t a_c, uint32_t 
 
 template <int KIND>
 __device__ __forceinline__ void issue_chunk_rt(int ksteps, int mbs, uint32_t d0, uint32_t a_c, uint32_t b_c,
-                                               uint64_t desc_hi, uint32_t m_stride, uint32_t n_cols, uint32_t idesc,
+                                               uint64_t adesc_hi, uint64_t desc_hi, uint32_t m_stride,
+                                               uint32_t n_cols, uint32_t idesc,
                                                bool first_chunk) {
   switch (ksteps * 4 + mbs) {
-    case 1 * 4 + 1: issue_chunk<KIND, 1, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
-    case 1 * 4 + 2: issue_chunk<KIND, 1, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
-    case 2 * 4 + 1: issue_chunk<KIND, 2, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
-    case 2 * 4 + 2: issue_chunk<KIND, 2, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
-    case 3 * 4 + 1: issue_chunk<KIND, 3, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
-    case 3 * 4 + 2: issue_chunk<KIND, 3, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
-    case 4 * 4 + 1: issue_chunk<KIND, 4, 1>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
-    default: issue_chunk<KIND, 4, 2>(d0, a_c, b_c, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 1 * 4 + 1: issue_chunk<KIND, 1, 1>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 1 * 4 + 2: issue_chunk<KIND, 1, 2>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 2 * 4 + 1: issue_chunk<KIND, 2, 1>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 2 * 4 + 2: issue_chunk<KIND, 2, 2>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 3 * 4 + 1: issue_chunk<KIND, 3, 1>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 3 * 4 + 2: issue_chunk<KIND, 3, 2>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    case 4 * 4 + 1: issue_chunk<KIND, 4, 1>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
+    default: issue_chunk<KIND, 4, 2>(d0, a_c, b_c, adesc_hi, desc_hi, m_stride, n_cols, idesc, first_chunk); break;
   }
 }
 
@@ -268,6 +269,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     fence_barrier_init();
     tma_prefetch_desc(&a.map_a);
     tma_prefetch_desc(&a.map_b);
+    if (GATHER && a.tail64) tma_prefetch_desc(&a.map_a2);
   }
   if (warp == 1) {
     tmem_alloc(s.tmem_base, a.tmem_cols);
@@ -343,6 +345,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
   const int k_cand_stride = a.cand_stride, k_swz = a.swz, k_n_kchunks = a.n_kchunks;
   const int k_R = a.R, k_MB = a.MB, k_KS = a.KS, k_spi = a.stages_per_item;
   const int k_RI = GATHER ? a.RI : a.R;      // rows an item covers (gather: fewer than the M block)
+  const bool k_tail64 = GATHER && a.tail64;   // gathered rows end in a 64-byte chunk (map_a2)
   const uint32_t k_a_stage_bytes = a.a_stage_bytes, k_b_slot_bytes = a.b_slot_bytes, k_idesc = a.idesc;
   const uint32_t k_meta_bytes = a.meta_bytes;
   const int64_t k_score_stride = a.score_stride;
@@ -455,7 +458,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
     uint32_t n_st = 0, n_bs = 0;
     const int rows_per_lane = k_R >> 5;
     const int groups = k_RI >> 2;                  // 4-row gathers per K-chunk
-    const uint32_t stage_tx = static_cast<uint32_t>(k_RI * k_swz * k_KS);   // bytes gathered per stage
+    // bytes gathered per stage (the stage holding a 64-byte last chunk: 64 B less a row)
+    const uint32_t stage_tx_full = static_cast<uint32_t>(k_RI * k_swz * k_KS);
+    const uint32_t stage_tx_last = stage_tx_full - (k_tail64 ? static_cast<uint32_t>(k_RI * 64) : 0u);
     Ring st, bs, ms;
     SegWalk w{s.prefix, n_groups};
     SegWalk wn{s.prefix, n_groups};                // one item ahead
@@ -524,7 +529,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       for (int sp = 0; sp < k_spi; ++sp) {
         if (!bounded_wait(&s.empty[st.i], st.ph ^ 1u, wc)) { ok = false; break; }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&s.full[st.i], stage_tx);   // both warps' copies land on it
+          // both warps' copies land on it
+          mbar_arrive_expect_tx(&s.full[st.i], sp == k_spi - 1 ? stage_tx_last : stage_tx_full);
           mbar_arrive(&s.ready[st.i]);
         }
         __syncwarp();
@@ -534,9 +540,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         for (int u = lane; u < (groups * k_KS + 1) / 2; u += 32) {
           const int c = u / groups, r0 = 4 * (u - c * groups);
           const int t0 = mtok[r0], t1 = mtok[r0 + 1], t2 = mtok[r0 + 2], t3 = mtok[r0 + 3];
-          tma_gather4(stage + static_cast<uint32_t>(c) * chunk_region + static_cast<uint32_t>(r0 * k_swz), &a.map_a,
-                      &s.full[st.i], (sp * k_KS + c) * elt_per_chunk, seq_row + (t0 >= 0 ? t0 : 0),
-                      seq_row + (t1 >= 0 ? t1 : 0), seq_row + (t2 >= 0 ? t2 : 0), seq_row + (t3 >= 0 ? t3 : 0));
+          const bool tail = k_tail64 && sp * k_KS + c == k_n_kchunks - 1;
+          tma_gather4(stage + static_cast<uint32_t>(c) * chunk_region + static_cast<uint32_t>(r0 * (tail ? 64 : k_swz)),
+                      tail ? &a.map_a2 : &a.map_a, &s.full[st.i], (sp * k_KS + c) * elt_per_chunk,
+                      seq_row + (t0 >= 0 ? t0 : 0), seq_row + (t1 >= 0 ? t1 : 0), seq_row + (t2 >= 0 ? t2 : 0),
+                      seq_row + (t3 >= 0 ? t3 : 0));
         }
         st.step(S);
         ++n_st;
@@ -574,9 +582,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
           for (int u = half + lane; u < nops; u += 32) {
             const int c = u / groups, r0 = 4 * (u - c * groups);
             const int t0 = mtok[r0], t1 = mtok[r0 + 1], t2 = mtok[r0 + 2], t3 = mtok[r0 + 3];
-            tma_gather4(stage + static_cast<uint32_t>(c) * chunk_region + static_cast<uint32_t>(r0 * k_swz),
-                        &a.map_a, &s.full[st.i], (sp * k_KS + c) * elt_per_chunk, seq_row + (t0 >= 0 ? t0 : 0),
-                        seq_row + (t1 >= 0 ? t1 : 0), seq_row + (t2 >= 0 ? t2 : 0), seq_row + (t3 >= 0 ? t3 : 0));
+            const bool tail = k_tail64 && sp * k_KS + c == k_n_kchunks - 1;
+            tma_gather4(stage + static_cast<uint32_t>(c) * chunk_region + static_cast<uint32_t>(r0 * (tail ? 64 : k_swz)),
+                        tail ? &a.map_a2 : &a.map_a, &s.full[st.i], (sp * k_KS + c) * elt_per_chunk,
+                        seq_row + (t0 >= 0 ? t0 : 0), seq_row + (t1 >= 0 ? t1 : 0), seq_row + (t2 >= 0 ? t2 : 0),
+                        seq_row + (t3 >= 0 ? t3 : 0));
           }
           st.step(S);
         }
@@ -600,6 +610,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
       // K-major swizzled descriptors: everything but the start address is
       // fixed, so only the address field is added per MMA.
       const uint64_t desc_hi = make_smem_desc(0, static_cast<uint32_t>(k_swz));
+      // a gathered row's 64-byte last chunk sits in a 64-byte-swizzled tile
+      const uint64_t desc_hi64 = make_smem_desc(0, 64u);
       const uint32_t m_off = static_cast<uint32_t>(mi * 128 * k_swz);   // this M block within a chunk
       const uint32_t ksteps = static_cast<uint32_t>(k_swz >> 5);
       for (int item = begin; item < end; ++item, ++lt) {
@@ -630,20 +642,23 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
             const int kc = sp * k_KS + c;
             const uint32_t a_c = a_base + static_cast<uint32_t>(c) * chunk_region;
             const uint32_t b_c = b_base + static_cast<uint32_t>(kc * k_N * k_swz);
+            const bool tail = k_tail64 && kc == k_n_kchunks - 1;
+            const int kst = tail ? 2 : static_cast<int>(ksteps);
+            const uint64_t adh = tail ? desc_hi64 : desc_hi;
             if constexpr (!SEG) {
-              issue_chunk_rt<KIND>(static_cast<int>(ksteps), 1, d0, a_c, b_c, desc_hi, 0u,
-                                   static_cast<uint32_t>(k_N), k_idesc, kc == 0);
+              issue_chunk_rt<KIND>(kst, 1, d0, a_c, b_c, adh, desc_hi, 0u, static_cast<uint32_t>(k_N), k_idesc, kc == 0);
             } else {
               // segmented scales: K steps before k_SK accumulate into the
               // first accumulator, the rest into the second (N columns on)
               const int g0 = kc * static_cast<int>(ksteps);
-              const int n0 = max(0, min(static_cast<int>(ksteps), k_SK - g0));
+              const int n0 = max(0, min(kst, k_SK - g0));
               if (n0 > 0)
-                issue_chunk_rt<KIND>(n0, 1, d0, a_c, b_c, desc_hi, 0u, static_cast<uint32_t>(k_N), k_idesc, kc == 0);
-              if (n0 < static_cast<int>(ksteps))
-                issue_chunk_rt<KIND>(static_cast<int>(ksteps) - n0, 1, d0 + static_cast<uint32_t>(k_N),
+                issue_chunk_rt<KIND>(n0, 1, d0, a_c, b_c, adh, desc_hi, 0u, static_cast<uint32_t>(k_N), k_idesc,
+                                     kc == 0);
+              if (n0 < kst)
+                issue_chunk_rt<KIND>(kst - n0, 1, d0 + static_cast<uint32_t>(k_N),
                                      a_c + static_cast<uint32_t>(n0) * 32u, b_c + static_cast<uint32_t>(n0) * 32u,
-                                     desc_hi, 0u, static_cast<uint32_t>(k_N), k_idesc, g0 + n0 == k_SK);
+                                     adh, desc_hi, 0u, static_cast<uint32_t>(k_N), k_idesc, g0 + n0 == k_SK);
             }
           }
           umma_commit(&s.empty[st.i]);
