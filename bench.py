@@ -393,6 +393,14 @@ class Step:
         self.W_K = [torch.from_numpy(x).to(dev, bf) for x in inp.W_K]
         self.hs_keys, self.dsa_keys = keys_per_step(wl, inp.lengths)
         self.graphs = None
+        # The HS path's query absorptions read only the step's queries and
+        # decoders: they run on a second stream, forked from the step's
+        # stream, beside the anchor's append.  A scan waits there only where
+        # its query may not be ready yet (a kernel with a second dependency
+        # loses its overlap with the kernel before it on its own stream).
+        # The DSA-style path's raw-query conversions are short and stay in
+        # line: moved aside the same way, they gained nothing.
+        self.side = torch.cuda.Stream(dev)
 
     def bind(self, k):
         """Point the step's calls at device input/output set k (0 or 1);
@@ -435,13 +443,32 @@ class Step:
         for kc in self.g.keys:
             kc.lengths.copy_(self.len_before)
 
+    def _queries_aside(self, convert):
+        """Run convert(l) for every layer on the side stream, forked from the
+        current stream; returns one event per layer, recorded when its
+        query is ready."""
+        fork = torch.cuda.Event()
+        fork.record()
+        self.side.wait_event(fork)
+        ready = []
+        with torch.cuda.stream(self.side):
+            for l in range(self.wl.group):
+                convert(l)
+                e = torch.cuda.Event()
+                e.record()
+                ready.append(e)
+        return ready
+
     def hs_path(self):
         li, g, wl = self.li, self.g, self.wl
         g.idx = self.hs_idx
+        ready = self._queries_aside(lambda l: li.li_absorb_query(
+            self.ctx, self.q[l], self.W_K[l], wl.d_c, g.dtype, g.q_abs[l], g.q_abs_scale[l]))
         g.append(self.h_anchor, self.W_down)
-        for l in range(wl.group):
-            li.li_absorb_query(self.ctx, self.q[l], self.W_K[l], wl.d_c, g.dtype, g.q_abs[l], g.q_abs_scale[l])
+        cur = torch.cuda.current_stream()
+        cur.wait_event(ready[0])
         g.hs_anchor(0)
+        cur.wait_event(ready[-1])          # every follower's query (in order on the side stream)
         for l in range(1, wl.group):
             g.hs_follower(l)
 
