@@ -88,6 +88,8 @@ struct li_ctx {
   int device = 0;
   int num_sms = 0;
   int max_smem_optin = 0;
+  // resident clusters of the single-launch selection, by cluster size 1..16
+  int cluster_cap[17] = {};
   EncodeTiledFn encode = nullptr;
   std::string last_error;
   uint64_t wait_ns = 2000000000ull;
@@ -560,13 +562,13 @@ li_status run_topk(li_ctx* ctx, TopkArgs& t, void* ws, const WsLayout& L, cudaSt
   if (static_cast<int64_t>(t.rows) * t.n > static_cast<int64_t>((L.scores - L.cand) / 8))
     return fail(ctx, LI_ERR_WORKSPACE, "selection of %d x %d exceeds the workspace candidate buffer", t.rows, t.n);
   // Rows of up to kClusterMaxN positions take the single-launch cluster
-  // kernel: sized for latency while its CTAs (rows x cluster size) stay
-  // within about one wave, for throughput beyond (measured on 1024 x 65536:
-  // 467 us, against 566 us for the chunked multi-kernel path).
+  // kernel: sized for latency while every row's cluster can be resident at
+  // once, for throughput beyond (measured on 1024 x 65536: 467 us, against
+  // 566 us for the chunked multi-kernel path).
   if (t.rows > 65535) return fail(ctx, LI_ERR_UNSUPPORTED, "more than 65535 selection rows");
   if (t.n <= kClusterMaxN) {
     const int rows_all = t.rows * (t.k2 > 0 ? 2 : 1);   // a second budget doubles the clusters
-    const int kpt = topk_keys_per_thread(t.n, rows_all, ctx->num_sms);
+    const int kpt = topk_keys_per_thread(t.n, rows_all, ctx->cluster_cap);
     int cs = 0;
     Launch Lc(ctx, st, "topk_cluster", 0, kClusterThreads, 0);
     const cudaError_t e = launch_topk_cluster(t, st, &cs, kpt);
@@ -667,6 +669,22 @@ li_status li_create(li_ctx** out, int device) {
     return LI_ERR_UNSUPPORTED;
   }
   c->device = device;
+  {
+    // the occupancy queries read the current device: select ours for them
+    int prev = 0;
+    e = cudaGetDevice(&prev);
+    if (e == cudaSuccess) e = cudaSetDevice(device);
+    for (int cs = 1; cs <= 16 && e == cudaSuccess; ++cs) {
+      c->cluster_cap[cs] = topk_cluster_capacity(cs, c->num_sms);
+      if (c->cluster_cap[cs] < 0) e = cudaErrorInvalidValue;
+    }
+    const cudaError_t e2 = cudaSetDevice(prev);
+    if (e == cudaSuccess) e = e2;
+    if (e != cudaSuccess) {
+      delete c;
+      return LI_ERR_CUDA;
+    }
+  }
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
   e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
@@ -1241,7 +1259,7 @@ extern "C" li_status li_score_topk_static(li_ctx* c, const li_cache* cache, cons
   {
     int cs = 0;
     Launch Lc(c, st, "topk_cluster", 0, kClusterThreads, 0);
-    e = launch_topk_cluster(t, st, &cs, topk_keys_per_thread(t.n, t.rows, c->num_sms));
+    e = launch_topk_cluster(t, st, &cs, topk_keys_per_thread(t.n, t.rows, c->cluster_cap));
     Lc.grid = cs * t.rows;
     Lc.done();
     if (e != cudaSuccess) return cuda_fail(c, e, "topk_cluster");

@@ -154,10 +154,15 @@ constexpr int kClusterMaxN = kClusterThreads * 32 * kClusterMaxSize;   // 131072
 // (kTopkKeysLatency for a few rows, kTopkKeysThroughput for many).
 constexpr int kTopkKeysLatency = 4, kTopkKeysThroughput = 32;
 int topk_cluster_size(int64_t n, int keys_per_thread, int rows);
+// How many clusters of cs CTAs (1..16) of the single-launch selection can be
+// resident at once on the current device; -1 if the query fails.
+int topk_cluster_capacity(int cs, int num_sms);
 // The keys-per-thread target of a selection of `rows` rows of n positions:
-// latency-sized while its CTAs stay within about one wave of the GPU's SMs,
-// throughput-sized beyond.
-int topk_keys_per_thread(int64_t n, int rows, int num_sms);
+// the latency target (4 keys a thread) when every row's cluster can be
+// resident at once, else 8 or 16 keys a thread (smaller clusters) when
+// those fit, else the throughput target.  cap[cs] is the residency for
+// cluster size cs (1..16), from topk_cluster_capacity.
+int topk_keys_per_thread(int64_t n, int rows, const int* cap);
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size,
                                 int keys_per_thread = kTopkKeysLatency);
 

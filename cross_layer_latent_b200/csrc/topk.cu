@@ -745,11 +745,50 @@ int topk_cluster_size(int64_t n, int keys_per_thread, int rows) {
   return static_cast<int>(cs < 1 ? 1 : (cs > kClusterMaxSize ? kClusterMaxSize : cs));
 }
 
-int topk_keys_per_thread(int64_t n, int rows, int num_sms) {
-  // measured on 1024 x 65536: 467 us at 32 keys a thread against 788 us at 4
-  const int64_t cs_lat = topk_cluster_size(n, kTopkKeysLatency, rows);
-  return static_cast<int64_t>(rows) * cs_lat <= 2 * static_cast<int64_t>(num_sms) ? kTopkKeysLatency
-                                                                                  : kTopkKeysThroughput;
+int topk_cluster_capacity(int cs, int num_sms) {
+  if (cs < 1 || cs > 16) return -1;
+  cudaError_t e;
+  if (cs == 1) {
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_radix_kernel<4, false>, kClusterThreads, 0);
+    return e == cudaSuccess ? per_sm * num_sms : -1;
+  }
+  // every instantiation of the clustered kernel is resident one CTA an SM
+  // (512 threads above 64 registers each), so one stands for all
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(cs), 1, 1);
+  cfg.blockDim = dim3(kClusterThreads, 1, 1);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cs > kClusterMaxSize) {
+    e = cudaFuncSetAttribute(topk_radix_kernel<16, true, 16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, topk_radix_kernel<16, true, 16>, &cfg);
+  } else {
+    e = cudaOccupancyMaxActiveClusters(&n, topk_radix_kernel<4, true>, &cfg);
+  }
+  return e == cudaSuccess ? n : -1;
+}
+
+int topk_keys_per_thread(int64_t n, int rows, const int* cap) {
+  // A few rows are latency-bound: more CTAs a row shorten every pass, as
+  // long as all the rows' clusters run in one wave (a second wave costs a
+  // whole selection).  Measured: 16 rows of 32768 (the HS anchor's two
+  // budgets over 8 sequences) took 30.7 us with the anchor scan at 4 keys a
+  // thread (8-CTA clusters, more than are resident at once) against 25.3 us
+  // at 16 (4-CTA clusters).  Many rows fill the GPU many times over: 32 keys
+  // a thread means fewer CTAs, each paying the per-pass overhead once for
+  // more keys (1024 x 65536: 467 us at 32 keys a thread against 788 us at 4).
+  for (int kpt = kTopkKeysLatency; kpt <= 16; kpt *= 2) {
+    const int cs = topk_cluster_size(n, kpt, rows);
+    if (cap[cs] >= rows) return kpt;
+  }
+  return kTopkKeysThroughput;
 }
 
 cudaError_t launch_topk_cluster(const TopkArgs& a, cudaStream_t st, int* cluster_size, int keys_per_thread) {
