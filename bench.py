@@ -75,7 +75,7 @@ def config_of(wl, paths="HS + DSA-style, with construction"):
                         f"H {wl.heads}, d_k {wl.d_k}, d_c {wl.d_c}, k {wl.k}, B {wl.B}, G {wl.group}",
             "batch": wl.batch, "ctx": wl.length_range[1], "cache": wl.cache_dtype, "heads": wl.heads,
             "d_k": wl.d_k, "d_c": wl.d_c, "k": wl.k, "B": wl.B, "group": wl.group, "d_model": wl.d_model,
-            "paths": paths, "l2": "flushed before every step (256 MiB write, outside the timed events)"}
+            "paths": paths, "l2": "flushed before each path of every step (256 MiB write, outside the timed events)"}
 
 
 # ------------------------------------------------------------------ CPU oracle leg
@@ -506,9 +506,11 @@ class Step:
 
 def timed_steps(step, steps, flush, stream, graphs):
     """Times `steps` group steps with CUDA events on the launching stream;
-    L2 is flushed (a 256 MiB write) before every step, outside the events.
-    Returns per-step (hs_ms, dsa_ms)."""
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    L2 is flushed (a 256 MiB write) before each path of every step, outside
+    the events, so that both paths start alike: from an L2 full of dirty
+    lines that their first reads must evict.  Returns per-step (hs_ms,
+    dsa_ms)."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for i in range(steps):
         flush.fill_(i & 0xFF)
         step.reset()
@@ -518,13 +520,15 @@ def timed_steps(step, steps, flush, stream, graphs):
         else:
             step.hs_path()
         ev[i][1].record(stream)
+        flush.fill_((i + 128) & 0xFF)
+        ev[i][2].record(stream)
         if graphs:
             graphs[1].replay()
         else:
             step.dsa_path()
-        ev[i][2].record(stream)
+        ev[i][3].record(stream)
     torch.cuda.synchronize()
-    return [e[0].elapsed_time(e[1]) for e in ev], [e[1].elapsed_time(e[2]) for e in ev]
+    return [e[0].elapsed_time(e[1]) for e in ev], [e[2].elapsed_time(e[3]) for e in ev]
 
 
 def profiled_steps(step, steps, flush, stream, lead_ms=4.0):
@@ -541,17 +545,22 @@ def profiled_steps(step, steps, flush, stream, lead_ms=4.0):
         flush.fill_(i & 0xFF)
         step.reset()
         torch.cuda._sleep(cycles)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         li.li_profile_enable(ctx, True)
         e[0].record(stream)
         step.hs_path()
         e[1].record(stream)
-        step.dsa_path()
+        li.li_profile_enable(ctx, False)
+        flush.fill_((i + 128) & 0xFF)
+        torch.cuda._sleep(cycles)
+        li.li_profile_enable(ctx, True)
         e[2].record(stream)
+        step.dsa_path()
+        e[3].record(stream)
         li.li_profile_enable(ctx, False)
         torch.cuda.synchronize()
         hs_ms.append(e[0].elapsed_time(e[1]))
-        dsa_ms.append(e[1].elapsed_time(e[2]))
+        dsa_ms.append(e[2].elapsed_time(e[3]))
         recs += li.li_profile_read(ctx)
         li.li_profile_reset(ctx)
     return recs, hs_ms, dsa_ms
