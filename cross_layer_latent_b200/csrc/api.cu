@@ -670,17 +670,22 @@ li_status li_create(li_ctx** out, int device) {
   }
   c->device = device;
   {
-    // the occupancy queries read the current device: select ours for them
+    // The occupancy queries read the current device: select ours for them.
+    // A cluster size whose query fails counts as never resident, so the
+    // selection sizes around it (the throughput form needs no residency).
     int prev = 0;
     e = cudaGetDevice(&prev);
     if (e == cudaSuccess) e = cudaSetDevice(device);
-    for (int cs = 1; cs <= 16 && e == cudaSuccess; ++cs) {
-      c->cluster_cap[cs] = topk_cluster_capacity(cs, c->num_sms);
-      if (c->cluster_cap[cs] < 0) e = cudaErrorInvalidValue;
-    }
-    const cudaError_t e2 = cudaSetDevice(prev);
-    if (e == cudaSuccess) e = e2;
     if (e != cudaSuccess) {
+      delete c;
+      return LI_ERR_CUDA;
+    }
+    for (int cs = 1; cs <= 16; ++cs) {
+      const int cap = topk_cluster_capacity(cs, c->num_sms);
+      c->cluster_cap[cs] = cap > 0 ? cap : 0;
+    }
+    (void)cudaGetLastError();   // a failed query leaves no sticky error behind
+    if (cudaSetDevice(prev) != cudaSuccess) {
       delete c;
       return LI_ERR_CUDA;
     }
