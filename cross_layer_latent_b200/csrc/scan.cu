@@ -179,6 +179,29 @@ __device__ __forceinline__ void relu_dot16(const float* v, const float* wq, floa
   }
 }
 
+// c0 += a0 * b0 and c1 += a1 * b1 as one paired fp32 FMA (sm_100's
+// fma.rn.f32x2): each lane is an IEEE fma, so the results equal two fmaf.
+__device__ __forceinline__ void ffma2(float& c0, float& c1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// relu_dot16 with paired FMAs (same arithmetic, same order): the epilogue of
+// several query rows per item is bound by its arithmetic and tensor-memory
+// loads, and this takes 4% off the prefill scan; the decode epilogue is not
+// bound by it and keeps the scalar form.
+__device__ __forceinline__ void relu_dot16_pk(const float* v, const float* wq, float (&acc)[4]) {
+#pragma unroll
+  for (int e = 0; e < 16; e += 4) {
+    const float4 w4 = *reinterpret_cast<const float4*>(wq + e);
+    ffma2(acc[0], acc[1], w4.x, w4.y, fmaxf(v[e], 0.f), fmaxf(v[e + 1], 0.f));
+    ffma2(acc[2], acc[3], w4.z, w4.w, fmaxf(v[e + 2], 0.f), fmaxf(v[e + 3], 0.f));
+  }
+}
+
 __device__ __forceinline__ void relu_dot16_beta(const float* v, const float* w, const float* qs,
                                                 const float* be, float cs, float (&acc)[4]) {
 #pragma unroll
@@ -787,7 +810,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(const __grid_cons
         const float* be = ep_beta + qi * k_H_pad;
 #pragma unroll
         for (int h0 = 0; h0 < HP; h0 += 16) {
-          if (!has_beta) relu_dot16(vq + h0, wq + h0, part);
+          if (!has_beta) relu_dot16_pk(vq + h0, wq + h0, part);
           else relu_dot16_beta(vq + h0, wq + h0, qs + h0, be + h0, cs, part);
         }
         float sc = (part[0] + part[1]) + (part[2] + part[3]);
